@@ -1,0 +1,443 @@
+#!/usr/bin/env python
+"""Benchmark of the speculative flash-decode step on synthetic caches.
+
+One step = one decode token through the 32 layers of a Llama-3.1-8B-shaped
+model at 131072 context (batch 1, 32 query / 8 KV heads, d 128, bf16 KV
+cache, sink 4, window 1024, lambda 0.10): per layer the sink-set kernel (on a
+high-priority stream), the split exact-attention kernel and the merge +
+relative-L2 + flag kernel, all captured in one CUDA graph.  Layers are
+independent caches generated from the seed; inputs are resident in HBM.
+
+Output: one JSON line on rank 0 (see the keys at the end of main()).
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl alspec|reference]
+With --impl reference the fp64 CPU oracle is timed on the host cores on a
+bounded sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "KV GB/s (fraction of HBM peak) and µs/decode-step to commit flag at 128K"
+FALLBACK_HBM_GBS = 6650.0
+MID_KERNEL_SRC = os.path.join(ROOT, "speculative_flash_decoding_b200", "csrc", "attn_kernels.cuh")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_mid_llama8b_128k_traffic.md")
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["alspec", "reference"], default="alspec")
+    ap.add_argument("--config", type=int, default=2, help="workload index (2 = 32 layers @128K)")
+    ap.add_argument("--layers", type=int, default=0, help="override the layer count (0 = workload's)")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="CPU-baseline budget (oracle time) on rank 0")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
+            int(os.environ.get("LOCAL_RANK", 0)))
+
+
+# ------------------------------------------------------------------ helpers
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            val = float(json.load(f)["hbm_gbs"])
+        return val, "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def stored_traffic():
+    """DRAM bytes per launch of the middle kernel from the committed ncu summary,
+    or None when the kernel source changed since it was captured."""
+    try:
+        text = open(TRAFFIC_FILE).read()
+    except OSError:
+        return None
+    m_hash = re.search(r"source_sha256:\s*([0-9a-f]{64})", text)
+    m_bytes = re.search(r"dram_bytes_per_launch:\s*([0-9]+)", text)
+    if not (m_hash and m_bytes):
+        return None
+    src = hashlib.sha256(open(MID_KERNEL_SRC, "rb").read()).hexdigest()
+    return int(m_bytes.group(1)) if src == m_hash.group(1) else None
+
+
+class ClockSampler:
+    """nvidia-smi samples of the SM clock and throttle reasons while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, uuid):
+        self.uuid = uuid
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def __enter__(self):
+        cmd = ["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+               "-lms", "100"]
+        if self.uuid:
+            cmd += ["-i", self.uuid]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            if self.thread:
+                self.thread.join(timeout=5)
+
+    def summary(self):
+        mhz, mx, reasons = [], None, set()
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                mhz.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for name, val in zip(self.NAMES, parts[3:7]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not mhz:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(mhz)}
+
+
+# ------------------------------------------------------------ CPU oracle leg
+
+def oracle_layer_sample(wl, layer, heads_kv=None):
+    """Generate one layer on the CPU and return oracle inputs (optionally only
+    the first heads_kv KV heads and their query heads) and its KV bytes."""
+    import numpy as np
+    import workloads
+    data = workloads.make_layer(wl, layer=layer, device="cpu")
+    q, k, v = data["q"], data["k"], data["v"]
+    if heads_kv is not None:
+        q = q[:, : heads_kv * wl.g].contiguous()
+        k = k[:, :heads_kv].contiguous()
+        v = v[:, :heads_kv].contiguous()
+    nkv = k.shape[1]
+    lens = np.array(data["lens"], np.int32)
+    bytes_ = int(sum(data["lens"]) * nkv * wl.d * 2 * wl.elem_bytes)
+    return (workloads.to_numpy_bits(q), workloads.to_numpy_bits(k), workloads.to_numpy_bits(v),
+            lens), bytes_
+
+
+def cpu_baseline(wl, budget_s):
+    """Time the oracle as it stands on whole layers until ~budget_s of oracle time."""
+    import oracle
+    total_bytes, total_t, layers, threads = 0, 0.0, 0, 0
+    for layer in range(wl.n_layers):
+        (q, k, v, lens), nbytes = oracle_layer_sample(wl, layer)
+        t0 = time.perf_counter()
+        res = oracle.decode(q, k, v, lens, wl.S, wl.W, wl.lam)
+        total_t += time.perf_counter() - t0
+        total_bytes += nbytes
+        threads = res["threads"]
+        layers += 1
+        if total_t >= budget_s:
+            break
+    return {"value": total_bytes / total_t / 1e9, "unit": "GB/s", "cores": threads,
+            "kind": "oracle",
+            "sample": f"{layers} of {wl.n_layers} layers of the {wl.name} step (full cache, all "
+                      f"heads), fp64 C oracle with OpenMP; {total_t:.1f} s oracle time",
+            "us_per_step": total_t / layers * wl.n_layers * 1e6}
+
+
+def run_reference(args, wl):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    import oracle
+    # Each step: one 128K layer of the workload, its first 2 of 8 KV heads
+    # (8 of 32 query heads), generated once outside the timed region.
+    (q, k, v, lens), nbytes = oracle_layer_sample(wl, 0, heads_kv=2)
+    for _ in range(args.warmup):
+        oracle.decode(q, k, v, lens, wl.S, wl.W, wl.lam)
+    times, threads = [], 0
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        res = oracle.decode(q, k, v, lens, wl.S, wl.W, wl.lam)
+        times.append(time.perf_counter() - t0)
+        threads = res["threads"]
+    t = sum(times) / len(times)
+    value = nbytes / t / 1e9
+    sample = (f"per step: layer 0 of {wl.name}, KV heads 0-1 with their 8 query heads "
+              f"({nbytes / 1e6:.0f} MB of KV), fp64 C oracle with OpenMP")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": t * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "context": wl.L, "sink": wl.S, "window": wl.W,
+                       "lambda": wl.lam, "sample": sample},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- GPU leg
+
+def run_alspec(args, wl):
+    import torch
+    import workloads
+    import speculative_flash_decoding_b200 as sfd
+
+    rank, world, local = dist_env()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+        pg = dist
+
+    n_layers = args.layers or wl.n_layers
+    layers = [workloads.make_layer(wl, layer=i, device=device) for i in range(n_layers)]
+    q_all = torch.stack([d["q"] for d in layers]).contiguous()      # [layers, B, Hq, d]
+    lens_all = torch.stack([d["seq_lens"] for d in layers]).contiguous()  # [layers, B]
+    for i, d in enumerate(layers):
+        d["q"] = q_all[i]
+        d["seq_lens"] = lens_all[i]
+    kv_bytes = sum(workloads.kv_bytes(wl, d["lens"]) for d in layers)
+    dec = sfd.Decoder(wl.B, wl.Hq, wl.Hkv, wl.d, wl.L, wl.dtype, wl.S, wl.W, device=device)
+    plan = dec.plan()
+    out_spec = torch.empty(n_layers, wl.B, wl.Hq, wl.d, dtype=torch.float32, device=device)
+    out_exact = torch.empty_like(out_spec)
+    rel_all = torch.empty(n_layers, wl.B, dtype=torch.float32, device=device)
+    commit_all = torch.empty(n_layers, wl.B, dtype=torch.uint8, device=device)
+    outs = [dict(out_spec=out_spec[i], out_exact=out_exact[i], rel_l2=rel_all[i],
+                 commit=commit_all[i]) for i in range(n_layers)]
+    stream = torch.cuda.Stream(device)
+
+    def new_events():
+        evs = [[torch.cuda.Event(enable_timing=True, external=True)
+                for _ in range(sfd.ALSPEC_PROF_EVENTS)] for _ in range(n_layers)]
+        for row in evs:      # torch creates the CUDA event at its first record
+            for e in row:
+                e.record(stream)
+        return evs
+
+    def capture(events):
+        with torch.cuda.stream(stream):
+            st = sfd.alspec_graph_begin(stream.cuda_stream)
+            assert st == 0, sfd.alspec_status_string(st)
+            for i, d in enumerate(layers):
+                dec.decode(d["q"], d["k"], d["v"], d["seq_lens"], wl.lam, out=outs[i],
+                           stream=stream, prof_events=events[i])
+            st, g = sfd.alspec_graph_end(stream.cuda_stream)
+            assert st == 0, sfd.alspec_status_string(st)
+        return g
+
+    # First call outside capture creates the library's stream and events.
+    with torch.cuda.stream(stream):
+        for i, d in enumerate(layers):
+            dec.decode(d["q"], d["k"], d["v"], d["seq_lens"], wl.lam, out=outs[i], stream=stream)
+    stream.synchronize()
+
+    warm_events = new_events()
+    warm_graph = capture(warm_events)
+    step_events = [new_events() for _ in range(args.steps)]
+    graphs = [capture(ev) for ev in step_events]
+
+    def barrier():
+        torch.cuda.synchronize(device)
+        if pg:
+            pg.barrier()
+
+    for _ in range(args.warmup):
+        sfd.alspec_graph_launch(warm_graph, stream.cuda_stream)
+    barrier()
+
+    uuid = None
+    try:
+        uuid = str(torch.cuda.get_device_properties(device).uuid)
+        uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+    except Exception:
+        uuid = None
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    step_marks = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    with ClockSampler(uuid) as clocks:
+        barrier()
+        t_start.record(stream)
+        for i in range(args.steps):
+            step_marks[i].record(stream)
+            st = sfd.alspec_graph_launch(graphs[i], stream.cuda_stream)
+            assert st == 0
+        step_marks[args.steps].record(stream)
+        t_end.record(stream)
+        barrier()
+    ms_total = t_start.elapsed_time(t_end)
+    ms_per_step = ms_total / args.steps
+    if pg:
+        t = torch.tensor([ms_per_step], device=device)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ms_per_step = float(t.item())
+    per_step = [step_marks[i].elapsed_time(step_marks[i + 1]) for i in range(args.steps)]
+
+    # Per-layer profiling events of every timed step.
+    mid_ms, spec_ms, layer_ms = [], [], []
+    for ev in step_events:
+        for e in ev:
+            mid_ms.append(e[2].elapsed_time(e[3]))
+            spec_ms.append(e[0].elapsed_time(e[1]))
+            layer_ms.append(e[0].elapsed_time(e[4]))
+    hit_rate = float(commit_all.float().mean().item())
+    st, err = dec.device_error(stream)
+    assert st == 0 and err == 0, f"device error word {err:#x}"
+
+    # End-to-end through the public API with host buffers: per step, copy the
+    # step's query vectors (all layers) and lengths in from pinned memory,
+    # replay the step, read every layer's rel_l2 and flag back.
+    e2e = None
+    if not args.no_e2e:
+        q_host = q_all.cpu().pin_memory()
+        lens_host = lens_all.cpu().pin_memory()
+        rel_host = torch.empty(rel_all.shape, dtype=rel_all.dtype).pin_memory()
+        com_host = torch.empty(commit_all.shape, dtype=commit_all.dtype).pin_memory()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        barrier()
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for i in range(args.steps):
+                q_all.copy_(q_host, non_blocking=True)
+                lens_all.copy_(lens_host, non_blocking=True)
+                sfd.alspec_graph_launch(graphs[i], stream.cuda_stream)
+                rel_host.copy_(rel_all, non_blocking=True)
+                com_host.copy_(commit_all, non_blocking=True)
+                stream.synchronize()
+            e1.record(stream)
+        barrier()
+        e2e_ms = e0.elapsed_time(e1) / args.steps
+        if pg:
+            t = torch.tensor([e2e_ms], device=device)
+            pg.all_reduce(t, op=pg.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        h2d = q_host.numel() * q_host.element_size() + lens_host.numel() * lens_host.element_size()
+        d2h = rel_host.numel() * rel_host.element_size() + com_host.numel() * com_host.element_size()
+        e2e = {"value": kv_bytes * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+               "us_per_step": e2e_ms * 1e3, "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(d2h)}
+
+    for g in [warm_graph] + graphs:
+        sfd.alspec_graph_destroy(g)
+    if pg:
+        pg.destroy_process_group()
+    if rank != 0:
+        return
+
+    peak, peak_kind = measured_peak()
+    mid_bytes = sum(
+        (max(0, L - wl.W - min(wl.S, L)) if L > wl.S + wl.W else 0) * wl.Hkv * wl.d * 2 *
+        wl.elem_bytes for L in layers[0]["lens"])
+    mid_avg_ms = sum(mid_ms) / len(mid_ms)
+    achieved = mid_bytes / (mid_avg_ms * 1e-3) / 1e9
+    traffic = stored_traffic()
+    value = kv_bytes * world / (ms_per_step * 1e-3) / 1e9
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl.replace(n_layers=n_layers), args.cpu_seconds)
+
+    spec_ratio = [s / l for s, l in zip(spec_ms, layer_ms)]
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_per_step,
+        "us_per_step": ms_per_step * 1e3,
+        "us_per_step_p10_p50_p90": [float(x * 1e3) for x in
+                                    statistics.quantiles(per_step, n=10)[::4]]
+        if len(per_step) >= 2 else None,
+        "frac_of_hbm_peak": value / world / peak,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": wl.dtype,
+        "data": "synthetic",
+        "config": {"workload": wl.name, "layers": n_layers, "batch": wl.B, "q_heads": wl.Hq,
+                   "kv_heads": wl.Hkv, "head_dim": wl.d, "context": wl.L, "sink": wl.S,
+                   "window": wl.W, "lambda": wl.lam, "kv_bytes_per_step": kv_bytes,
+                   "l2": "inputs larger than L2: 537 MB of KV per layer, 17.2 GB per step; no flush",
+                   "parallelism": "replicas" if world > 1 else "single",
+                   "timing": "CUDA graph per step, CUDA events on the launch stream",
+                   "plan": plan},
+        "roofline": {"bound": "hbm", "kernel": "attn_kernel<bf16,128,4,mid>",
+                     "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_kind": peak_kind,
+                     "bytes_per_launch": mid_bytes, "avg_launch_us": mid_avg_ms * 1e3,
+                     "launches_measured": len(mid_ms), "traffic": traffic},
+        "spec_latency": {"us_median": statistics.median(spec_ms) * 1e3,
+                         "ratio_to_layer_median": statistics.median(spec_ratio),
+                         "layer_us_median": statistics.median(layer_ms) * 1e3},
+        "hit_rate": hit_rate,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": args.steps * n_layers * (3 if plan["n2"] > 0 else 2),
+        "clocks": clocks.summary(),
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    import workloads
+    wl = workloads.CONFIGS[args.config]
+    if args.impl == "reference":
+        run_reference(args, wl)
+    else:
+        run_alspec(args, wl)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,194 @@
+/*
+ * alspec.h -- C ABI of the speculative flash-decode library (libalspec.so).
+ *
+ * The operation (Attention-Level Speculation, ICML 2025; atlas.scime.ai
+ * summary, one-line summary and "Approach"; ICML 2025 poster page,
+ * abstract): for each decode query, the library computes
+ *   - O_spec : softmax attention over the "attention sink", i.e. the first
+ *              n_sink tokens plus the last `window` tokens of the cache
+ *              (a set union, each token once), published early;
+ *   - O_exact: softmax attention over every cached token (flash decoding,
+ *              the method the summary lists under "Builds on");
+ *   - rel_l2 : ||O_exact - O_spec||_2 / ||O_exact||_2 per decode token, over
+ *              all n_q_heads * head_dim outputs of that token's attention op;
+ *   - commit : 1 when rel_l2 <= lambda (the approximation is kept), else 0
+ *              (it is discarded and the exact output is used).
+ * The softmax scale is 1/sqrt(head_dim).  Query head h reads KV head
+ * h / (n_q_heads / n_kv_heads) (grouped-query attention).
+ *
+ * Conventions for every entry point:
+ *   - Pointers named "device" are CUDA device pointers; "host" pointers are
+ *     ordinary host memory.  The caller owns every buffer.  The library never
+ *     allocates device memory in alspec_decode; it owns only one
+ *     high-priority stream and two events per device, created on first use
+ *     and released by alspec_shutdown().
+ *   - Streams and events are passed as `void*` holding a cudaStream_t /
+ *     cudaEvent_t (NULL stream = the legacy default stream).
+ *   - Calls are asynchronous on the given stream unless stated otherwise;
+ *     no entry point except alspec_get_device_error synchronizes.
+ *   - Arguments that can be checked on the host are checked before anything
+ *     is launched; a failed check returns a status and launches nothing.
+ *     Nothing aborts, traps or exits.
+ */
+#ifndef ALSPEC_H
+#define ALSPEC_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    ALSPEC_OK = 0,
+    ALSPEC_ERR_INVALID_ARG = 1,  /* bad pointer, shape, alignment or value   */
+    ALSPEC_ERR_UNSUPPORTED = 2,  /* valid but not built: head_dim, group size */
+    ALSPEC_ERR_WORKSPACE = 3,    /* workspace missing or too small            */
+    ALSPEC_ERR_CUDA = 4,         /* a CUDA runtime call failed                */
+    ALSPEC_ERR_TIMEOUT = 5,      /* reported by alspec_get_device_error only  */
+    ALSPEC_ERR_DEVICE_DATA = 6   /* reported by alspec_get_device_error only  */
+} alspec_status;
+
+typedef enum {
+    ALSPEC_F32 = 0,   /* IEEE binary32                       */
+    ALSPEC_BF16 = 1   /* bfloat16 (upper half of a binary32) */
+} alspec_dtype;
+
+/* Number of events alspec_decode's prof_events array holds. */
+#define ALSPEC_PROF_EVENTS 5
+
+/* Bits of the device error word (alspec_get_device_error). */
+#define ALSPEC_DEVERR_SEQ_LEN 0x1u   /* a seq_lens entry outside [1, max_seq_len]; it was clamped */
+#define ALSPEC_DEVERR_TIMEOUT 0x2u   /* a bounded wait inside a kernel gave up; outputs invalid   */
+
+/*
+ * Problem description.  Shapes (row-major, last index fastest):
+ *   q                    [batch, n_q_heads, head_dim]
+ *   k_cache, v_cache     [batch, n_kv_heads, max_seq_len, head_dim]
+ * q, k_cache and v_cache share `dtype`.  Supported: head_dim in {64, 128};
+ * n_q_heads / n_kv_heads in {1, 2, 4, 8}.
+ * split_tokens: tokens per work item of the exact-attention split
+ * (a multiple of 16); 0 lets the library choose from the GPU's SM count.
+ */
+typedef struct {
+    int batch;
+    int n_q_heads;
+    int n_kv_heads;
+    int head_dim;
+    int max_seq_len;
+    int dtype;          /* alspec_dtype */
+    int split_tokens;   /* 0 = automatic */
+    int timeout_ms;     /* bound on any in-kernel wait; 0 = 2000 ms */
+} alspec_desc;
+
+/*
+ * Bytes of device workspace alspec_decode needs for this description and
+ * sink set.  Host only, no CUDA call.  Returns 0 if the description is
+ * invalid or unsupported.
+ */
+size_t alspec_workspace_size(const alspec_desc* desc, int n_sink, int window);
+
+/*
+ * Zero a workspace before its first use (cudaMemsetAsync on `stream`).
+ * The kernels leave every counter in the workspace at zero when they finish,
+ * so a workspace needs this once, not per call.
+ */
+alspec_status alspec_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * One speculative decode-attention step (one layer, `batch` decode tokens).
+ *
+ *   desc        host; shapes as above
+ *   q           device [batch, n_q_heads, head_dim], 16-byte aligned
+ *   k_cache     device [batch, n_kv_heads, max_seq_len, head_dim], 16-byte aligned
+ *   v_cache     device, same shape and alignment as k_cache
+ *   seq_lens    device int32 [batch]; 1 <= L_b <= max_seq_len.  Sequence b
+ *               attends to cache rows [0, L_b).  Out-of-range entries are
+ *               clamped and flagged in the device error word.
+ *   n_sink      S >= 0 sink tokens; window W >= 0 recent tokens; S + W >= 1
+ *   lambda      relative-L2 threshold, finite and >= 0
+ *   out_spec    device fp32 [batch, n_q_heads, head_dim]: O_spec
+ *   out_exact   device fp32 [batch, n_q_heads, head_dim]: O_exact
+ *   rel_l2      device fp32 [batch]
+ *   commit      device uint8 [batch]: 1 commit, 0 discard
+ *   workspace   device, >= alspec_workspace_size() bytes, zeroed once by
+ *               alspec_workspace_init; one call at a time per workspace
+ *   stream      the caller's stream; everything is ordered on it
+ *   spec_event  optional cudaEvent_t (NULL for none).  It is recorded as
+ *               soon as out_spec is complete, before the exact path ends,
+ *               so a consumer may start work on O_spec early by waiting on
+ *               it.  out_exact, rel_l2 and commit are complete when
+ *               `stream` reaches the point of this call.
+ *   prof_events optional array of ALSPEC_PROF_EVENTS timing-enabled
+ *               cudaEvent_t (NULL for none), recorded with
+ *               cudaEventRecordExternal so that they become event nodes when
+ *               the call is captured in a graph:
+ *                 [0] on `stream` when the call starts,
+ *                 [1] on the high-priority stream when O_spec is complete,
+ *                 [2] on `stream` before the exact-path (middle) kernel,
+ *                 [3] on `stream` after it,
+ *                 [4] on `stream` when the call's work is complete.
+ *               [1]-[0] is the latency of O_spec, [3]-[2] the duration of
+ *               the middle kernel, [4]-[0] the latency of the whole step.
+ *
+ * The sink-set attention runs on a high-priority stream forked from
+ * `stream` with events; the rest runs on `stream`.  Safe to capture in a
+ * CUDA graph (no host synchronization, no allocation).  With
+ * L_b <= S + W the two outputs are bit-identical and rel_l2 is exactly 0.
+ */
+alspec_status alspec_decode(const alspec_desc* desc,
+                            const void* q, const void* k_cache, const void* v_cache,
+                            const int32_t* seq_lens, int n_sink, int window,
+                            float lambda, float* out_spec, float* out_exact,
+                            float* rel_l2, uint8_t* commit,
+                            void* workspace, size_t workspace_bytes,
+                            void* stream, void* spec_event, void* const* prof_events);
+
+/*
+ * Work plan the library would use (host only, no CUDA call except the SM
+ * count query).  info[] receives, in order:
+ *   0 tokens per sink-set work item      1 sink-set items per (b, kv head)
+ *   2 tokens per exact-path work item    3 exact-path items per (b, kv head)
+ *   4 persistent CTAs of the exact path  5 threads per CTA
+ *   6 dynamic shared memory per CTA      7 pipeline stages
+ * n_info is the capacity of info (8 fills all).
+ */
+alspec_status alspec_query_plan(const alspec_desc* desc, int n_sink, int window,
+                                int* info, int n_info);
+
+/*
+ * Read (and clear) the device error word of a workspace: a bitwise OR of
+ * ALSPEC_DEVERR_* raised by kernels since the last read.  Synchronizes
+ * `stream`.  *err receives the word; returns ALSPEC_OK, or
+ * ALSPEC_ERR_DEVICE_DATA / ALSPEC_ERR_TIMEOUT when the word is non-zero.
+ */
+alspec_status alspec_get_device_error(void* workspace, size_t workspace_bytes,
+                                      void* stream, uint32_t* err);
+
+/*
+ * Static-graph helpers (the single-GPU analogue of the pages' static-graph
+ * runtime with priority gating): capture a sequence of alspec_decode calls
+ * on `stream` into a CUDA graph whose sink-set kernels keep their high
+ * launch priority.  begin/end bracket the capture; launch replays it on a
+ * stream; destroy frees it.  *graph receives an opaque handle.
+ */
+alspec_status alspec_graph_begin(void* stream);
+alspec_status alspec_graph_end(void* stream, void** graph);
+alspec_status alspec_graph_launch(void* graph, void* stream);
+alspec_status alspec_graph_destroy(void* graph);
+
+/* Release the library's streams and events on every device it touched. */
+alspec_status alspec_shutdown(void);
+
+/* Human-readable name of a status (static string, never NULL). */
+const char* alspec_status_string(alspec_status status);
+
+/* Library ABI version: major * 10000 + minor * 100 + patch. */
+int alspec_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ALSPEC_H */

@@ -1,0 +1,229 @@
+"""ctypes binding of libalspec.so (the C ABI in include/alspec.h).
+
+Argument marshalling only: every step of the decode path runs in the CUDA
+kernels of libalspec.so.  There is no CPU fallback -- if the library is
+missing or cannot be loaded, importing this module raises.
+
+The functions named ``alspec_*`` mirror the C entry points one to one and
+take plain integers (device pointers, stream/event handles) and sizes.
+``Decoder`` is a convenience layer that takes torch tensors, owns a
+workspace and raises ``AlspecError`` on a non-OK status.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libalspec.so")
+
+ALSPEC_OK = 0
+ALSPEC_ERR_INVALID_ARG = 1
+ALSPEC_ERR_UNSUPPORTED = 2
+ALSPEC_ERR_WORKSPACE = 3
+ALSPEC_ERR_CUDA = 4
+ALSPEC_ERR_TIMEOUT = 5
+ALSPEC_ERR_DEVICE_DATA = 6
+
+ALSPEC_F32 = 0
+ALSPEC_BF16 = 1
+
+ALSPEC_PROF_EVENTS = 5
+
+ALSPEC_DEVERR_SEQ_LEN = 0x1
+ALSPEC_DEVERR_TIMEOUT = 0x2
+
+# Every symbol the header declares, with (restype, argtypes).
+_vp, _i, _f, _sz, _u32p = (ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t,
+                          ctypes.POINTER(ctypes.c_uint32))
+
+
+class alspec_desc(ctypes.Structure):
+    _fields_ = [("batch", _i), ("n_q_heads", _i), ("n_kv_heads", _i), ("head_dim", _i),
+                ("max_seq_len", _i), ("dtype", _i), ("split_tokens", _i), ("timeout_ms", _i)]
+
+
+_descp = ctypes.POINTER(alspec_desc)
+
+SIGNATURES = {
+    "alspec_workspace_size": (_sz, [_descp, _i, _i]),
+    "alspec_workspace_init": (_i, [_vp, _sz, _vp]),
+    "alspec_decode": (_i, [_descp, _vp, _vp, _vp, _vp, _i, _i, _f, _vp, _vp, _vp, _vp, _vp, _sz,
+                           _vp, _vp, ctypes.POINTER(_vp)]),
+    "alspec_query_plan": (_i, [_descp, _i, _i, ctypes.POINTER(_i), _i]),
+    "alspec_get_device_error": (_i, [_vp, _sz, _vp, _u32p]),
+    "alspec_graph_begin": (_i, [_vp]),
+    "alspec_graph_end": (_i, [_vp, ctypes.POINTER(_vp)]),
+    "alspec_graph_launch": (_i, [_vp, _vp]),
+    "alspec_graph_destroy": (_i, [_vp]),
+    "alspec_shutdown": (_i, []),
+    "alspec_status_string": (ctypes.c_char_p, [_i]),
+    "alspec_version": (_i, []),
+}
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"libalspec.so not found at {LIB_PATH}; build it with "
+            "`python speculative_flash_decoding_b200/build.py` (there is no CPU fallback)")
+    lib = ctypes.CDLL(LIB_PATH)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+_lib = _load()
+
+
+class AlspecError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {alspec_status_string(status)} (status {status})")
+        self.status = status
+
+
+# ------------------------------------------------------------ C entry points
+
+def alspec_workspace_size(desc: alspec_desc, n_sink: int, window: int) -> int:
+    return int(_lib.alspec_workspace_size(ctypes.byref(desc), n_sink, window))
+
+
+def alspec_workspace_init(workspace: int, workspace_bytes: int, stream: int) -> int:
+    return int(_lib.alspec_workspace_init(workspace, workspace_bytes, stream))
+
+
+def alspec_decode(desc: alspec_desc, q: int, k_cache: int, v_cache: int, seq_lens: int,
+                  n_sink: int, window: int, lam: float, out_spec: int, out_exact: int,
+                  rel_l2: int, commit: int, workspace: int, workspace_bytes: int,
+                  stream: int, spec_event: int = 0, prof_events=None) -> int:
+    """prof_events: None or a sequence of ALSPEC_PROF_EVENTS event handles."""
+    prof = None
+    if prof_events is not None:
+        prof = (ctypes.c_void_p * ALSPEC_PROF_EVENTS)(*[e or None for e in prof_events])
+    return int(_lib.alspec_decode(ctypes.byref(desc), q, k_cache, v_cache, seq_lens, n_sink,
+                                  window, lam, out_spec, out_exact, rel_l2, commit, workspace,
+                                  workspace_bytes, stream, spec_event or None, prof))
+
+
+def alspec_query_plan(desc: alspec_desc, n_sink: int, window: int):
+    info = (ctypes.c_int * 8)()
+    st = int(_lib.alspec_query_plan(ctypes.byref(desc), n_sink, window, info, 8))
+    keys = ("c1", "n1", "c2", "n2", "grid2", "threads", "smem", "stages")
+    return st, dict(zip(keys, list(info)))
+
+
+def alspec_get_device_error(workspace: int, workspace_bytes: int, stream: int):
+    err = ctypes.c_uint32(0)
+    st = int(_lib.alspec_get_device_error(workspace, workspace_bytes, stream, ctypes.byref(err)))
+    return st, int(err.value)
+
+
+def alspec_graph_begin(stream: int) -> int:
+    return int(_lib.alspec_graph_begin(stream))
+
+
+def alspec_graph_end(stream: int):
+    g = ctypes.c_void_p(0)
+    st = int(_lib.alspec_graph_end(stream, ctypes.byref(g)))
+    return st, int(g.value or 0)
+
+
+def alspec_graph_launch(graph: int, stream: int) -> int:
+    return int(_lib.alspec_graph_launch(graph, stream))
+
+
+def alspec_graph_destroy(graph: int) -> int:
+    return int(_lib.alspec_graph_destroy(graph))
+
+
+def alspec_shutdown() -> int:
+    return int(_lib.alspec_shutdown())
+
+
+def alspec_status_string(status: int) -> str:
+    return _lib.alspec_status_string(int(status)).decode()
+
+
+def alspec_version() -> int:
+    return int(_lib.alspec_version())
+
+
+# ------------------------------------------------------------ torch layer
+
+def make_desc(batch, n_q_heads, n_kv_heads, head_dim, max_seq_len, dtype, split_tokens=0,
+              timeout_ms=0) -> alspec_desc:
+    code = {"bf16": ALSPEC_BF16, "f32": ALSPEC_F32}.get(dtype, dtype)
+    return alspec_desc(batch, n_q_heads, n_kv_heads, head_dim, max_seq_len, int(code),
+                       split_tokens, timeout_ms)
+
+
+def _check(status: int, where: str):
+    if status != ALSPEC_OK:
+        raise AlspecError(status, where)
+
+
+class Decoder:
+    """One decode-attention shape with its own device workspace.
+
+    ``decode`` takes device tensors (q [B, Hq, d], k/v [B, Hkv, Lmax, d] in
+    bf16 or fp32, seq_lens int32 [B]) and returns (or fills) out_spec,
+    out_exact (fp32 [B, Hq, d]), rel_l2 (fp32 [B]) and commit (uint8 [B]).
+    """
+
+    def __init__(self, batch, n_q_heads, n_kv_heads, head_dim, max_seq_len, dtype, n_sink,
+                 window, device=None, split_tokens=0, timeout_ms=0):
+        import torch
+        self.torch = torch
+        self.desc = make_desc(batch, n_q_heads, n_kv_heads, head_dim, max_seq_len, dtype,
+                              split_tokens, timeout_ms)
+        self.n_sink, self.window = int(n_sink), int(window)
+        nbytes = alspec_workspace_size(self.desc, self.n_sink, self.window)
+        if nbytes == 0:
+            raise AlspecError(ALSPEC_ERR_INVALID_ARG, "alspec_workspace_size")
+        self.device = torch.device(device) if device is not None else torch.device("cuda")
+        self.workspace = torch.zeros(nbytes, dtype=torch.uint8, device=self.device)
+        self.workspace_bytes = nbytes
+
+    def plan(self):
+        st, info = alspec_query_plan(self.desc, self.n_sink, self.window)
+        _check(st, "alspec_query_plan")
+        return info
+
+    def alloc_outputs(self):
+        t = self.torch
+        d = self.desc
+        kw = dict(device=self.device)
+        return dict(out_spec=t.empty(d.batch, d.n_q_heads, d.head_dim, dtype=t.float32, **kw),
+                    out_exact=t.empty(d.batch, d.n_q_heads, d.head_dim, dtype=t.float32, **kw),
+                    rel_l2=t.empty(d.batch, dtype=t.float32, **kw),
+                    commit=t.empty(d.batch, dtype=t.uint8, **kw))
+
+    def decode(self, q, k, v, seq_lens, lam, out=None, stream=None, spec_event=None,
+               prof_events=None):
+        """prof_events: None or ALSPEC_PROF_EVENTS torch.cuda.Event(enable_timing=True)."""
+        t = self.torch
+        out = out if out is not None else self.alloc_outputs()
+        s = stream if stream is not None else t.cuda.current_stream(self.device)
+        ev = spec_event.cuda_event if spec_event is not None else 0
+        prof = None
+        if prof_events is not None:
+            prof = [e.cuda_event for e in prof_events]
+        if (spec_event is not None and not ev) or (prof is not None and not all(prof)):
+            # torch creates the CUDA event lazily at its first record().
+            raise ValueError("event has no CUDA handle yet: record() it once before passing it")
+        st = alspec_decode(self.desc, q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                           seq_lens.data_ptr(), self.n_sink, self.window, float(lam),
+                           out["out_spec"].data_ptr(), out["out_exact"].data_ptr(),
+                           out["rel_l2"].data_ptr(), out["commit"].data_ptr(),
+                           self.workspace.data_ptr(), self.workspace_bytes, s.cuda_stream, ev,
+                           prof)
+        _check(st, "alspec_decode")
+        return out
+
+    def device_error(self, stream=None):
+        t = self.torch
+        s = stream if stream is not None else t.cuda.current_stream(self.device)
+        return alspec_get_device_error(self.workspace.data_ptr(), self.workspace_bytes,
+                                       s.cuda_stream)

@@ -1,0 +1,124 @@
+"""The C ABI: the library loads, exports every declared symbol, and rejects
+bad arguments on the host without launching anything (no GPU needed)."""
+import ctypes
+import math
+import os
+import re
+
+import pytest
+
+import speculative_flash_decoding_b200 as sfd
+from speculative_flash_decoding_b200 import alspec as ab
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include",
+                      "alspec.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(alspec_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_surface():
+    names = declared_functions()
+    assert "alspec_decode" in names and "alspec_workspace_size" in names
+    assert set(names) == set(ab.SIGNATURES), "binding and header disagree"
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(sfd.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), f"libalspec.so does not export {name}"
+
+
+def test_version_and_status_strings():
+    assert sfd.alspec_version() == 100
+    for st in range(7):
+        assert sfd.alspec_status_string(st) and "unknown" not in sfd.alspec_status_string(st)
+    assert "unknown" in sfd.alspec_status_string(99)
+
+
+DESC = dict(batch=1, n_q_heads=32, n_kv_heads=8, head_dim=128, max_seq_len=131072, dtype="bf16")
+
+
+def desc(**kw):
+    d = dict(DESC)
+    d.update(kw)
+    return sfd.make_desc(**d)
+
+
+def test_workspace_size_and_plan():
+    d = desc()
+    n = sfd.alspec_workspace_size(d, 4, 1024)
+    assert n > 0 and n % 256 == 0
+    st, plan = sfd.alspec_query_plan(d, 4, 1024)
+    assert st == 0
+    assert plan["c1"] % 16 == 0 and plan["c2"] % 16 == 0
+    assert plan["n1"] * plan["c1"] >= 1028 > (plan["n1"] - 1) * plan["c1"]
+    mid = 131072 - 4 - 1024
+    assert plan["n2"] * plan["c2"] >= mid > (plan["n2"] - 1) * plan["c2"]
+    assert 0 < plan["smem"] <= 227 * 1024 and plan["threads"] % 32 == 0
+    # A fixed split size is honoured (rounded to the 16-token tile).
+    st, plan = sfd.alspec_query_plan(desc(split_tokens=1000), 4, 1024)
+    assert st == 0 and plan["c2"] == 1008
+    # Whole cache inside the sink set: no middle items at all.
+    st, plan = sfd.alspec_query_plan(desc(max_seq_len=1000), 4, 1024)
+    assert st == 0 and plan["n2"] == 0
+
+
+@pytest.mark.parametrize("kw,S,W,code", [
+    (dict(n_q_heads=30), 4, 8, ab.ALSPEC_ERR_INVALID_ARG),      # Hq % Hkv != 0
+    (dict(head_dim=96), 4, 8, ab.ALSPEC_ERR_UNSUPPORTED),
+    (dict(n_q_heads=96, n_kv_heads=8), 4, 8, ab.ALSPEC_ERR_UNSUPPORTED),  # g = 12
+    (dict(batch=0), 4, 8, ab.ALSPEC_ERR_INVALID_ARG),
+    (dict(max_seq_len=0), 4, 8, ab.ALSPEC_ERR_INVALID_ARG),
+    (dict(dtype=7), 4, 8, ab.ALSPEC_ERR_INVALID_ARG),
+    (dict(), 0, 0, ab.ALSPEC_ERR_INVALID_ARG),                  # empty sink set
+    (dict(), -1, 8, ab.ALSPEC_ERR_INVALID_ARG),
+])
+def test_bad_descriptions(kw, S, W, code):
+    d = desc(**kw)
+    assert sfd.alspec_workspace_size(d, S, W) == 0
+    st, _ = sfd.alspec_query_plan(d, S, W)
+    assert st == code
+    # alspec_decode rejects it before touching any pointer.
+    fake = 1 << 20
+    st = sfd.alspec_decode(d, fake, fake, fake, fake, S, W, 0.1, fake, fake, fake, fake, fake,
+                           1 << 30, 0, 0, None)
+    assert st == code
+
+
+def _decode_with(**over):
+    d = desc(max_seq_len=4096)
+    fake = 1 << 20
+    args = dict(q=fake, k=fake, v=fake, seq=fake, S=4, W=64, lam=0.1, os_=fake, oe=fake, r=fake,
+                c=fake, ws=fake, wsb=sfd.alspec_workspace_size(d, 4, 64))
+    args.update(over)
+    return sfd.alspec_decode(d, args["q"], args["k"], args["v"], args["seq"], args["S"], args["W"],
+                             args["lam"], args["os_"], args["oe"], args["r"], args["c"], args["ws"],
+                             args["wsb"], 0)
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(q=0), ab.ALSPEC_ERR_INVALID_ARG),
+    (dict(k=0), ab.ALSPEC_ERR_INVALID_ARG),
+    (dict(seq=0), ab.ALSPEC_ERR_INVALID_ARG),
+    (dict(c=0), ab.ALSPEC_ERR_INVALID_ARG),
+    (dict(k=(1 << 20) + 8), ab.ALSPEC_ERR_INVALID_ARG),          # not 16-byte aligned
+    (dict(lam=-0.5), ab.ALSPEC_ERR_INVALID_ARG),
+    (dict(lam=math.nan), ab.ALSPEC_ERR_INVALID_ARG),
+    (dict(lam=math.inf), ab.ALSPEC_ERR_INVALID_ARG),
+    (dict(ws=0), ab.ALSPEC_ERR_WORKSPACE),
+    (dict(wsb=256), ab.ALSPEC_ERR_WORKSPACE),
+])
+def test_bad_arguments_return_codes(over, code):
+    assert _decode_with(**over) == code
+
+
+def test_null_handles():
+    assert sfd.alspec_graph_launch(0, 0) == ab.ALSPEC_ERR_INVALID_ARG
+    assert sfd.alspec_graph_destroy(0) == ab.ALSPEC_ERR_INVALID_ARG
+    assert sfd.alspec_workspace_init(0, 16, 0) == ab.ALSPEC_ERR_INVALID_ARG
+    st, err = sfd.alspec_get_device_error(0, 1024, 0)
+    assert st == ab.ALSPEC_ERR_INVALID_ARG

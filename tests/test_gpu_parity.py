@@ -1,0 +1,189 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle.
+
+Small cases span several 16-token tiles and a ragged tail so the oracle
+finishes in seconds; the full-size cases run in the launch configuration the
+benchmark times and compare the sequences the oracle can do in seconds.
+"""
+import numpy as np
+import pytest
+import torch
+
+import workloads
+from parity import assert_parity, gpu_decode, oracle_decode
+
+pytestmark = pytest.mark.gpu
+
+
+def _small(i):
+    wl = workloads.CONFIGS[i]
+    return {
+        0: wl,
+        1: wl.replace(L=8192 + 5),
+        2: wl.replace(L=16384 + 16),
+        3: wl.replace(L=9000, W=512, ragged=(2000, 9000)),
+        4: wl.replace(L=8192 + 7, W=1024),
+    }[i]
+
+
+@pytest.mark.parametrize("cfg", [0, 1, 2, 3, 4])
+def test_small_configs(cuda_device, cfg):
+    wl = _small(cfg)
+    for layer in range(3 if cfg == 2 else 1):
+        data = workloads.make_layer(wl, layer=layer, device=cuda_device, poison_tail=True)
+        dec, out = gpu_decode(wl, data, cuda_device)
+        ref = oracle_decode(wl, data)
+        assert_parity(out, ref, wl.lam, what=f"cfg{cfg} layer{layer}")
+        st, err = dec.device_error()
+        assert st == 0 and err == 0
+
+
+def test_commit_variant_gives_both_flags(cuda_device):
+    wl = workloads.COMMIT_VARIANT.replace(B=8, L=8192, ragged=(6000, 8192))
+    data = workloads.make_layer(wl, device=cuda_device)
+    _, out = gpu_decode(wl, data, cuda_device)
+    ref = oracle_decode(wl, data)
+    assert_parity(out, ref, wl.lam, what="commit variant")
+    assert 0 < ref["commit"].sum() < wl.B, "variant should mix commit and discard"
+
+
+EDGE = []
+for dtype, d in (("f32", 64), ("bf16", 64), ("bf16", 128), ("f32", 128)):
+    for g in (1, 2, 4, 8):
+        EDGE.append((dtype, d, g))
+
+
+@pytest.mark.parametrize("dtype,d,g", EDGE)
+def test_edge_lengths(cuda_device, dtype, d, g):
+    """L = 1, L < S, L = S + W, L = S + W + 1, W = 0, S = 0, ragged tails."""
+    Hkv = 2
+    for S, W in ((4, 16), (0, 16), (4, 0), (1, 1)):
+        lens = sorted({1, 3, S + W, S + W + 1, 37, 250, 16 * 9 + 5})
+        lens = [L for L in lens if L >= 1]
+        wl = workloads.Workload("edge", B=len(lens), Hq=g * Hkv, Hkv=Hkv, d=d, L=max(lens), S=S,
+                                W=W, lam=0.3, dtype=dtype, seed=777 + g + d)
+        data = workloads.make_layer(wl, device=cuda_device)
+        data["lens"] = lens
+        data["seq_lens"] = torch.tensor(lens, dtype=torch.int32, device=cuda_device)
+        _, out = gpu_decode(wl, data, cuda_device)
+        ref = oracle_decode(wl, data)
+        assert_parity(out, ref, wl.lam, what=f"{dtype} d{d} g{g} S{S} W{W}")
+        for b, L in enumerate(lens):
+            if L <= S + W:
+                assert torch.equal(out["out_spec"][b], out["out_exact"][b])
+                assert out["rel_l2"][b].item() == 0.0 and out["commit"][b].item() == 1
+
+
+def test_deterministic_and_reusable_workspace(cuda_device):
+    wl = _small(1)
+    data = workloads.make_layer(wl, device=cuda_device)
+    dec, a = gpu_decode(wl, data, cuda_device)
+    for _ in range(3):
+        _, b = gpu_decode(wl, data, cuda_device, dec=dec)
+        for k in a:
+            assert torch.equal(a[k], b[k]), k
+
+
+def test_split_sizes_agree(cuda_device):
+    """Different item sizes change only the fp32 summation order."""
+    wl = _small(3)
+    data = workloads.make_layer(wl, device=cuda_device)
+    ref = oracle_decode(wl, data)
+    for split in (16, 112, 1024, 100000):
+        _, out = gpu_decode(wl, data, cuda_device, split_tokens=split)
+        assert_parity(out, ref, wl.lam, what=f"split {split}")
+
+
+def test_bad_seq_lens_are_clamped_and_flagged(cuda_device):
+    wl = _small(1).replace(B=3, L=600, W=64)
+    data = workloads.make_layer(wl, device=cuda_device)
+    data["seq_lens"] = torch.tensor([0, 600, 9999], dtype=torch.int32, device=cuda_device)
+    dec, out = gpu_decode(wl, data, cuda_device)
+    st, err = dec.device_error()
+    assert err & 1 and st != 0
+    ref = oracle_decode(wl, data, lens=[1, 600, 600])
+    assert_parity(out, ref, wl.lam, what="clamped")
+    st, err = dec.device_error()
+    assert st == 0 and err == 0  # reading clears the word
+
+
+def test_spec_event_marks_o_spec_complete(cuda_device):
+    wl = _small(1)
+    data = workloads.make_layer(wl, device=cuda_device)
+    from speculative_flash_decoding_b200 import Decoder
+    dec = Decoder(wl.B, wl.Hq, wl.Hkv, wl.d, wl.L, wl.dtype, wl.S, wl.W, device=cuda_device)
+    ev = torch.cuda.Event()
+    ev.record()  # creates the CUDA event
+    out = dec.decode(data["q"], data["k"], data["v"], data["seq_lens"], wl.lam, spec_event=ev)
+    ev.synchronize()
+    spec_at_event = out["out_spec"].cpu()
+    torch.cuda.synchronize()
+    assert torch.equal(spec_at_event, out["out_spec"].cpu())
+    ref = oracle_decode(wl, data)
+    assert_parity({k: v.cpu() for k, v in out.items()}, ref, wl.lam, what="spec event")
+
+
+def test_graph_replay_matches_direct_calls(cuda_device):
+    import speculative_flash_decoding_b200 as sfd
+    wl = _small(2)
+    layers = [workloads.make_layer(wl, layer=i, device=cuda_device) for i in range(2)]
+    dec = sfd.Decoder(wl.B, wl.Hq, wl.Hkv, wl.d, wl.L, wl.dtype, wl.S, wl.W, device=cuda_device)
+    outs = [dec.alloc_outputs() for _ in layers]
+    direct = []
+    for data, o in zip(layers, outs):
+        dec.decode(data["q"], data["k"], data["v"], data["seq_lens"], wl.lam, out=o)
+        torch.cuda.synchronize()
+        direct.append({k: v.clone() for k, v in o.items()})
+        for v in o.values():
+            v.zero_()
+    stream = torch.cuda.Stream(cuda_device)
+    with torch.cuda.stream(stream):
+        assert sfd.alspec_graph_begin(stream.cuda_stream) == 0
+        for data, o in zip(layers, outs):
+            dec.decode(data["q"], data["k"], data["v"], data["seq_lens"], wl.lam, out=o,
+                       stream=stream)
+        st, graph = sfd.alspec_graph_end(stream.cuda_stream)
+        assert st == 0 and graph
+        for _ in range(2):
+            assert sfd.alspec_graph_launch(graph, stream.cuda_stream) == 0
+        stream.synchronize()
+        assert sfd.alspec_graph_destroy(graph) == 0
+    for d, o in zip(direct, outs):
+        for k in d:
+            assert torch.equal(d[k], o[k]), k
+
+
+# --------------------------------------------------------------- full size
+
+def test_full_size_128k_layer(cuda_device):
+    """A Llama-8B-shaped 128K layer, as timed by the benchmark."""
+    wl = workloads.CONFIGS[2]
+    data = workloads.make_layer(wl, layer=0, device=cuda_device)
+    _, out = gpu_decode(wl, data, cuda_device)
+    ref = oracle_decode(wl, data)
+    assert_parity(out, ref, wl.lam, what="cfg2 layer0 full")
+
+
+def test_full_size_32k_layer(cuda_device):
+    wl = workloads.CONFIGS[1]
+    data = workloads.make_layer(wl, device=cuda_device)
+    _, out = gpu_decode(wl, data, cuda_device)
+    assert_parity(out, oracle_decode(wl, data), wl.lam, what="cfg1 full")
+
+
+def test_full_size_ragged_batch(cuda_device):
+    wl = workloads.CONFIGS[3]
+    data = workloads.make_layer(wl, device=cuda_device, poison_tail=True)
+    _, out = gpu_decode(wl, data, cuda_device)
+    lens = np.array(data["lens"])
+    pick = [int(lens.argmin()), int(lens.argmax())]
+    ref = oracle_decode(wl, data, batch=pick)
+    assert_parity(out, ref, wl.lam, batch=pick, what="cfg3 full")
+    assert torch.isfinite(out["out_exact"]).all()
+
+
+def test_full_size_70b_layer(cuda_device):
+    wl = workloads.CONFIGS[4]
+    data = workloads.make_layer(wl, device=cuda_device)
+    _, out = gpu_decode(wl, data, cuda_device)
+    ref = oracle_decode(wl, data, batch=[0])
+    assert_parity(out, ref, wl.lam, batch=[0], what="cfg4 full b0")
