@@ -38,7 +38,7 @@ TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_mid_llama8b_128k_traffic.md"
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["alspec", "reference"], default="alspec")
     ap.add_argument("--config", type=int, default=2, help="workload index (2 = 32 layers @128K)")
@@ -98,7 +98,7 @@ class ClockSampler:
 
     def __enter__(self):
         cmd = ["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
-               "-lms", "100"]
+               "-lms", "20"]
         if self.uuid:
             cmd += ["-i", self.uuid]
         try:
@@ -412,7 +412,10 @@ def run_alspec(args, wl):
                    "parallelism": "replicas" if world > 1 else "single",
                    "timing": "CUDA graph per step, CUDA events on the launch stream",
                    "plan": plan},
-        "roofline": {"bound": "hbm", "kernel": "attn_kernel<bf16,128,4,mid>",
+        "roofline": {"bound": "hbm",
+                     "kernel": "attn_kernel<%s,%d,%d,middle,%s>" % (
+                         wl.dtype, wl.d, wl.g,
+                         {1: "cuda_cores", 2: "tensor_cores"}.get(plan["engine"], "?")),
                      "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_kind": peak_kind,
                      "bytes_per_launch": mid_bytes, "avg_launch_us": mid_avg_ms * 1e3,

@@ -55,6 +55,13 @@ typedef enum {
     ALSPEC_BF16 = 1   /* bfloat16 (upper half of a binary32) */
 } alspec_dtype;
 
+/* Compute engine of the attention kernels (alspec_desc.engine). */
+typedef enum {
+    ALSPEC_ENGINE_AUTO = 0,          /* tensor cores for bf16, CUDA cores for fp32 */
+    ALSPEC_ENGINE_CUDA_CORES = 1,    /* packed fp32 FMAs; any dtype               */
+    ALSPEC_ENGINE_TENSOR_CORES = 2   /* bf16 m16n8k16 MMAs; bf16 only             */
+} alspec_engine;
+
 /* Number of events alspec_decode's prof_events array holds. */
 #define ALSPEC_PROF_EVENTS 5
 
@@ -68,8 +75,10 @@ typedef enum {
  *   k_cache, v_cache     [batch, n_kv_heads, max_seq_len, head_dim]
  * q, k_cache and v_cache share `dtype`.  Supported: head_dim in {64, 128};
  * n_q_heads / n_kv_heads in {1, 2, 4, 8}.
- * split_tokens: tokens per work item of the exact-attention split
- * (a multiple of 16); 0 lets the library choose from the GPU's SM count.
+ * batch * n_kv_heads * max_seq_len must stay below 2^31.
+ * split_tokens: tokens per work item of the exact-attention split (rounded
+ * up to the engine's tile, 16 or 32 tokens); 0 lets the library choose from
+ * the GPU's SM count.
  */
 typedef struct {
     int batch;
@@ -80,6 +89,7 @@ typedef struct {
     int dtype;          /* alspec_dtype */
     int split_tokens;   /* 0 = automatic */
     int timeout_ms;     /* bound on any in-kernel wait; 0 = 2000 ms */
+    int engine;         /* alspec_engine; 0 = automatic */
 } alspec_desc;
 
 /*
@@ -152,7 +162,9 @@ alspec_status alspec_decode(const alspec_desc* desc,
  *   2 tokens per exact-path work item    3 exact-path items per (b, kv head)
  *   4 persistent CTAs of the exact path  5 threads per CTA
  *   6 dynamic shared memory per CTA      7 pipeline stages
- * n_info is the capacity of info (8 fills all).
+ *   8 engine (alspec_engine, resolved)
+ * (entries 5-7 describe the exact-path kernel).  n_info is the capacity of
+ * info (9 fills all).
  */
 alspec_status alspec_query_plan(const alspec_desc* desc, int n_sink, int window,
                                 int* info, int n_info);
@@ -186,6 +198,13 @@ const char* alspec_status_string(alspec_status status);
 
 /* Library ABI version: major * 10000 + minor * 100 + patch. */
 int alspec_version(void);
+
+/*
+ * The cudaError_t of the most recent CUDA runtime call that failed inside
+ * this library on the calling thread (0 if none did); it explains an
+ * ALSPEC_ERR_CUDA status.
+ */
+int alspec_last_cuda_error(void);
 
 #ifdef __cplusplus
 }

@@ -38,9 +38,15 @@ _vp, _i, _f, _sz, _u32p = (ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes
                           ctypes.POINTER(ctypes.c_uint32))
 
 
+ALSPEC_ENGINE_AUTO = 0
+ALSPEC_ENGINE_CUDA_CORES = 1
+ALSPEC_ENGINE_TENSOR_CORES = 2
+
+
 class alspec_desc(ctypes.Structure):
     _fields_ = [("batch", _i), ("n_q_heads", _i), ("n_kv_heads", _i), ("head_dim", _i),
-                ("max_seq_len", _i), ("dtype", _i), ("split_tokens", _i), ("timeout_ms", _i)]
+                ("max_seq_len", _i), ("dtype", _i), ("split_tokens", _i), ("timeout_ms", _i),
+                ("engine", _i)]
 
 
 _descp = ctypes.POINTER(alspec_desc)
@@ -59,6 +65,7 @@ SIGNATURES = {
     "alspec_shutdown": (_i, []),
     "alspec_status_string": (ctypes.c_char_p, [_i]),
     "alspec_version": (_i, []),
+    "alspec_last_cuda_error": (_i, []),
 }
 
 
@@ -80,7 +87,10 @@ _lib = _load()
 
 class AlspecError(RuntimeError):
     def __init__(self, status: int, where: str):
-        super().__init__(f"{where}: {alspec_status_string(status)} (status {status})")
+        extra = ""
+        if status == ALSPEC_ERR_CUDA:
+            extra = f", cudaError {alspec_last_cuda_error()}"
+        super().__init__(f"{where}: {alspec_status_string(status)} (status {status}{extra})")
         self.status = status
 
 
@@ -108,9 +118,9 @@ def alspec_decode(desc: alspec_desc, q: int, k_cache: int, v_cache: int, seq_len
 
 
 def alspec_query_plan(desc: alspec_desc, n_sink: int, window: int):
-    info = (ctypes.c_int * 8)()
-    st = int(_lib.alspec_query_plan(ctypes.byref(desc), n_sink, window, info, 8))
-    keys = ("c1", "n1", "c2", "n2", "grid2", "threads", "smem", "stages")
+    info = (ctypes.c_int * 9)()
+    st = int(_lib.alspec_query_plan(ctypes.byref(desc), n_sink, window, info, 9))
+    keys = ("c1", "n1", "c2", "n2", "grid2", "threads", "smem", "stages", "engine")
     return st, dict(zip(keys, list(info)))
 
 
@@ -150,13 +160,22 @@ def alspec_version() -> int:
     return int(_lib.alspec_version())
 
 
+def alspec_last_cuda_error() -> int:
+    return int(_lib.alspec_last_cuda_error())
+
+
 # ------------------------------------------------------------ torch layer
 
+ENGINES = {"auto": ALSPEC_ENGINE_AUTO, "cuda_cores": ALSPEC_ENGINE_CUDA_CORES,
+           "tensor_cores": ALSPEC_ENGINE_TENSOR_CORES}
+
+
 def make_desc(batch, n_q_heads, n_kv_heads, head_dim, max_seq_len, dtype, split_tokens=0,
-              timeout_ms=0) -> alspec_desc:
+              timeout_ms=0, engine="auto") -> alspec_desc:
     code = {"bf16": ALSPEC_BF16, "f32": ALSPEC_F32}.get(dtype, dtype)
+    eng = ENGINES.get(engine, engine)
     return alspec_desc(batch, n_q_heads, n_kv_heads, head_dim, max_seq_len, int(code),
-                       split_tokens, timeout_ms)
+                       split_tokens, timeout_ms, int(eng))
 
 
 def _check(status: int, where: str):
@@ -173,11 +192,11 @@ class Decoder:
     """
 
     def __init__(self, batch, n_q_heads, n_kv_heads, head_dim, max_seq_len, dtype, n_sink,
-                 window, device=None, split_tokens=0, timeout_ms=0):
+                 window, device=None, split_tokens=0, timeout_ms=0, engine="auto"):
         import torch
         self.torch = torch
         self.desc = make_desc(batch, n_q_heads, n_kv_heads, head_dim, max_seq_len, dtype,
-                              split_tokens, timeout_ms)
+                              split_tokens, timeout_ms, engine)
         self.n_sink, self.window = int(n_sink), int(window)
         nbytes = alspec_workspace_size(self.desc, self.n_sink, self.window)
         if nbytes == 0:

@@ -1,6 +1,8 @@
 // Host side of libalspec.so: argument checks, work planning, workspace
 // layout, the fork/join onto a high-priority stream, kernel launches and the
 // C ABI declared in include/alspec.h.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -19,7 +21,27 @@ namespace alspec {
 namespace {
 
 constexpr int kMaxDevices = 64;
+constexpr int kMaxSpecItems = 32;  // sink-set items per (sequence, KV head)
 constexpr size_t kAlign = 256;
+
+thread_local cudaError_t t_last_error = cudaSuccess;
+
+// Remember the most recent failing CUDA call of this thread.
+bool ok(cudaError_t e) {
+    if (e != cudaSuccess) t_last_error = e;
+    return e == cudaSuccess;
+}
+
+// Record an event so that, under stream capture, it becomes an event node
+// whose timestamp is taken at replay; outside capture it is a plain record.
+cudaError_t record_event(cudaEvent_t ev, cudaStream_t s) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    const cudaError_t e = cudaStreamIsCapturing(s, &cs);
+    if (e != cudaSuccess) return e;
+    return cs == cudaStreamCaptureStatusActive
+               ? cudaEventRecordWithFlags(ev, s, cudaEventRecordExternal)
+               : cudaEventRecord(ev, s);
+}
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 int ceil_div(int a, int b) { return (a + b - 1) / b; }
@@ -42,16 +64,16 @@ DeviceState g_dev[kMaxDevices];
 
 alspec_status get_device_state(DeviceState** out) {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ALSPEC_ERR_CUDA;
+    if (!ok(cudaGetDevice(&dev)) || dev < 0 || dev >= kMaxDevices) return ALSPEC_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_mutex);
     DeviceState& d = g_dev[dev];
     if (!d.ready) {
         int lo = 0, hi = 0;
-        if (cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-            cudaDeviceGetStreamPriorityRange(&lo, &hi) != cudaSuccess ||
-            cudaStreamCreateWithPriority(&d.hi, cudaStreamNonBlocking, hi) != cudaSuccess ||
-            cudaEventCreateWithFlags(&d.fork, cudaEventDisableTiming) != cudaSuccess ||
-            cudaEventCreateWithFlags(&d.join, cudaEventDisableTiming) != cudaSuccess) {
+        if (!ok(cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev)) ||
+            !ok(cudaDeviceGetStreamPriorityRange(&lo, &hi)) ||
+            !ok(cudaStreamCreateWithPriority(&d.hi, cudaStreamNonBlocking, hi)) ||
+            !ok(cudaEventCreateWithFlags(&d.fork, cudaEventDisableTiming)) ||
+            !ok(cudaEventCreateWithFlags(&d.join, cudaEventDisableTiming))) {
             return ALSPEC_ERR_CUDA;
         }
         d.prio_hi = hi;
@@ -72,6 +94,8 @@ int sm_count_for_plan() {
 // ------------------------------------------------------------- planning
 
 struct Plan {
+    int engine;   // ALSPEC_ENGINE_CUDA_CORES or ALSPEC_ENGINE_TENSOR_CORES
+    int tt;       // tokens per pipeline tile of that engine
     int c1, n1, c2, n2;
     int grid2;
     int threads, smem, stages;
@@ -81,6 +105,12 @@ struct Plan {
 
 bool supported_g(int g) { return g == 1 || g == 2 || g == 4 || g == 8; }
 
+int resolve_engine(const alspec_desc* d) {
+    if (d->engine == ALSPEC_ENGINE_AUTO)
+        return d->dtype == ALSPEC_BF16 ? ALSPEC_ENGINE_TENSOR_CORES : ALSPEC_ENGINE_CUDA_CORES;
+    return d->engine;
+}
+
 alspec_status check_desc(const alspec_desc* d, int S, int W) {
     if (!d) return ALSPEC_ERR_INVALID_ARG;
     if (d->batch < 1 || d->n_q_heads < 1 || d->n_kv_heads < 1 || d->max_seq_len < 1 ||
@@ -88,46 +118,58 @@ alspec_status check_desc(const alspec_desc* d, int S, int W) {
         (long long)S + W < 1 || d->split_tokens < 0 || d->timeout_ms < 0)
         return ALSPEC_ERR_INVALID_ARG;
     if (d->dtype != ALSPEC_F32 && d->dtype != ALSPEC_BF16) return ALSPEC_ERR_INVALID_ARG;
+    if (d->engine < ALSPEC_ENGINE_AUTO || d->engine > ALSPEC_ENGINE_TENSOR_CORES)
+        return ALSPEC_ERR_INVALID_ARG;
     if (d->head_dim != 64 && d->head_dim != 128) return ALSPEC_ERR_UNSUPPORTED;
     if (!supported_g(d->n_q_heads / d->n_kv_heads)) return ALSPEC_ERR_UNSUPPORTED;
-    // Item indices and row offsets must fit their integer types.
-    const long long heads = (long long)d->batch * d->n_kv_heads;
-    if (heads * d->max_seq_len > (1ll << 40) || heads > (1 << 20)) return ALSPEC_ERR_UNSUPPORTED;
+    if (resolve_engine(d) == ALSPEC_ENGINE_TENSOR_CORES && d->dtype != ALSPEC_BF16)
+        return ALSPEC_ERR_UNSUPPORTED;
+    // Row indices (TMA coordinates, item arithmetic) are 32-bit.
+    const long long rows = (long long)d->batch * d->n_kv_heads * d->max_seq_len;
+    if (rows >= (1ll << 31) || (long long)d->batch * d->n_kv_heads > (1 << 20))
+        return ALSPEC_ERR_UNSUPPORTED;
     return ALSPEC_OK;
 }
 
-void kernel_shape(int dtype, int D, int G, int* threads, int* smem, int* stages);
+void kernel_shape(int dtype, int D, int G, int engine, int* threads, int* smem, int* stages);
 
-// Item sizes: the sink-set list (at most S + W tokens per head) is cut so
-// that all heads together give about one CTA per SM; the middle is cut so
-// that the persistent grid (one CTA per SM) gets a couple of items per CTA
-// for a single sequence and more for batches, whose lengths may differ.
+// Item sizes: the sink-set list (at most S + W tokens per head, tiled as a
+// sink run and a window run) is cut so that all heads together use about a
+// quarter of the SMs -- few, long CTAs keep the sink-set kernel's fixed costs
+// and its merge short while the middle kernel takes the rest of the GPU; the
+// middle is cut so that the persistent grid (one CTA per SM) gets a couple
+// of items per CTA for a single sequence and more for batches, whose
+// lengths may differ.  Item sizes are multiples of the engine's tile.
 void make_plan(const alspec_desc& d, int S, int W, int sms, Plan* pl) {
+    pl->engine = resolve_engine(&d);
+    const int TT = pl->engine == ALSPEC_ENGINE_TENSOR_CORES ? 32 : 16;
+    pl->tt = TT;
     const int heads = d.batch * d.n_kv_heads;
     const int L = d.max_seq_len;
-    const int nspec_max = std::min<long long>((long long)S + W, L);
-    const int per_head1 = std::max(1, sms / std::max(1, heads));
-    pl->c1 = round_up(std::max(1, ceil_div(nspec_max, per_head1)), kTile);
-    pl->n1 = ceil_div(nspec_max, pl->c1);
+    const int tiles_max = ceil_div(std::min(S, L), TT) + ceil_div(std::min(W, L), TT);
+    const int per_head1 = std::min(kMaxSpecItems, std::max(1, sms / 4 / std::max(1, heads)));
+    const int tiles_per_item = std::max(1, ceil_div(tiles_max, per_head1));
+    pl->c1 = tiles_per_item * TT;
+    pl->n1 = ceil_div(tiles_max, tiles_per_item);
 
     const int ns = std::min(S, L);
     const int mid_max = std::max(0, std::max(ns, L - W) - ns);
     if (mid_max == 0) {
-        pl->c2 = kTile;
+        pl->c2 = TT;
         pl->n2 = 0;
     } else if (d.split_tokens > 0) {
-        pl->c2 = round_up(d.split_tokens, kTile);
+        pl->c2 = round_up(d.split_tokens, TT);
         pl->n2 = ceil_div(mid_max, pl->c2);
     } else {
         const int target = (d.batch == 1 ? 2 : 8) * sms;
         const int per_head2 = std::max(1, ceil_div(target, heads));
-        pl->c2 = round_up(std::max(1, ceil_div(mid_max, per_head2)), kTile);
+        pl->c2 = round_up(std::max(1, ceil_div(mid_max, per_head2)), TT);
         pl->n2 = ceil_div(mid_max, pl->c2);
     }
     const long long items2 = (long long)heads * pl->n2;
     pl->grid2 = (int)std::min<long long>(sms, items2);
     const int G = d.n_q_heads / d.n_kv_heads;
-    kernel_shape(d.dtype, d.head_dim, G, &pl->threads, &pl->smem, &pl->stages);
+    kernel_shape(d.dtype, d.head_dim, G, pl->engine, &pl->threads, &pl->smem, &pl->stages);
 
     const size_t B = d.batch, Hq = d.n_q_heads, D = d.head_dim;
     const size_t n1 = pl->n1, n2 = std::max(pl->n2, 1);
@@ -155,54 +197,90 @@ using KernelFn = void (*)(Params);
 struct KernelSet {
     KernelFn spec;
     KernelFn mid;
-    int smem;
-    int stages;
-    int threads;
+    int smem_spec, smem_mid;
+    int threads_spec, threads_mid;
+    int stages_mid;
 };
 
-template <typename T, int D, int G>
+template <typename T, int D, int G, bool MMA>
 KernelSet kernels_for() {
-    using C = Cfg<T, D, G>;
-    return KernelSet{attn_kernel<T, D, G, true>, attn_kernel<T, D, G, false>, C::kSmemBytes,
-                     C::STAGES, C::kThreads};
+    using CS = Cfg<T, D, G, true, MMA>;
+    using CM = Cfg<T, D, G, false, MMA>;
+    return KernelSet{attn_kernel<T, D, G, true, MMA>, attn_kernel<T, D, G, false, MMA>,
+                     CS::kSmemBytes, CM::kSmemBytes, CS::kThreads, CM::kThreads, CM::STAGES};
 }
 
-template <typename T, int D>
+template <typename T, int D, bool MMA>
 bool pick_g(int G, KernelSet* ks) {
     switch (G) {
-    case 1: *ks = kernels_for<T, D, 1>(); return true;
-    case 2: *ks = kernels_for<T, D, 2>(); return true;
-    case 4: *ks = kernels_for<T, D, 4>(); return true;
-    case 8: *ks = kernels_for<T, D, 8>(); return true;
+    case 1: *ks = kernels_for<T, D, 1, MMA>(); return true;
+    case 2: *ks = kernels_for<T, D, 2, MMA>(); return true;
+    case 4: *ks = kernels_for<T, D, 4, MMA>(); return true;
+    case 8: *ks = kernels_for<T, D, 8, MMA>(); return true;
     default: return false;
     }
 }
 
-bool pick(int dtype, int D, int G, KernelSet* ks) {
+bool pick(int dtype, int D, int G, int engine, KernelSet* ks) {
+    const bool mma = engine == ALSPEC_ENGINE_TENSOR_CORES;
     if (dtype == ALSPEC_BF16) {
-        if (D == 128) return pick_g<__nv_bfloat16, 128>(G, ks);
-        if (D == 64) return pick_g<__nv_bfloat16, 64>(G, ks);
-    } else if (dtype == ALSPEC_F32) {
-        if (D == 128) return pick_g<float, 128>(G, ks);
-        if (D == 64) return pick_g<float, 64>(G, ks);
+        if (mma) {
+            if (D == 128) return pick_g<__nv_bfloat16, 128, true>(G, ks);
+            if (D == 64) return pick_g<__nv_bfloat16, 64, true>(G, ks);
+        } else {
+            if (D == 128) return pick_g<__nv_bfloat16, 128, false>(G, ks);
+            if (D == 64) return pick_g<__nv_bfloat16, 64, false>(G, ks);
+        }
+    } else if (dtype == ALSPEC_F32 && !mma) {
+        if (D == 128) return pick_g<float, 128, false>(G, ks);
+        if (D == 64) return pick_g<float, 64, false>(G, ks);
     }
     return false;
 }
 
-void kernel_shape(int dtype, int D, int G, int* threads, int* smem, int* stages) {
+void kernel_shape(int dtype, int D, int G, int engine, int* threads, int* smem, int* stages) {
     KernelSet ks{};
-    const bool ok = pick(dtype, D, G, &ks);
-    *threads = ok ? ks.threads : 0;
-    *smem = ok ? ks.smem : 0;
-    *stages = ok ? ks.stages : 0;
+    const bool found = pick(dtype, D, G, engine, &ks);
+    *threads = found ? ks.threads_mid : 0;
+    *smem = found ? ks.smem_mid : 0;
+    *stages = found ? ks.stages_mid : 0;
+}
+
+// cuTensorMapEncodeTiled from the driver, looked up once.
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+alspec_status encode_kv_map(CUtensorMap* map, const void* base, const alspec_desc& d) {
+    {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        if (!g_encode) {
+            cudaDriverEntryPointQueryResult q{};
+            void* fn = nullptr;
+            if (!ok(cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q)) ||
+                q != cudaDriverEntryPointSuccess || !fn)
+                return ALSPEC_ERR_CUDA;
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+        }
+    }
+    // A 2-D view of the cache: rows = (b, kv head, token), d columns; boxes of
+    // 64 columns (128 bytes) x 32 rows with 128-byte swizzle.
+    const cuuint64_t rows = (cuuint64_t)d.batch * d.n_kv_heads * d.max_seq_len;
+    const cuuint64_t dims[2] = {(cuuint64_t)d.head_dim, rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)d.head_dim * 2};
+    const cuuint32_t box[2] = {64, 32};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base),
+                                dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? ALSPEC_OK : ALSPEC_ERR_INVALID_ARG;
 }
 
 alspec_status ensure_smem_attr(DeviceState* ds, KernelFn fn, int bytes) {
     std::lock_guard<std::mutex> lock(g_mutex);
     const void* key = reinterpret_cast<const void*>(fn);
     if (ds->attr_done.count(key)) return ALSPEC_OK;
-    if (cudaFuncSetAttribute(reinterpret_cast<const void*>(fn),
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+    if (!ok(cudaFuncSetAttribute(reinterpret_cast<const void*>(fn),
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, bytes)))
         return ALSPEC_ERR_CUDA;
     ds->attr_done.insert(key);
     return ALSPEC_OK;
@@ -222,7 +300,7 @@ alspec_status launch(KernelFn fn, dim3 grid, dim3 block, int smem, cudaStream_t 
         cfg.attrs = attr;
         cfg.numAttrs = 1;
     }
-    return cudaLaunchKernelEx(&cfg, fn, p) == cudaSuccess ? ALSPEC_OK : ALSPEC_ERR_CUDA;
+    return ok(cudaLaunchKernelEx(&cfg, fn, p)) ? ALSPEC_OK : ALSPEC_ERR_CUDA;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -256,8 +334,9 @@ alspec_status alspec_query_plan(const alspec_desc* desc, int n_sink, int window,
     if (!info || n_info < 0) return ALSPEC_ERR_INVALID_ARG;
     Plan pl{};
     make_plan(*desc, n_sink, window, sm_count_for_plan(), &pl);
-    const int vals[8] = {pl.c1, pl.n1, pl.c2, pl.n2, pl.grid2, pl.threads, pl.smem, pl.stages};
-    for (int i = 0; i < n_info && i < 8; ++i) info[i] = vals[i];
+    const int vals[9] = {pl.c1,      pl.n1,      pl.c2,   pl.n2,     pl.grid2,
+                         pl.threads, pl.smem,    pl.stages, pl.engine};
+    for (int i = 0; i < n_info && i < 9; ++i) info[i] = vals[i];
     return ALSPEC_OK;
 }
 
@@ -282,12 +361,16 @@ alspec_status alspec_decode(const alspec_desc* desc, const void* q, const void* 
     if ((st = get_device_state(&ds)) != ALSPEC_OK) return st;
     const int G = desc->n_q_heads / desc->n_kv_heads;
     KernelSet ks{};
-    if (!pick(desc->dtype, desc->head_dim, G, &ks)) return ALSPEC_ERR_UNSUPPORTED;
-    if ((st = ensure_smem_attr(ds, ks.spec, ks.smem)) != ALSPEC_OK) return st;
-    if ((st = ensure_smem_attr(ds, ks.mid, ks.smem)) != ALSPEC_OK) return st;
+    if (!pick(desc->dtype, desc->head_dim, G, pl.engine, &ks)) return ALSPEC_ERR_UNSUPPORTED;
+    if ((st = ensure_smem_attr(ds, ks.spec, ks.smem_spec)) != ALSPEC_OK) return st;
+    if ((st = ensure_smem_attr(ds, ks.mid, ks.smem_mid)) != ALSPEC_OK) return st;
 
     char* ws = static_cast<char*>(workspace);
     Params p{};
+    if (pl.engine == ALSPEC_ENGINE_TENSOR_CORES) {
+        if ((st = encode_kv_map(&p.tmap_k, k_cache, *desc)) != ALSPEC_OK) return st;
+        if ((st = encode_kv_map(&p.tmap_v, v_cache, *desc)) != ALSPEC_OK) return st;
+    }
     p.q = q;
     p.k = k_cache;
     p.v = v_cache;
@@ -321,32 +404,30 @@ alspec_status alspec_decode(const alspec_desc* desc, const void* q, const void* 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     auto prof = [&](int i, cudaStream_t on) {
         return !prof_events || !prof_events[i] ||
-               cudaEventRecordWithFlags(static_cast<cudaEvent_t>(prof_events[i]), on,
-                                        cudaEventRecordExternal) == cudaSuccess;
+               ok(record_event(static_cast<cudaEvent_t>(prof_events[i]), on));
     };
     if (!prof(0, s)) return ALSPEC_ERR_CUDA;
     // Fork: the sink-set kernel runs on the high-priority stream.
-    if (cudaEventRecord(ds->fork, s) != cudaSuccess ||
-        cudaStreamWaitEvent(ds->hi, ds->fork, 0) != cudaSuccess)
+    if (!ok(cudaEventRecord(ds->fork, s)) || !ok(cudaStreamWaitEvent(ds->hi, ds->fork, 0)))
         return ALSPEC_ERR_CUDA;
-    const dim3 block(pl.threads);
     const dim3 grid1(desc->batch * desc->n_kv_heads * pl.n1);
-    if ((st = launch(ks.spec, grid1, block, ks.smem, ds->hi, p, true, ds->prio_hi)) != ALSPEC_OK)
+    if ((st = launch(ks.spec, grid1, dim3(ks.threads_spec), ks.smem_spec, ds->hi, p, true,
+                     ds->prio_hi)) != ALSPEC_OK)
         return st;
-    if (spec_event && cudaEventRecordWithFlags(static_cast<cudaEvent_t>(spec_event), ds->hi,
-                                               cudaEventRecordExternal) != cudaSuccess)
+    if (spec_event && !ok(record_event(static_cast<cudaEvent_t>(spec_event), ds->hi)))
         return ALSPEC_ERR_CUDA;
     if (!prof(1, ds->hi)) return ALSPEC_ERR_CUDA;
-    if (cudaEventRecord(ds->join, ds->hi) != cudaSuccess) return ALSPEC_ERR_CUDA;
+    if (!ok(cudaEventRecord(ds->join, ds->hi))) return ALSPEC_ERR_CUDA;
     // The middle of every sequence on the caller's stream.
     if (!prof(2, s)) return ALSPEC_ERR_CUDA;
     if (pl.n2 > 0) {
-        if ((st = launch(ks.mid, dim3(pl.grid2), block, ks.smem, s, p, false, 0)) != ALSPEC_OK)
+        if ((st = launch(ks.mid, dim3(pl.grid2), dim3(ks.threads_mid), ks.smem_mid, s, p, false,
+                         0)) != ALSPEC_OK)
             return st;
     }
     if (!prof(3, s)) return ALSPEC_ERR_CUDA;
     // Join, then merge + relative L2 + flag.
-    if (cudaStreamWaitEvent(s, ds->join, 0) != cudaSuccess) return ALSPEC_ERR_CUDA;
+    if (!ok(cudaStreamWaitEvent(s, ds->join, 0))) return ALSPEC_ERR_CUDA;
     KernelFn mk = desc->head_dim == 128 ? merge_kernel<128> : merge_kernel<64>;
     if ((st = launch(mk, dim3(desc->n_q_heads, desc->batch), dim3(desc->head_dim), 0, s, p, false,
                      0)) != ALSPEC_OK)
@@ -443,5 +524,7 @@ const char* alspec_status_string(alspec_status status) {
 }
 
 int alspec_version(void) { return 100; }
+
+int alspec_last_cuda_error(void) { return (int)t_last_error; }
 
 }  // extern "C"

@@ -19,22 +19,30 @@
 //   * the merge kernel combines the sink-set partial with the middle
 //     partials into O_exact, then computes rel_l2 and the flag.
 //
-// Inside a CTA: one producer lane issues bulk asynchronous copies (the TMA
-// engine's 1-D form) of 16-token K and V tiles into a ring of shared-memory
-// stages guarded by mbarriers; eight consumer warps compute.  Every token
-// row is handled by 8 lanes (each owning head_dim/8 elements, read as 16-byte
-// chunks at stride 128 bytes, which is free of bank conflicts), so a warp
-// covers the 16 tokens of a tile: 4 rows per 8-lane group.  Dot products use
-// packed fp32x2 FMAs on bf16 values widened in registers; the 8 partial dots
-// of a row are combined by a reduce-scatter so that each lane pair ends up
-// owning one token's scores.  Online softmax keeps a warp-uniform running
-// max per head.  At the end of an item the warps' states are merged through
-// shared memory and one partial per query head is written.
+// Inside a CTA one producer lane fills a ring of shared-memory stages with
+// K and V tiles through the TMA engine (mbarrier completion); consumer warps
+// compute.  Each stage belongs to one consumer warp ("token slot"), so a
+// warp visits its stages in order and every item is padded to a multiple
+// of the slot count.  At the end of an item the warps' states are merged
+// through shared memory and one partial per query head is written.
+//
+// Two compute engines share that pipeline:
+//   * tensor cores (bf16 caches): 32-token tiles loaded as 2-D TMA boxes
+//     with 128-byte swizzle.  S^T = Q K^T and O += P V run as m16n8k16 MMAs
+//     (fp32 accumulation): the query heads of a KV group are the 16 rows of
+//     the A operand (rows 8..15 zero), K and V fragments come from ldmatrix,
+//     and the score fragment is reused as the A operand of P V.  P is split
+//     into a bf16 high part (rows 0..7) and the bf16 rounding residual
+//     (rows 8..15), so P V keeps ~16 bits of P instead of 8;
+//   * CUDA cores (fp32 caches, and bf16 on request): 16-token tiles loaded by
+//     1-D bulk copies; 8 lanes per token row with packed fp32x2 FMAs and a
+//     reduce-scatter of the partial dot products.
 //
 // Every wait is bounded (global nanosecond timer); on expiry the kernel sets
 // an error bit, stops issuing copies, drains the ones in flight and returns.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 
 #include <cstdint>
@@ -43,7 +51,6 @@
 
 namespace alspec {
 
-constexpr int kTile = 16;             // tokens per pipeline stage
 constexpr int kSmemLimit = 227 * 1024;
 
 constexpr unsigned kErrSeqLen = 1u;   // ALSPEC_DEVERR_SEQ_LEN
@@ -59,6 +66,8 @@ constexpr int kCtrFixed = 4;
 constexpr int kLastTileFlag = 1;
 
 struct Params {
+    CUtensorMap tmap_k;  // 2-D views [rows = B*Hkv*Lmax, d] (tensor-core engine)
+    CUtensorMap tmap_v;
     const void* q;
     const void* k;
     const void* v;
@@ -83,57 +92,90 @@ struct Params {
     unsigned long long timeout_ns;
 };
 
+__host__ __device__ __forceinline__ int cdiv(int a, int b) { return (a + b - 1) / b; }
+
 // Token geometry of one sequence: sink tokens [0, ns), window [ws, L),
-// middle [ns, ws).  Out-of-range lengths are clamped (and flagged).
+// middle [ns, ws).
 struct SeqGeom {
-    int L, ns, ws, nspec, mid_len;
+    int L, ns, ws, mid_len;
 };
 
+__host__ __device__ __forceinline__ SeqGeom geom_of(int L, int S, int W) {
+    SeqGeom g;
+    g.L = L;
+    g.ns = L < S ? L : S;
+    const int w0 = L - W;
+    g.ws = w0 > g.ns ? w0 : g.ns;
+    g.mid_len = g.ws - g.ns;
+    return g;
+}
+
+// Reads seq_lens[b]; out-of-range lengths are clamped (and flagged).
 __device__ __forceinline__ SeqGeom seq_geom(const Params& p, int b, bool flag) {
     int L = __ldg(p.seq_lens + b);
     if (L < 1 || L > p.Lmax) {
         if (flag) atomicOr(p.ctr + kCtrError, kErrSeqLen);
         L = L < 1 ? 1 : p.Lmax;
     }
-    SeqGeom g;
-    g.L = L;
-    g.ns = min(p.S, L);
-    g.ws = max(g.ns, L - p.W);
-    g.nspec = g.ns + (L - g.ws);
-    g.mid_len = g.ws - g.ns;
-    return g;
+    return geom_of(L, p.S, p.W);
 }
 
-// One work item: n tokens, the first na of them at [a0, a0 + na) and the
-// rest at [a1, a1 + n - na).
+// Tiles of the sink-set list: the sink run and the window run are tiled
+// separately, so every tile is one contiguous run of cache rows.
+__host__ __device__ __forceinline__ int spec_tiles(const SeqGeom& g, int TT) {
+    return cdiv(g.ns, TT) + cdiv(g.L - g.ws, TT);
+}
+
+// One work item: a range of tiles of one (sequence, KV head).
 struct Item {
-    int b, kvh, chunk, n, a0, na, a1;
+    int b, kvh, chunk, ntiles;
+    int t0, ns, ws, L;  // sink-set items
+    int lo, hi;         // middle items
 };
 
-template <bool SPEC>
+template <bool SPEC, int TT>
 __device__ __forceinline__ Item decode_item(const Params& p, int item, bool flag) {
     Item it;
     const int bh = item % (p.B * p.Hkv);
     it.chunk = item / (p.B * p.Hkv);
     it.b = bh / p.Hkv;
     it.kvh = bh % p.Hkv;
-    SeqGeom g = seq_geom(p, it.b, flag);
+    const SeqGeom g = seq_geom(p, it.b, flag);
+    it.ns = g.ns;
+    it.ws = g.ws;
+    it.L = g.L;
     if (SPEC) {
-        const int lo = it.chunk * p.c1;
-        const int hi = min(lo + p.c1, g.nspec);
-        it.n = max(0, hi - lo);
-        it.a0 = lo;
-        it.na = max(0, min(hi, g.ns) - lo);
-        it.a1 = g.ws + max(lo, g.ns) - g.ns;
+        const int per = p.c1 / TT;
+        it.t0 = it.chunk * per;
+        const int t1 = min(it.t0 + per, spec_tiles(g, TT));
+        it.ntiles = max(0, t1 - it.t0);
+        it.lo = it.hi = 0;
     } else {
-        const int lo = g.ns + it.chunk * p.c2;
-        const int hi = min(lo + p.c2, g.ws);
-        it.n = max(0, hi - lo);
-        it.a0 = lo;
-        it.na = it.n;
-        it.a1 = 0;
+        it.lo = g.ns + it.chunk * p.c2;
+        it.hi = min(it.lo + p.c2, g.ws);
+        it.ntiles = it.hi > it.lo ? cdiv(it.hi - it.lo, TT) : 0;
+        it.t0 = 0;
     }
     return it;
+}
+
+// First cache row (within the head) and valid row count of tile t.
+template <bool SPEC, int TT>
+__device__ __forceinline__ void tile_rows(const Item& it, int t, int& start, int& nvalid) {
+    if (SPEC) {
+        const int tg = it.t0 + t;
+        const int tsink = cdiv(it.ns, TT);
+        if (tg < tsink) {
+            start = tg * TT;
+            nvalid = min(TT, it.ns - start);
+        } else {
+            start = it.ws + (tg - tsink) * TT;
+            nvalid = min(TT, it.L - start);
+        }
+    } else {
+        start = it.lo + t * TT;
+        nvalid = min(TT, it.hi - start);
+    }
 }
 
 // ------------------------------------------------------------ element types
@@ -167,43 +209,48 @@ struct Elem<__nv_bfloat16> {
 
 // ------------------------------------------------------------ configuration
 
-template <typename T, int D, int G>
+// Pipeline shape shared by both engines.
+//   TT    tokens per stage            GW   heads a consumer warp holds
+//   NHW   warps sharing a stage       NTW  token slots (stages per round)
+//   SPW   stages per token slot
+template <typename T, int D, int G, bool SPEC, bool MMA>
 struct Cfg {
     static constexpr int kRowBytes = D * (int)sizeof(T);
-    static constexpr int kChunks = kRowBytes / 128;        // 16-B chunks per lane per row
-    static constexpr int kPairs = Elem<T>::kPairs;         // float2 per chunk
-    static constexpr int kLanePairs = kChunks * kPairs;    // float2 per lane per row
-    static constexpr int kElemPerChunk = 16 / (int)sizeof(T);
-    static constexpr int kElemPer128 = 128 / (int)sizeof(T);
-    static constexpr int GW = G < 4 ? G : 4;               // heads per consumer warp
-    static constexpr int NHW = G / GW;                     // warps sharing a tile
-    // Warps are spread over the SM's four sub-partitions, each with 16K
-    // registers: 8 warps per CTA allow 255 registers a thread, 9 only 168.
-    // Configurations holding 4 heads x 16 elements of q and o per lane need
-    // the former, so they run 7 consumer warps plus the producer.
-    static constexpr bool kHeavy = GW * kLanePairs >= 32;
-    static constexpr int NTW = (kHeavy ? 7 : 8) / NHW;     // tiles in flight per round
-    static constexpr int NCW = NTW * NHW;                  // consumer warps
+    static constexpr int TT = MMA ? 32 : 16;
+    static constexpr int GW = MMA ? G : (G < 4 ? G : 4);
+    static constexpr int NHW = G / GW;
+    // CUDA-core engine: warps are spread over the SM's four sub-partitions
+    // with 16K registers each; 8 warps per CTA allow 255 registers a thread,
+    // 9 only 168.  Holding 4 heads x 16 elements of q and o per lane needs
+    // the former, so those configurations run 7 consumer warps.
+    static constexpr int kLanePairs = (kRowBytes / 128) * Elem<T>::kPairs;
+    static constexpr bool kHeavy = !MMA && GW * kLanePairs >= 32;
+    static constexpr int NTW = MMA ? 4 : (kHeavy ? 7 : 8) / NHW;
+    static constexpr int NCW = NTW * NHW;
     static constexpr int kThreads = (NCW + 1) * 32;
-    static constexpr int kTileBytes = kTile * kRowBytes;   // K or V part of a stage
+    static constexpr int kTileBytes = TT * kRowBytes;  // K or V part of a stage
     static constexpr int kStageBytes = 2 * kTileBytes;
     static constexpr int kSlotFloats = GW * (D + 2);
     static constexpr int kDepositBytes = NCW * kSlotFloats * 4;
+    static constexpr int kSpwMax = SPEC ? 1 : (MMA ? 3 : 4);
     static constexpr int kSpwBudget =
-        (kSmemLimit - kDepositBytes - 4096) / (NTW * kStageBytes);
-    static constexpr int SPW = kSpwBudget < 1 ? 1 : (kSpwBudget > 4 ? 4 : kSpwBudget);
+        (kSmemLimit - 1024 - kDepositBytes - 4096) / (NTW * kStageBytes);
+    static constexpr int SPW = kSpwBudget < 1 ? 1 : (kSpwBudget > kSpwMax ? kSpwMax : kSpwBudget);
     static constexpr int STAGES = NTW * SPW;
-    // Dynamic shared memory layout.
+    // Dynamic shared memory layout (offsets from a 1024-byte aligned base).
     static constexpr int kOffDeposit = STAGES * kStageBytes;
     static constexpr int kOffMeta = kOffDeposit + kDepositBytes;
     static constexpr int kOffBar = kOffMeta + STAGES * 16;
     static constexpr int kNumBars = 2 * STAGES + 3;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-    static constexpr int kSmemBytes = kOffMisc + 16;
+    static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
     static_assert(kRowBytes % 128 == 0, "row must be a multiple of 128 bytes");
     static_assert(G == 1 || G == 2 || G == 4 || G == 8, "group size");
+    static_assert(!MMA || (sizeof(T) == 2 && G <= 8), "tensor-core engine: bf16, g <= 8");
     static_assert(kSmemBytes <= kSmemLimit, "shared memory budget");
     static_assert(NTW >= 1 && NCW <= 8, "warp split");
+    // The sink-set merge reuses the deposit area for (m, l) of G x 32 items.
+    static_assert(kDepositBytes >= G * 32 * 8, "deposit area too small");
 };
 
 // ---------------------------------------------------------------- waiting
@@ -256,159 +303,371 @@ __device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, volati
     }
 }
 
-// ------------------------------------------------------------ consumer state
-
-template <class C>
-struct WarpState {
-    float2 q[C::GW][C::kLanePairs];  // prescaled query slice
-    float2 o[C::GW][C::kLanePairs];  // unnormalised output slice
-    float m[C::GW];                  // warp-uniform running max (log2 domain)
-    float l[C::GW];                  // this lane's share of the exponential sum
-};
-
-template <class C>
-__device__ __forceinline__ void reset_state(WarpState<C>& st) {
-#pragma unroll
-    for (int h = 0; h < C::GW; ++h) {
-        st.m[h] = -INFINITY;
-        st.l[h] = 0.f;
-#pragma unroll
-        for (int j = 0; j < C::kLanePairs; ++j) st.o[h][j] = make_float2(0.f, 0.f);
-    }
-}
-
-template <typename T, class C>
-__device__ __forceinline__ void load_query(WarpState<C>& st, const Params& p, int b, int head0,
-                                           int li) {
-#pragma unroll
-    for (int h = 0; h < C::GW; ++h) {
-        const char* row = reinterpret_cast<const char*>(p.q) +
-                          ((size_t)b * p.Hq + head0 + h) * C::kRowBytes + li * 16;
-#pragma unroll
-        for (int c = 0; c < C::kChunks; ++c) {
-            const uint4 raw = __ldg(reinterpret_cast<const uint4*>(row + c * 128));
-            float2 f[C::kPairs];
-            Elem<T>::unpack(raw, f);
-#pragma unroll
-            for (int j = 0; j < C::kPairs; ++j)
-                st.q[h][c * C::kPairs + j] = make_float2(f[j].x * p.qscale, f[j].y * p.qscale);
-        }
-    }
-}
-
-// One 16-token tile: scores, online-softmax update, value accumulation.
-template <typename T, class C>
-__device__ __forceinline__ void consume_tile(WarpState<C>& st, const char* ks, const char* vs,
-                                             int nvalid, int lane) {
-    const int grp = lane >> 3;
-    const int li = lane & 7;
-    const unsigned full = 0xffffffffu;
-
-    // Partial dot products of this lane's slice for the group's 4 rows.
-    float acc[4][C::GW];
-#pragma unroll
-    for (int t = 0; t < 4; ++t) {
-        const char* krow = ks + (grp * 4 + t) * C::kRowBytes + li * 16;
-        float2 a[C::GW];
-#pragma unroll
-        for (int h = 0; h < C::GW; ++h) a[h] = make_float2(0.f, 0.f);
-#pragma unroll
-        for (int c = 0; c < C::kChunks; ++c) {
-            const uint4 raw = *reinterpret_cast<const uint4*>(krow + c * 128);
-            float2 kf[C::kPairs];
-            Elem<T>::unpack(raw, kf);
-#pragma unroll
-            for (int j = 0; j < C::kPairs; ++j)
-#pragma unroll
-                for (int h = 0; h < C::GW; ++h)
-                    a[h] = __ffma2_rn(st.q[h][c * C::kPairs + j], kf[j], a[h]);
-        }
-#pragma unroll
-        for (int h = 0; h < C::GW; ++h) acc[t][h] = a[h].x + a[h].y;
-    }
-
-    // Reduce-scatter over the 8 lanes of the group: lanes 2u and 2u+1 end up
-    // with the full score of row u.
-    const bool b2 = (li & 4) != 0;
-    const bool b1 = (li & 2) != 0;
-    const int own = li >> 1;
-    const bool valid = grp * 4 + own < nvalid;
-    float s[C::GW];
-#pragma unroll
-    for (int h = 0; h < C::GW; ++h) {
-        const float k0 = b2 ? acc[2][h] : acc[0][h];
-        const float s0 = b2 ? acc[0][h] : acc[2][h];
-        const float k1 = b2 ? acc[3][h] : acc[1][h];
-        const float s1 = b2 ? acc[1][h] : acc[3][h];
-        const float w0 = k0 + __shfl_xor_sync(full, s0, 4);
-        const float w1 = k1 + __shfl_xor_sync(full, s1, 4);
-        const float kk = b1 ? w1 : w0;
-        const float ss = b1 ? w0 : w1;
-        float x = kk + __shfl_xor_sync(full, ss, 2);
-        x += __shfl_xor_sync(full, x, 1);
-        s[h] = valid ? x : -INFINITY;
-    }
-
-    // Online softmax with a warp-uniform running max.
-    float pr[C::GW];
-#pragma unroll
-    for (int h = 0; h < C::GW; ++h) {
-        float mx = s[h];
-        mx = fmaxf(mx, __shfl_xor_sync(full, mx, 2));
-        mx = fmaxf(mx, __shfl_xor_sync(full, mx, 4));
-        mx = fmaxf(mx, __shfl_xor_sync(full, mx, 8));
-        mx = fmaxf(mx, __shfl_xor_sync(full, mx, 16));
-        if (mx > st.m[h]) {
-            const float sc = exp2f(st.m[h] - mx);
-            const float2 sc2 = make_float2(sc, sc);
-#pragma unroll
-            for (int j = 0; j < C::kLanePairs; ++j) st.o[h][j] = __fmul2_rn(st.o[h][j], sc2);
-            st.l[h] *= sc;
-            st.m[h] = mx;
-        }
-        pr[h] = valid ? exp2f(s[h] - st.m[h]) : 0.f;
-        st.l[h] += (li & 1) ? 0.f : pr[h];
-    }
-
-    // Weighted value rows.
-#pragma unroll
-    for (int t = 0; t < 4; ++t) {
-        float pt[C::GW];
-#pragma unroll
-        for (int h = 0; h < C::GW; ++h) pt[h] = __shfl_sync(full, pr[h], (lane & 24) | (t << 1));
-        if (grp * 4 + t < nvalid) {
-            const char* vrow = vs + (grp * 4 + t) * C::kRowBytes + li * 16;
-#pragma unroll
-            for (int c = 0; c < C::kChunks; ++c) {
-                const uint4 raw = *reinterpret_cast<const uint4*>(vrow + c * 128);
-                float2 vf[C::kPairs];
-                Elem<T>::unpack(raw, vf);
-#pragma unroll
-                for (int h = 0; h < C::GW; ++h) {
-                    const float2 pp = make_float2(pt[h], pt[h]);
-#pragma unroll
-                    for (int j = 0; j < C::kPairs; ++j)
-                        st.o[h][c * C::kPairs + j] =
-                            __ffma2_rn(pp, vf[j], st.o[h][c * C::kPairs + j]);
-                }
-            }
-        }
-    }
-}
-
 // Weight of a partial with max m against the merged max M: exactly 1 when
 // m == M, so merging one partial with empty ones reproduces it bit for bit.
 __device__ __forceinline__ float merge_weight(float m, float M) {
     return m == M ? 1.f : exp2f(m - M);
 }
 
+// ====================================================== CUDA-core engine
+
+template <class C, typename T>
+struct CoreEngine {
+    static constexpr int kPairs = Elem<T>::kPairs;
+    static constexpr int kChunks = C::kRowBytes / 128;
+    static constexpr int kLanePairs = kChunks * kPairs;
+    static constexpr int kElemPerChunk = 16 / (int)sizeof(T);
+    static constexpr int kElemPer128 = 128 / (int)sizeof(T);
+    static constexpr int kD = C::kRowBytes / (int)sizeof(T);
+
+    float2 q[C::GW][kLanePairs];  // prescaled query slice
+    float2 o[C::GW][kLanePairs];  // unnormalised output slice
+    float m[C::GW];               // warp-uniform running max (log2 domain)
+    float l[C::GW];               // this lane's share of the exponential sum
+
+    __device__ __forceinline__ void reset() {
+#pragma unroll
+        for (int h = 0; h < C::GW; ++h) {
+            m[h] = -INFINITY;
+            l[h] = 0.f;
+#pragma unroll
+            for (int j = 0; j < kLanePairs; ++j) o[h][j] = make_float2(0.f, 0.f);
+        }
+    }
+
+    __device__ __forceinline__ void load_query(const Params& p, int b, int head0, int lane) {
+        const int li = lane & 7;
+#pragma unroll
+        for (int h = 0; h < C::GW; ++h) {
+            const char* row = reinterpret_cast<const char*>(p.q) +
+                              ((size_t)b * p.Hq + head0 + h) * C::kRowBytes + li * 16;
+#pragma unroll
+            for (int c = 0; c < kChunks; ++c) {
+                const uint4 raw = __ldg(reinterpret_cast<const uint4*>(row + c * 128));
+                float2 f[kPairs];
+                Elem<T>::unpack(raw, f);
+#pragma unroll
+                for (int j = 0; j < kPairs; ++j)
+                    q[h][c * kPairs + j] = make_float2(f[j].x * p.qscale, f[j].y * p.qscale);
+            }
+        }
+    }
+
+    // One 16-token tile: lanes 8u..8u+7 ("group" u) own rows 4u..4u+3.
+    __device__ __forceinline__ void tile(char* ks, char* vs, int nvalid, int lane, float) {
+        const int grp = lane >> 3;
+        const int li = lane & 7;
+        const unsigned full = 0xffffffffu;
+
+        float acc[4][C::GW];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            const char* krow = ks + (grp * 4 + t) * C::kRowBytes + li * 16;
+            float2 a[C::GW];
+#pragma unroll
+            for (int h = 0; h < C::GW; ++h) a[h] = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int c = 0; c < kChunks; ++c) {
+                const uint4 raw = *reinterpret_cast<const uint4*>(krow + c * 128);
+                float2 kf[kPairs];
+                Elem<T>::unpack(raw, kf);
+#pragma unroll
+                for (int j = 0; j < kPairs; ++j)
+#pragma unroll
+                    for (int h = 0; h < C::GW; ++h)
+                        a[h] = __ffma2_rn(q[h][c * kPairs + j], kf[j], a[h]);
+            }
+#pragma unroll
+            for (int h = 0; h < C::GW; ++h) acc[t][h] = a[h].x + a[h].y;
+        }
+
+        // Reduce-scatter over the 8 lanes of the group: lanes 2u and 2u+1
+        // end up with the full score of row u of the group.
+        const bool b2 = (li & 4) != 0;
+        const bool b1 = (li & 2) != 0;
+        const int own = li >> 1;
+        const bool valid = grp * 4 + own < nvalid;
+        float s[C::GW];
+#pragma unroll
+        for (int h = 0; h < C::GW; ++h) {
+            const float k0 = b2 ? acc[2][h] : acc[0][h];
+            const float s0 = b2 ? acc[0][h] : acc[2][h];
+            const float k1 = b2 ? acc[3][h] : acc[1][h];
+            const float s1 = b2 ? acc[1][h] : acc[3][h];
+            const float w0 = k0 + __shfl_xor_sync(full, s0, 4);
+            const float w1 = k1 + __shfl_xor_sync(full, s1, 4);
+            const float kk = b1 ? w1 : w0;
+            const float ss = b1 ? w0 : w1;
+            float x = kk + __shfl_xor_sync(full, ss, 2);
+            x += __shfl_xor_sync(full, x, 1);
+            s[h] = valid ? x : -INFINITY;
+        }
+
+        float pr[C::GW];
+#pragma unroll
+        for (int h = 0; h < C::GW; ++h) {
+            float mx = s[h];
+            mx = fmaxf(mx, __shfl_xor_sync(full, mx, 2));
+            mx = fmaxf(mx, __shfl_xor_sync(full, mx, 4));
+            mx = fmaxf(mx, __shfl_xor_sync(full, mx, 8));
+            mx = fmaxf(mx, __shfl_xor_sync(full, mx, 16));
+            if (mx > m[h]) {
+                const float sc = exp2f(m[h] - mx);
+                const float2 sc2 = make_float2(sc, sc);
+#pragma unroll
+                for (int j = 0; j < kLanePairs; ++j) o[h][j] = __fmul2_rn(o[h][j], sc2);
+                l[h] *= sc;
+                m[h] = mx;
+            }
+            pr[h] = valid ? exp2f(s[h] - m[h]) : 0.f;
+            l[h] += (li & 1) ? 0.f : pr[h];
+        }
+
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            float pt[C::GW];
+#pragma unroll
+            for (int h = 0; h < C::GW; ++h) pt[h] = __shfl_sync(full, pr[h], (lane & 24) | (t << 1));
+            if (grp * 4 + t < nvalid) {
+                const char* vrow = vs + (grp * 4 + t) * C::kRowBytes + li * 16;
+#pragma unroll
+                for (int c = 0; c < kChunks; ++c) {
+                    const uint4 raw = *reinterpret_cast<const uint4*>(vrow + c * 128);
+                    float2 vf[kPairs];
+                    Elem<T>::unpack(raw, vf);
+#pragma unroll
+                    for (int h = 0; h < C::GW; ++h) {
+                        const float2 pp = make_float2(pt[h], pt[h]);
+#pragma unroll
+                        for (int j = 0; j < kPairs; ++j)
+                            o[h][c * kPairs + j] = __ffma2_rn(pp, vf[j], o[h][c * kPairs + j]);
+                    }
+                }
+            }
+        }
+    }
+
+    // Reduce over the warp and store (m, l, o) of the GW heads into `slot`.
+    __device__ __forceinline__ void deposit(float* slot, int lane) {
+        const unsigned fm = 0xffffffffu;
+        const int li = lane & 7;
+#pragma unroll
+        for (int h = 0; h < C::GW; ++h) {
+            float lsum = l[h];
+#pragma unroll
+            for (int x = 1; x < 32; x <<= 1) lsum += __shfl_xor_sync(fm, lsum, x);
+#pragma unroll
+            for (int j = 0; j < kLanePairs; ++j) {
+                float2 v = o[h][j];
+                v.x += __shfl_xor_sync(fm, v.x, 8);
+                v.y += __shfl_xor_sync(fm, v.y, 8);
+                v.x += __shfl_xor_sync(fm, v.x, 16);
+                v.y += __shfl_xor_sync(fm, v.y, 16);
+                o[h][j] = v;
+            }
+            float* hs = slot + h * (kD + 2);
+            if (lane == 0) {
+                hs[0] = m[h];
+                hs[1] = lsum;
+            }
+            if (lane < 8) {
+#pragma unroll
+                for (int c = 0; c < kChunks; ++c)
+#pragma unroll
+                    for (int j = 0; j < kPairs; ++j) {
+                        const int e = c * kElemPer128 + li * kElemPerChunk + 2 * j;
+                        *reinterpret_cast<float2*>(hs + 2 + e) = o[h][c * kPairs + j];
+                    }
+            }
+        }
+    }
+};
+
+// ==================================================== tensor-core engine
+
+// Byte offset of 16-byte chunk `c` (0..7) of row `r` inside a 2-D TMA box
+// written with 128-byte swizzle (rows of 128 bytes).
+__device__ __forceinline__ uint32_t swz(int r, int c) {
+    return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+template <class C, int D, int G>
+struct MmaEngine {
+    static constexpr int TT = C::TT;            // 32 tokens: 4 score n-tiles, 2 PV k-steps
+    static constexpr int KS = D / 16;            // QK k-steps
+    static constexpr int NT = D / 8;             // PV n-tiles
+    static constexpr int kHalf = TT * 128;       // bytes of one 64-column box
+    static constexpr int kHalves = D / 64;
+
+    uint32_t qa[KS][2];  // A fragment words (row g, k 2r..2r+1) and (row g, k 2r+8..)
+    float o[NT][4];      // P V accumulators: rows g (high part of P) and g+8 (residual)
+    float m;             // running max of row g (log2 domain)
+    float l;             // this lane's share of the exponential sum of row g
+
+    __device__ __forceinline__ void reset() {
+        m = -INFINITY;
+        l = 0.f;
+#pragma unroll
+        for (int j = 0; j < NT; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+    }
+
+    __device__ __forceinline__ void load_query(const Params& p, int b, int head0, int lane) {
+        const int g = lane >> 2;
+        const int r = lane & 3;
+        if (g < G) {
+            const uint32_t* row = reinterpret_cast<const uint32_t*>(
+                reinterpret_cast<const __nv_bfloat16*>(p.q) + ((size_t)b * p.Hq + head0 + g) * D);
+#pragma unroll
+            for (int kk = 0; kk < KS; ++kk) {
+                qa[kk][0] = __ldg(row + kk * 8 + r);
+                qa[kk][1] = __ldg(row + kk * 8 + 4 + r);
+            }
+        } else {
+#pragma unroll
+            for (int kk = 0; kk < KS; ++kk) qa[kk][0] = qa[kk][1] = 0u;
+        }
+    }
+
+    // Row `r`, 16-byte chunk `c` (0..D/8-1) of a K or V tile in a stage.
+    __device__ __forceinline__ static uint32_t addr(uint32_t base, int r, int c) {
+        return base + (uint32_t)((c >> 3) * kHalf) + swz(r, c & 7);
+    }
+
+    __device__ __forceinline__ void tile(char* ks, char* vs, int nvalid, int lane, float qscale) {
+        const int g = lane >> 2;
+        const int r = lane & 3;
+        const unsigned full = 0xffffffffu;
+        // Rows past the end of the item may hold anything (even NaN): zero
+        // their values so that 0 * V stays 0 in the P V products.
+        if (nvalid < TT) {
+            const int n = (TT - nvalid) * kHalves * 8;  // 16-byte chunks to clear
+            for (int i = lane; i < n; i += 32) {
+                const int row = nvalid + i / (kHalves * 8);
+                const int rem = i % (kHalves * 8);
+                *reinterpret_cast<uint4*>(vs + (rem >> 3) * kHalf + row * 128 + (rem & 7) * 16) =
+                    make_uint4(0u, 0u, 0u, 0u);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+        }
+        const uint32_t kb = smem_addr(ks);
+        const uint32_t vb = smem_addr(vs);
+
+        // S^T = Q K^T: 4 n-tiles of 8 tokens.
+        float s[TT / 8][4];
+#pragma unroll
+        for (int j = 0; j < TT / 8; ++j) {
+            s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
+#pragma unroll
+            for (int kp = 0; kp < KS / 2; ++kp) {
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4(addr(kb, 8 * j + (lane & 7), 4 * kp + (lane >> 3)), b0, b1, b2, b3);
+                mma_bf16_16816(s[j], qa[2 * kp][0], 0u, qa[2 * kp][1], 0u, b0, b1);
+                mma_bf16_16816(s[j], qa[2 * kp + 1][0], 0u, qa[2 * kp + 1][1], 0u, b2, b3);
+            }
+        }
+
+        // Online softmax on row g (lanes 4g..4g+3 hold its 32 scores).
+        float mx = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < TT / 8; ++j)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const bool ok = g < G && 8 * j + 2 * r + e < nvalid;
+                s[j][e] = ok ? s[j][e] * qscale : -INFINITY;
+                mx = fmaxf(mx, s[j][e]);
+            }
+        mx = fmaxf(mx, __shfl_xor_sync(full, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(full, mx, 2));
+        const bool grow = mx > m;
+        if (__any_sync(full, grow)) {
+            const float sc = grow ? exp2f(m - mx) : 1.f;
+#pragma unroll
+            for (int j = 0; j < NT; ++j) {
+                o[j][0] *= sc;
+                o[j][1] *= sc;
+                o[j][2] *= sc;
+                o[j][3] *= sc;
+            }
+            l *= sc;
+            m = grow ? mx : m;
+        }
+        uint32_t pa[TT / 16][4];
+#pragma unroll
+        for (int t2 = 0; t2 < TT / 16; ++t2) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int j = 2 * t2 + h;
+                const float p0 = s[j][0] == -INFINITY ? 0.f : exp2f(s[j][0] - m);
+                const float p1 = s[j][1] == -INFINITY ? 0.f : exp2f(s[j][1] - m);
+                l += p0 + p1;
+                const uint32_t hi = pack_bf16(p0, p1);
+                const float r0 = p0 - __uint_as_float(hi << 16);
+                const float r1 = p1 - __uint_as_float(hi & 0xffff0000u);
+                pa[t2][2 * h] = hi;                     // rows g: high part
+                pa[t2][2 * h + 1] = pack_bf16(r0, r1);  // rows g+8: residual
+            }
+        }
+
+        // O += P V over the 2 k-steps of 16 tokens.
+#pragma unroll
+        for (int t2 = 0; t2 < TT / 16; ++t2) {
+#pragma unroll
+            for (int jp = 0; jp < NT / 2; ++jp) {
+                uint32_t b0, b1, b2, b3;
+                const int row = 16 * t2 + ((lane >> 3) & 1) * 8 + (lane & 7);
+                ldsm_x4_t(addr(vb, row, 2 * jp + (lane >> 4)), b0, b1, b2, b3);
+                mma_bf16_16816(o[2 * jp], pa[t2][0], pa[t2][1], pa[t2][2], pa[t2][3], b0, b1);
+                mma_bf16_16816(o[2 * jp + 1], pa[t2][0], pa[t2][1], pa[t2][2], pa[t2][3], b2, b3);
+            }
+        }
+    }
+
+    __device__ __forceinline__ void deposit(float* slot, int lane) {
+        const int g = lane >> 2;
+        const int r = lane & 3;
+        float lsum = l;
+        lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
+        lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
+        if (g < G) {
+            float* hs = slot + g * (D + 2);
+            if (r == 0) {
+                hs[0] = m;
+                hs[1] = lsum;
+            }
+#pragma unroll
+            for (int j = 0; j < NT; ++j)
+                *reinterpret_cast<float2*>(hs + 2 + 8 * j + 2 * r) =
+                    make_float2(o[j][0] + o[j][2], o[j][1] + o[j][3]);
+        }
+    }
+};
+
+template <class C, typename T, int D, int G, bool MMA>
+struct EngineOf {
+    using type = CoreEngine<C, T>;
+};
+template <class C, typename T, int D, int G>
+struct EngineOf<C, T, D, G, true> {
+    using type = MmaEngine<C, D, G>;
+};
+
 // ------------------------------------------------------------ the kernel
 
-template <typename T, int D, int G, bool SPEC>
-__global__ void __launch_bounds__(Cfg<T, D, G>::kThreads, 1)
+template <typename T, int D, int G, bool SPEC, bool MMA>
+__global__ void __launch_bounds__(Cfg<T, D, G, SPEC, MMA>::kThreads, 1)
     attn_kernel(const __grid_constant__ Params p) {
-    using C = Cfg<T, D, G>;
-    extern __shared__ __align__(128) unsigned char smem[];
+    using C = Cfg<T, D, G, SPEC, MMA>;
+    using Engine = typename EngineOf<C, T, D, G, MMA>::type;
+    constexpr int TT = C::TT;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* smem = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float* deposit = reinterpret_cast<float*>(smem + C::kOffDeposit);
     int4* meta = reinterpret_cast<int4*>(smem + C::kOffMeta);
     uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
@@ -440,6 +699,10 @@ __global__ void __launch_bounds__(Cfg<T, D, G>::kThreads, 1)
     if (warp == C::NCW) {
         // ---------------------------------------------------- producer
         if (lane != 0) return;
+        if (MMA) {
+            prefetch_tmap(&p.tmap_k);
+            prefetch_tmap(&p.tmap_v);
+        }
         uint32_t gt = 0;
         bool ok = true;
         for (int iter = 0; ok; ++iter) {
@@ -450,43 +713,42 @@ __global__ void __launch_bounds__(Cfg<T, D, G>::kThreads, 1)
                 item = (int)atomicAdd(p.ctr + kCtrQueue, 1u);
             }
             if (item >= n_items || *abort) break;
-            const Item it = decode_item<SPEC>(p, item, true);
-            if (it.n == 0) continue;
-            const size_t head_row = ((size_t)it.b * p.Hkv + it.kvh) * (size_t)p.Lmax;
-            const char* kbase = reinterpret_cast<const char*>(p.k) + head_row * C::kRowBytes;
-            const char* vbase = reinterpret_cast<const char*>(p.v) + head_row * C::kRowBytes;
-            int ntiles = (it.n + kTile - 1) / kTile;
-            ntiles = (ntiles + C::NTW - 1) / C::NTW * C::NTW;
+            const Item it = decode_item<SPEC, TT>(p, item, true);
+            if (it.ntiles == 0) continue;
+            const int head_row = (it.b * p.Hkv + it.kvh) * p.Lmax;
+            const size_t head_byte = (size_t)head_row * C::kRowBytes;
+            const int ntiles = (it.ntiles + C::NTW - 1) / C::NTW * C::NTW;
             for (int t = 0; t < ntiles; ++t, ++gt) {
                 const int s = gt % C::STAGES;
                 if (!wait_one(empty_bar + s, ((gt / C::STAGES) & 1) ^ 1, abort, p)) {
                     ok = false;
                     break;
                 }
-                const int first = t * kTile;
-                const int nvalid = max(0, min(kTile, it.n - first));
+                int start = 0, nvalid = 0;
+                if (t < it.ntiles) tile_rows<SPEC, TT>(it, t, start, nvalid);
                 meta[s] = make_int4(item, t, nvalid, t >= ntiles - C::NTW ? kLastTileFlag : 0);
                 if (nvalid == 0) {
                     mbar_arrive(full_bar + s);
                     continue;
                 }
-                mbar_arrive_expect_tx(full_bar + s, 2u * nvalid * C::kRowBytes);
                 char* ks = reinterpret_cast<char*>(smem) + s * C::kStageBytes;
                 char* vs = ks + C::kTileBytes;
-                // Up to two contiguous runs of rows (sink run, then window run).
-                const int ra = max(0, min(nvalid, it.na - first));
-                if (ra > 0) {
-                    const size_t tok = (size_t)(it.a0 + first);
-                    bulk_load(ks, kbase + tok * C::kRowBytes, ra * C::kRowBytes, full_bar + s);
-                    bulk_load(vs, vbase + tok * C::kRowBytes, ra * C::kRowBytes, full_bar + s);
-                }
-                if (nvalid > ra) {
-                    const size_t tok = (size_t)(it.a1 + (first + ra - it.na));
-                    const int rb = nvalid - ra;
-                    bulk_load(ks + ra * C::kRowBytes, kbase + tok * C::kRowBytes,
-                              rb * C::kRowBytes, full_bar + s);
-                    bulk_load(vs + ra * C::kRowBytes, vbase + tok * C::kRowBytes,
-                              rb * C::kRowBytes, full_bar + s);
+                if (MMA) {
+                    // Whole boxes; rows past the tensor end arrive as zeros.
+                    mbar_arrive_expect_tx(full_bar + s, (uint32_t)C::kStageBytes);
+#pragma unroll
+                    for (int h = 0; h < D / 64; ++h) {
+                        tma_load_2d(ks + h * TT * 128, &p.tmap_k, 64 * h, head_row + start,
+                                    full_bar + s);
+                        tma_load_2d(vs + h * TT * 128, &p.tmap_v, 64 * h, head_row + start,
+                                    full_bar + s);
+                    }
+                } else {
+                    const uint32_t bytes = (uint32_t)nvalid * C::kRowBytes;
+                    mbar_arrive_expect_tx(full_bar + s, 2u * bytes);
+                    const size_t off = head_byte + (size_t)start * C::kRowBytes;
+                    bulk_load(ks, reinterpret_cast<const char*>(p.k) + off, bytes, full_bar + s);
+                    bulk_load(vs, reinterpret_cast<const char*>(p.v) + off, bytes, full_bar + s);
                 }
             }
         }
@@ -528,19 +790,14 @@ __global__ void __launch_bounds__(Cfg<T, D, G>::kThreads, 1)
     // -------------------------------------------------------- consumers
     const int hw = warp / C::NTW;   // which GW heads of the group
     const int tw = warp % C::NTW;   // which token slot of the round
-    const int li = lane & 7;
-    WarpState<C> st;
-    reset_state(st);
+    Engine st;
+    st.reset();
     uint32_t gt = tw;
     int items_done = 0;
-    bool ok = true;
     int b = 0, kvh = 0, chunk = 0;
     for (;; gt += C::NTW) {
         const int s = gt % C::STAGES;
-        if (!wait_warp(full_bar + s, (gt / C::STAGES) & 1, abort, p, lane)) {
-            ok = false;
-            break;
-        }
+        if (!wait_warp(full_bar + s, (gt / C::STAGES) & 1, abort, p, lane)) break;
         const int4 mt = meta[s];
         if (mt.x < 0) break;
         if (mt.y < C::NTW) {
@@ -548,63 +805,22 @@ __global__ void __launch_bounds__(Cfg<T, D, G>::kThreads, 1)
             chunk = mt.x / (p.B * p.Hkv);
             b = bh / p.Hkv;
             kvh = bh % p.Hkv;
-            load_query<T, C>(st, p, b, kvh * G + hw * C::GW, li);
+            st.load_query(p, b, kvh * G + hw * C::GW, lane);
         }
         if (mt.z > 0) {
-            const char* ks = reinterpret_cast<const char*>(smem) + s * C::kStageBytes;
-            consume_tile<T, C>(st, ks, ks + C::kTileBytes, mt.z, lane);
+            char* ks = reinterpret_cast<char*>(smem) + s * C::kStageBytes;
+            st.tile(ks, ks + C::kTileBytes, mt.z, lane, p.qscale);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(empty_bar + s);
         if (!(mt.w & kLastTileFlag)) continue;
 
         // ---- end of this item: combine the warps' states into one partial.
-        const unsigned fm = 0xffffffffu;
-#pragma unroll
-        for (int h = 0; h < C::GW; ++h) {
-            float l = st.l[h];
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) l += __shfl_xor_sync(fm, l, o);
-            st.l[h] = l;
-#pragma unroll
-            for (int j = 0; j < C::kLanePairs; ++j) {
-                float2 v = st.o[h][j];
-                v.x += __shfl_xor_sync(fm, v.x, 8);
-                v.y += __shfl_xor_sync(fm, v.y, 8);
-                v.x += __shfl_xor_sync(fm, v.x, 16);
-                v.y += __shfl_xor_sync(fm, v.y, 16);
-                st.o[h][j] = v;
-            }
-        }
-        if (items_done > 0 &&
-            !wait_warp(free_bar, (items_done - 1) & 1, abort, p, lane)) {
-            ok = false;
-            break;
-        }
-        float* slot = deposit + (hw * C::NTW + tw) * C::kSlotFloats;
-#pragma unroll
-        for (int h = 0; h < C::GW; ++h) {
-            float* hs = slot + h * (D + 2);
-            if (lane == 0) {
-                hs[0] = st.m[h];
-                hs[1] = st.l[h];
-            }
-            if (lane < 8) {
-#pragma unroll
-                for (int c = 0; c < C::kChunks; ++c)
-#pragma unroll
-                    for (int j = 0; j < C::kPairs; ++j) {
-                        const int e = c * C::kElemPer128 + li * C::kElemPerChunk + 2 * j;
-                        *reinterpret_cast<float2*>(hs + 2 + e) = st.o[h][c * C::kPairs + j];
-                    }
-            }
-        }
+        if (items_done > 0 && !wait_warp(free_bar, (items_done - 1) & 1, abort, p, lane)) break;
+        st.deposit(deposit + (hw * C::NTW + tw) * C::kSlotFloats, lane);
         __syncwarp();
         if (lane == 0) mbar_arrive(dep_bar);
-        if (!wait_warp(dep_bar, items_done & 1, abort, p, lane)) {
-            ok = false;
-            break;
-        }
+        if (!wait_warp(dep_bar, items_done & 1, abort, p, lane)) break;
         {
             const int ctid = warp * 32 + lane;
             float* part_ml = SPEC ? p.spart_ml : p.mid_ml;
@@ -637,19 +853,16 @@ __global__ void __launch_bounds__(Cfg<T, D, G>::kThreads, 1)
         if (SPEC) __threadfence();
         __syncwarp();
         if (lane == 0) mbar_arrive(free_bar);
-        reset_state(st);
+        st.reset();
         ++items_done;
         if (!SPEC) continue;
 
         // ---- sink-set kernel: the CTA finishing last for (b, kv head)
         // merges every item of that head into O_spec.
-        if (!wait_warp(free_bar, (items_done - 1) & 1, abort, p, lane)) {
-            ok = false;
-            break;
-        }
+        if (!wait_warp(free_bar, (items_done - 1) & 1, abort, p, lane)) break;
         if (warp == 0 && lane == 0) {
             const SeqGeom g = seq_geom(p, b, false);
-            const int nch = (g.nspec + p.c1 - 1) / p.c1;
+            const int nch = cdiv(spec_tiles(g, TT), p.c1 / TT);
             unsigned* ticket = p.ctr + kCtrFixed + b * p.Hkv + kvh;
             const unsigned t = atomicAdd(ticket, 1u);
             sh->last = (t == (unsigned)(nch - 1)) ? nch : 0;
@@ -657,25 +870,32 @@ __global__ void __launch_bounds__(Cfg<T, D, G>::kThreads, 1)
             __threadfence();
             mbar_arrive(tk_bar);
         }
-        if (!wait_warp(tk_bar, 0, abort, p, lane)) {
-            ok = false;
-            break;
-        }
+        if (!wait_warp(tk_bar, 0, abort, p, lane)) break;
         const int nch = sh->last;
         if (nch > 0) {
+            // Stage every item's (m, l) in shared memory (the deposit area is
+            // free now), then each thread merges its outputs.
+            float2* ml = reinterpret_cast<float2*>(deposit);
             const int ctid = warp * 32 + lane;
+            for (int i = ctid; i < G * nch; i += C::NCW * 32) {
+                const size_t r = ((size_t)b * p.Hq + kvh * G + i / nch) * p.n1 + i % nch;
+                ml[i] = __ldcg(reinterpret_cast<const float2*>(p.spart_ml) + r);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(dep_bar);
+            if (!wait_warp(dep_bar, items_done & 1, abort, p, lane)) break;
             for (int idx = ctid; idx < G * D; idx += C::NCW * 32) {
                 const int hh = idx / D;
                 const int e = idx % D;
                 const size_t bh = (size_t)b * p.Hq + kvh * G + hh;
                 float M = -INFINITY;
-                for (int c = 0; c < nch; ++c) M = fmaxf(M, __ldcg(p.spart_ml + (bh * p.n1 + c) * 2));
+                for (int c = 0; c < nch; ++c) M = fmaxf(M, ml[hh * nch + c].x);
                 float L = 0.f, O = 0.f;
+#pragma unroll 8
                 for (int c = 0; c < nch; ++c) {
-                    const size_t r = bh * p.n1 + c;
-                    const float f = merge_weight(__ldcg(p.spart_ml + r * 2), M);
-                    L = fmaf(f, __ldcg(p.spart_ml + r * 2 + 1), L);
-                    O = fmaf(f, __ldcg(p.spart_o + r * D + e), O);
+                    const float f = merge_weight(ml[hh * nch + c].x, M);
+                    L = fmaf(f, ml[hh * nch + c].y, L);
+                    O = fmaf(f, __ldcg(p.spart_o + (bh * p.n1 + c) * D + e), O);
                 }
                 if (e == 0) {
                     p.spec_ml[bh * 2] = M;
@@ -687,7 +907,6 @@ __global__ void __launch_bounds__(Cfg<T, D, G>::kThreads, 1)
         }
         // A sink-set CTA owns exactly one item; its end marker follows.
     }
-    (void)ok;
 }
 
 // ------------------------------------------------------- merge + verify
@@ -705,24 +924,37 @@ __global__ void __launch_bounds__(D) merge_kernel(const __grid_constant__ Params
     const int b = blockIdx.y;
     const int e = threadIdx.x;
     const SeqGeom g = seq_geom(p, b, false);
-    const int nmid = (g.mid_len + p.c2 - 1) / p.c2;
+    const int nmid = cdiv(g.mid_len, p.c2);
     const size_t bh = (size_t)b * p.Hq + h;
+    const float2* mid_ml = reinterpret_cast<const float2*>(p.mid_ml) + bh * p.n2;
+    const float* mid_o = p.mid_o + bh * p.n2 * D + e;
+    __shared__ float red[2][D / 32];
 
-    const float ms = p.spec_ml[bh * 2];
-    const float ls = p.spec_ml[bh * 2 + 1];
+    const float2 sml = *reinterpret_cast<const float2*>(p.spec_ml + bh * 2);
     const float os = p.spec_o[bh * D + e];
-    const float o_spec = __fdiv_rn(os, ls);
+    const float o_spec = __fdiv_rn(os, sml.y);
 
-    float M = ms;
-    for (int c = 0; c < nmid; ++c) M = fmaxf(M, p.mid_ml[(bh * p.n2 + c) * 2]);
-    const float f0 = merge_weight(ms, M);
+    // Merged max: every thread takes a strided share of the middle partials,
+    // then a block reduction.
+    float M = sml.x;
+    for (int c = e; c < nmid; c += D) M = fmaxf(M, __ldg(&mid_ml[c].x));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    if ((e & 31) == 0) red[0][e >> 5] = M;
+    __syncthreads();
+#pragma unroll
+    for (int w = 0; w < D / 32; ++w) M = fmaxf(M, red[0][w]);
+    __syncthreads();
+
+    const float f0 = merge_weight(sml.x, M);
     float acc = f0 * os;
-    float lsum = f0 * ls;
+    float lsum = f0 * sml.y;
+#pragma unroll 8
     for (int c = 0; c < nmid; ++c) {
-        const size_t r = bh * p.n2 + c;
-        const float f = merge_weight(p.mid_ml[r * 2], M);
-        lsum = fmaf(f, p.mid_ml[r * 2 + 1], lsum);
-        acc = fmaf(f, p.mid_o[r * D + e], acc);
+        const float2 ml = __ldg(&mid_ml[c]);
+        const float f = merge_weight(ml.x, M);
+        lsum = fmaf(f, ml.y, lsum);
+        acc = fmaf(f, __ldg(mid_o + (size_t)c * D), acc);
     }
     const float o_exact = __fdiv_rn(acc, lsum);
     p.out_exact[bh * D + e] = o_exact;
@@ -735,7 +967,6 @@ __global__ void __launch_bounds__(D) merge_kernel(const __grid_constant__ Params
         dd += __shfl_xor_sync(0xffffffffu, dd, o);
         nn += __shfl_xor_sync(0xffffffffu, nn, o);
     }
-    __shared__ float red[2][D / 32];
     if ((e & 31) == 0) {
         red[0][e >> 5] = dd;
         red[1][e >> 5] = nn;

@@ -59,9 +59,17 @@ def test_workspace_size_and_plan():
     mid = 131072 - 4 - 1024
     assert plan["n2"] * plan["c2"] >= mid > (plan["n2"] - 1) * plan["c2"]
     assert 0 < plan["smem"] <= 227 * 1024 and plan["threads"] % 32 == 0
-    # A fixed split size is honoured (rounded to the 16-token tile).
+    # A fixed split size is honoured, rounded up to the engine's tile:
+    # 32 tokens for the tensor-core engine, 16 for the CUDA-core engine.
     st, plan = sfd.alspec_query_plan(desc(split_tokens=1000), 4, 1024)
-    assert st == 0 and plan["c2"] == 1008
+    assert st == 0 and plan["engine"] == ab.ALSPEC_ENGINE_TENSOR_CORES and plan["c2"] == 1024
+    st, plan = sfd.alspec_query_plan(desc(split_tokens=1000, engine="cuda_cores"), 4, 1024)
+    assert st == 0 and plan["engine"] == ab.ALSPEC_ENGINE_CUDA_CORES and plan["c2"] == 1008
+    # fp32 caches have no tensor-core engine.
+    st, _ = sfd.alspec_query_plan(desc(dtype="f32", engine="tensor_cores"), 4, 1024)
+    assert st == ab.ALSPEC_ERR_UNSUPPORTED
+    st, plan = sfd.alspec_query_plan(desc(dtype="f32"), 4, 1024)
+    assert st == 0 and plan["engine"] == ab.ALSPEC_ENGINE_CUDA_CORES
     # Whole cache inside the sink set: no middle items at all.
     st, plan = sfd.alspec_query_plan(desc(max_seq_len=1000), 4, 1024)
     assert st == 0 and plan["n2"] == 0
@@ -74,6 +82,8 @@ def test_workspace_size_and_plan():
     (dict(batch=0), 4, 8, ab.ALSPEC_ERR_INVALID_ARG),
     (dict(max_seq_len=0), 4, 8, ab.ALSPEC_ERR_INVALID_ARG),
     (dict(dtype=7), 4, 8, ab.ALSPEC_ERR_INVALID_ARG),
+    (dict(engine=3), 4, 8, ab.ALSPEC_ERR_INVALID_ARG),
+    (dict(max_seq_len=1 << 29), 4, 8, ab.ALSPEC_ERR_UNSUPPORTED),  # rows >= 2^31
     (dict(), 0, 0, ab.ALSPEC_ERR_INVALID_ARG),                  # empty sink set
     (dict(), -1, 8, ab.ALSPEC_ERR_INVALID_ARG),
 ])

@@ -25,20 +25,32 @@ def _small(i):
     }[i]
 
 
-@pytest.mark.parametrize("cfg", [0, 1, 2, 3, 4])
-def test_small_configs(cuda_device, cfg):
+@pytest.mark.parametrize("cfg,engine", [(0, "auto"), (1, "auto"), (2, "auto"), (3, "auto"),
+                                        (4, "auto"), (1, "cuda_cores"), (4, "cuda_cores")])
+def test_small_configs(cuda_device, cfg, engine):
     wl = _small(cfg)
     for layer in range(3 if cfg == 2 else 1):
         data = workloads.make_layer(wl, layer=layer, device=cuda_device, poison_tail=True)
-        dec, out = gpu_decode(wl, data, cuda_device)
+        dec, out = gpu_decode(wl, data, cuda_device, engine=engine)
         ref = oracle_decode(wl, data)
-        assert_parity(out, ref, wl.lam, what=f"cfg{cfg} layer{layer}")
+        assert_parity(out, ref, wl.lam, what=f"cfg{cfg} layer{layer} {engine}")
         st, err = dec.device_error()
         assert st == 0 and err == 0
 
 
+def test_engines_agree(cuda_device):
+    """Tensor-core and CUDA-core engines on the same bf16 inputs."""
+    wl = _small(1)
+    data = workloads.make_layer(wl, device=cuda_device)
+    _, a = gpu_decode(wl, data, cuda_device, engine="tensor_cores")
+    _, b = gpu_decode(wl, data, cuda_device, engine="cuda_cores")
+    from parity import per_head_rel
+    for name in ("out_spec", "out_exact"):
+        assert per_head_rel(a[name].double().numpy(), b[name].double().numpy()).max() < 1e-3
+
+
 def test_commit_variant_gives_both_flags(cuda_device):
-    wl = workloads.COMMIT_VARIANT.replace(B=8, L=8192, ragged=(6000, 8192))
+    wl = workloads.COMMIT_VARIANT.replace(L=8192, ragged=(6000, 8192))
     data = workloads.make_layer(wl, device=cuda_device)
     _, out = gpu_decode(wl, data, cuda_device)
     ref = oracle_decode(wl, data)
@@ -47,16 +59,19 @@ def test_commit_variant_gives_both_flags(cuda_device):
 
 
 EDGE = []
-for dtype, d in (("f32", 64), ("bf16", 64), ("bf16", 128), ("f32", 128)):
+for dtype, d, engine in (("f32", 64, "cuda_cores"), ("bf16", 64, "cuda_cores"),
+                         ("bf16", 128, "cuda_cores"), ("f32", 128, "cuda_cores"),
+                         ("bf16", 64, "tensor_cores"), ("bf16", 128, "tensor_cores")):
     for g in (1, 2, 4, 8):
-        EDGE.append((dtype, d, g))
+        EDGE.append((dtype, d, g, engine))
 
 
-@pytest.mark.parametrize("dtype,d,g", EDGE)
-def test_edge_lengths(cuda_device, dtype, d, g):
-    """L = 1, L < S, L = S + W, L = S + W + 1, W = 0, S = 0, ragged tails."""
+@pytest.mark.parametrize("dtype,d,g,engine", EDGE)
+def test_edge_lengths(cuda_device, dtype, d, g, engine):
+    """L = 1, L < S, L = S + W, L = S + W + 1, W = 0, S = 0, ragged tails,
+    sink and window runs longer than a tile."""
     Hkv = 2
-    for S, W in ((4, 16), (0, 16), (4, 0), (1, 1)):
+    for S, W in ((4, 16), (0, 16), (4, 0), (1, 1), (40, 70)):
         lens = sorted({1, 3, S + W, S + W + 1, 37, 250, 16 * 9 + 5})
         lens = [L for L in lens if L >= 1]
         wl = workloads.Workload("edge", B=len(lens), Hq=g * Hkv, Hkv=Hkv, d=d, L=max(lens), S=S,
@@ -64,9 +79,9 @@ def test_edge_lengths(cuda_device, dtype, d, g):
         data = workloads.make_layer(wl, device=cuda_device)
         data["lens"] = lens
         data["seq_lens"] = torch.tensor(lens, dtype=torch.int32, device=cuda_device)
-        _, out = gpu_decode(wl, data, cuda_device)
+        _, out = gpu_decode(wl, data, cuda_device, engine=engine)
         ref = oracle_decode(wl, data)
-        assert_parity(out, ref, wl.lam, what=f"{dtype} d{d} g{g} S{S} W{W}")
+        assert_parity(out, ref, wl.lam, what=f"{dtype} d{d} g{g} S{S} W{W} {engine}")
         for b, L in enumerate(lens):
             if L <= S + W:
                 assert torch.equal(out["out_spec"][b], out["out_exact"][b])
@@ -88,9 +103,10 @@ def test_split_sizes_agree(cuda_device):
     wl = _small(3)
     data = workloads.make_layer(wl, device=cuda_device)
     ref = oracle_decode(wl, data)
-    for split in (16, 112, 1024, 100000):
-        _, out = gpu_decode(wl, data, cuda_device, split_tokens=split)
-        assert_parity(out, ref, wl.lam, what=f"split {split}")
+    for engine in ("tensor_cores", "cuda_cores"):
+        for split in (16, 112, 1024, 100000):
+            _, out = gpu_decode(wl, data, cuda_device, split_tokens=split, engine=engine)
+            assert_parity(out, ref, wl.lam, what=f"split {split} {engine}")
 
 
 def test_bad_seq_lens_are_clamped_and_flagged(cuda_device):

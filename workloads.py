@@ -91,11 +91,12 @@ CONFIGS = {
 }
 
 # Supplementary variant (not one of the five): stronger sinks so that the
-# approximation is accurate when no needle is present, giving a mixed
-# commit/discard outcome.  Same shapes as workload 1.
-COMMIT_VARIANT = CONFIGS[1].replace(name="llama8b-layer-32k-commit", seed=20259,
-                                    sink_bump=24.0, needle_bump=32.0,
-                                    needles=("kv_frac", 0.25))
+# approximation is accurate where no needle is present, and needles in only
+# 1/16 of the (sequence, KV head) pairs, so a batch mixes commit and discard.
+# Llama-3.1-8B head shapes, batch 8, ragged 24K-32K.
+COMMIT_VARIANT = CONFIGS[1].replace(name="llama8b-b8-32k-commit", B=8, seed=20259,
+                                    ragged=(24576, 32768), sink_bump=24.0, needle_bump=32.0,
+                                    needles=("pair_frac", 0.0625))
 
 
 def layer_seed(wl: Workload, layer: int) -> int:
