@@ -322,12 +322,16 @@ def run_alspec(args, wl):
     per_step = [step_marks[i].elapsed_time(step_marks[i + 1]) for i in range(args.steps)]
 
     # Per-layer profiling events of every timed step.
-    mid_ms, spec_ms, layer_ms = [], [], []
+    mid_ms, spec_ms, layer_ms, pre_ms, post_ms, gap_ms = [], [], [], [], [], []
     for ev in step_events:
-        for e in ev:
+        for i, e in enumerate(ev):
             mid_ms.append(e[2].elapsed_time(e[3]))
             spec_ms.append(e[0].elapsed_time(e[1]))
             layer_ms.append(e[0].elapsed_time(e[4]))
+            pre_ms.append(e[0].elapsed_time(e[2]))
+            post_ms.append(e[3].elapsed_time(e[4]))
+            if i + 1 < len(ev):
+                gap_ms.append(e[4].elapsed_time(ev[i + 1][0]))
     hit_rate = float(commit_all.float().mean().item())
     st, err = dec.device_error(stream)
     assert st == 0 and err == 0, f"device error word {err:#x}"
@@ -423,6 +427,11 @@ def run_alspec(args, wl):
         "spec_latency": {"us_median": statistics.median(spec_ms) * 1e3,
                          "ratio_to_layer_median": statistics.median(spec_ratio),
                          "layer_us_median": statistics.median(layer_ms) * 1e3},
+        "layer_breakdown_us_median": {
+            "start_to_middle_kernel": statistics.median(pre_ms) * 1e3,
+            "middle_kernel": statistics.median(mid_ms) * 1e3,
+            "middle_end_to_layer_end": statistics.median(post_ms) * 1e3,
+            "between_layers": statistics.median(gap_ms) * 1e3 if gap_ms else None},
         "hit_rate": hit_rate,
         "cpu_baseline": cpu,
         "e2e": e2e,

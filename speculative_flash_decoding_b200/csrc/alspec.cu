@@ -179,7 +179,7 @@ void make_plan(const alspec_desc& d, int S, int W, int sms, Plan* pl) {
         off = align_up(off + bytes, kAlign);
         return o;
     };
-    pl->off_ctr = take((kCtrFixed + B * d.n_kv_heads + B) * sizeof(unsigned));
+    pl->off_ctr = take((size_t)ctr_words(d.batch, d.n_kv_heads) * sizeof(unsigned));
     pl->off_spart_ml = take(B * Hq * n1 * 2 * sizeof(float));
     pl->off_spart_o = take(B * Hq * n1 * D * sizeof(float));
     pl->off_spec_ml = take(B * Hq * 2 * sizeof(float));
@@ -426,12 +426,9 @@ alspec_status alspec_decode(const alspec_desc* desc, const void* q, const void* 
             return st;
     }
     if (!prof(3, s)) return ALSPEC_ERR_CUDA;
-    // Join, then merge + relative L2 + flag.
+    // Join: O_exact, rel_l2 and the flag are written by whichever of the two
+    // kernels completes a head group last.
     if (!ok(cudaStreamWaitEvent(s, ds->join, 0))) return ALSPEC_ERR_CUDA;
-    KernelFn mk = desc->head_dim == 128 ? merge_kernel<128> : merge_kernel<64>;
-    if ((st = launch(mk, dim3(desc->n_q_heads, desc->batch), dim3(desc->head_dim), 0, s, p, false,
-                     0)) != ALSPEC_OK)
-        return st;
     if (!prof(4, s)) return ALSPEC_ERR_CUDA;
     return ALSPEC_OK;
 }

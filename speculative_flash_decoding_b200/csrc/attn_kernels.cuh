@@ -16,8 +16,12 @@
 //     items in the CTA that finishes last and writes O_spec;
 //   * the middle kernel (MID) is persistent: CTAs pull items from an atomic
 //     queue and stream the cache through shared memory;
-//   * the merge kernel combines the sink-set partial with the middle
-//     partials into O_exact, then computes rel_l2 and the flag.
+//   * whichever CTA -- of either kernel -- completes the last piece of a
+//     (sequence, KV head) merges the sink-set partial with the middle
+//     partials into O_exact for that head group, and the warp completing the
+//     last head of a sequence computes rel_l2 and the commit flag.  Both
+//     kernels only count completions with atomics; nothing waits on the
+//     other kernel.
 //
 // Inside a CTA one producer lane fills a ring of shared-memory stages with
 // K and V tiles through the TMA engine (mbarrier completion); consumer warps
@@ -53,15 +57,38 @@ namespace alspec {
 
 constexpr int kSmemLimit = 227 * 1024;
 
+// Stages per token slot of the tensor-core middle kernel: 2 slots of 16 KB
+// per consumer warp keep ~128 KB in flight per SM, enough for the HBM
+// bandwidth-latency product without queueing loads longer than necessary.
+#ifndef ALSPEC_MID_SPW
+#define ALSPEC_MID_SPW 2
+#endif
+
 constexpr unsigned kErrSeqLen = 1u;   // ALSPEC_DEVERR_SEQ_LEN
 constexpr unsigned kErrTimeout = 2u;  // ALSPEC_DEVERR_TIMEOUT
 
-// Counter words at the head of the workspace; the sink-set tickets
-// [B * Hkv] and merge tickets [B] follow.
+// Counter words at the head of the workspace.  Then, per (sequence, KV
+// head), the sink-set item tickets [B * Hkv] and the completion tickets
+// [B * Hkv]; then the per-sequence head tickets [B].  Whoever takes the last
+// ticket of a group resets it, so the words are zero between calls.
 constexpr int kCtrQueue = 0;
 constexpr int kCtrDone = 1;
 constexpr int kCtrError = 2;
 constexpr int kCtrFixed = 4;
+
+__host__ __device__ __forceinline__ int ctr_spec(int B, int Hkv, int b, int kvh) {
+    (void)B;
+    return kCtrFixed + b * Hkv + kvh;
+}
+__host__ __device__ __forceinline__ int ctr_fin(int B, int Hkv, int b, int kvh) {
+    return kCtrFixed + B * Hkv + b * Hkv + kvh;
+}
+__host__ __device__ __forceinline__ int ctr_seq(int B, int Hkv, int b) {
+    return kCtrFixed + 2 * B * Hkv + b;
+}
+__host__ __device__ __forceinline__ int ctr_words(int B, int Hkv) {
+    return kCtrFixed + 2 * B * Hkv + B;
+}
 
 constexpr int kLastTileFlag = 1;
 
@@ -232,7 +259,7 @@ struct Cfg {
     static constexpr int kStageBytes = 2 * kTileBytes;
     static constexpr int kSlotFloats = GW * (D + 2);
     static constexpr int kDepositBytes = NCW * kSlotFloats * 4;
-    static constexpr int kSpwMax = SPEC ? 1 : (MMA ? 3 : 4);
+    static constexpr int kSpwMax = SPEC ? 3 : (MMA ? ALSPEC_MID_SPW : 4);
     static constexpr int kSpwBudget =
         (kSmemLimit - 1024 - kDepositBytes - 4096) / (NTW * kStageBytes);
     static constexpr int SPW = kSpwBudget < 1 ? 1 : (kSpwBudget > kSpwMax ? kSpwMax : kSpwBudget);
@@ -241,7 +268,7 @@ struct Cfg {
     static constexpr int kOffDeposit = STAGES * kStageBytes;
     static constexpr int kOffMeta = kOffDeposit + kDepositBytes;
     static constexpr int kOffBar = kOffMeta + STAGES * 16;
-    static constexpr int kNumBars = 2 * STAGES + 3;
+    static constexpr int kNumBars = 2 * STAGES + 4;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
     static_assert(kRowBytes % 128 == 0, "row must be a multiple of 128 bytes");
@@ -657,6 +684,101 @@ struct EngineOf<C, T, D, G, true> {
     using type = MmaEngine<C, D, G>;
 };
 
+// ------------------------------------------------------- merge + verify
+
+// Final merge for the G query heads of (sequence b, KV head kvh), run by the
+// consumer warps of the CTA that completed the group's last piece; warp w
+// takes heads w, w + nwarps, ...  O_exact merges the sink-set partial with
+// the nmid middle partials; O_spec is rebuilt from the same sink-set partial
+// with the same division, so the two are bit-identical when the middle is
+// empty.  Each head's squared distance and squared norm are reduced in a
+// fixed order; the warp that completes the last head of the sequence sums
+// them over heads (fixed order, fp64) and writes rel_l2 and the flag.
+template <int D, int G>
+__device__ __noinline__ void finish_group(const Params& p, int b, int kvh, int nmid, int warp,
+                                          int nwarps, int lane) {
+    constexpr int E = D / 32;  // output elements per lane
+    const unsigned full = 0xffffffffu;
+    int mine = 0;
+    for (int hh = warp; hh < G; hh += nwarps, ++mine) {
+        const size_t bh = (size_t)b * p.Hq + kvh * G + hh;
+        const float2 sml = __ldcg(reinterpret_cast<const float2*>(p.spec_ml) + bh);
+        const float2* mml = reinterpret_cast<const float2*>(p.mid_ml) + bh * p.n2;
+        float M = sml.x;
+        for (int c = lane; c < nmid; c += 32) M = fmaxf(M, __ldcg(&mml[c].x));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(full, M, o));
+        const float f0 = merge_weight(sml.x, M);
+        float os[E], acc[E];
+        float lsum = f0 * sml.y;
+#pragma unroll
+        for (int i = 0; i < E; ++i) {
+            os[i] = __ldcg(p.spec_o + bh * D + lane + 32 * i);
+            acc[i] = f0 * os[i];
+        }
+        const float* mo = p.mid_o + bh * p.n2 * D + lane;
+#pragma unroll 4
+        for (int c = 0; c < nmid; ++c) {
+            const float2 ml = __ldcg(&mml[c]);
+            const float f = merge_weight(ml.x, M);
+            lsum = fmaf(f, ml.y, lsum);
+#pragma unroll
+            for (int i = 0; i < E; ++i) acc[i] = fmaf(f, __ldcg(mo + (size_t)c * D + 32 * i), acc[i]);
+        }
+        float dd = 0.f, nn = 0.f;
+#pragma unroll
+        for (int i = 0; i < E; ++i) {
+            const float o_spec = __fdiv_rn(os[i], sml.y);
+            const float o_exact = __fdiv_rn(acc[i], lsum);
+            p.out_exact[bh * D + lane + 32 * i] = o_exact;
+            const float diff = o_exact - o_spec;
+            dd = fmaf(diff, diff, dd);
+            nn = fmaf(o_exact, o_exact, nn);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            dd += __shfl_xor_sync(full, dd, o);
+            nn += __shfl_xor_sync(full, nn, o);
+        }
+        if (lane == 0) *reinterpret_cast<float2*>(p.dn + bh * 2) = make_float2(dd, nn);
+    }
+    if (mine == 0) return;
+    // Count this warp's heads towards the sequence.
+    int last = 0;
+    if (lane == 0) {
+        __threadfence();
+        unsigned* word = p.ctr + ctr_seq(p.B, p.Hkv, b);
+        const unsigned t = atomicAdd(word, (unsigned)mine);
+        last = t + (unsigned)mine == (unsigned)p.Hq;
+        if (last) {
+            atomicExch(word, 0u);
+            __threadfence();
+        }
+    }
+    if (!__shfl_sync(full, last, 0)) return;
+    double D2 = 0.0, N2 = 0.0;
+    for (int h = lane; h < p.Hq; h += 32) {
+        const float2 v = __ldcg(reinterpret_cast<const float2*>(p.dn) + (size_t)b * p.Hq + h);
+        D2 += (double)v.x;
+        N2 += (double)v.y;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        D2 += __shfl_xor_sync(full, D2, o);
+        N2 += __shfl_xor_sync(full, N2, o);
+    }
+    if (lane == 0) {
+        double r;
+        if (N2 == 0.0) {
+            r = D2 == 0.0 ? 0.0 : (double)INFINITY;
+        } else {
+            r = sqrt(D2 / N2);
+        }
+        p.rel_l2[b] = (float)r;
+        p.commit[b] = r <= (double)p.lambda ? 1 : 0;
+    }
+}
+
 // ------------------------------------------------------------ the kernel
 
 template <typename T, int D, int G, bool SPEC, bool MMA>
@@ -672,8 +794,8 @@ __global__ void __launch_bounds__(Cfg<T, D, G, SPEC, MMA>::kThreads, 1)
     int4* meta = reinterpret_cast<int4*>(smem + C::kOffMeta);
     uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
     uint64_t* empty_bar = full_bar + C::STAGES;
-    uint64_t* dep_bar = empty_bar + C::STAGES;  // warps deposited their state
-    uint64_t* free_bar = dep_bar + 1;           // warps finished the merge
+    uint64_t* dep_bar = empty_bar + C::STAGES;  // consumer warps: phase sync
+    uint64_t* free_bar = dep_bar + 1;           // consumer warps: writes done
     uint64_t* tk_bar = dep_bar + 2;             // ticket result published
     Shared* sh = reinterpret_cast<Shared*>(smem + C::kOffMisc);
     volatile int* abort = &sh->abort;
@@ -792,15 +914,43 @@ __global__ void __launch_bounds__(Cfg<T, D, G, SPEC, MMA>::kThreads, 1)
     const int tw = warp % C::NTW;   // which token slot of the round
     Engine st;
     st.reset();
+    // Phase counters of the consumer-only barriers (all consumer warps run
+    // the same sequence of syncs, so the counters agree across warps).
+    uint32_t ph_dep = 0, ph_free = 0, ph_tk = 0;
+    auto sync_on = [&](uint64_t* bar, uint32_t& ph) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar);
+        return wait_warp(bar, (ph++) & 1, abort, p, lane);
+    };
+    // Ticket taken by one thread; the result reaches every consumer warp.
+    auto ticket = [&](unsigned* word, unsigned total) {
+        if (warp == 0 && lane == 0) {
+            const unsigned t = atomicAdd(word, 1u);
+            const int last = t == total - 1;
+            if (last) atomicExch(word, 0u);
+            __threadfence();
+            sh->last = last;
+            mbar_arrive(tk_bar);
+        }
+        if (!wait_warp(tk_bar, (ph_tk++) & 1, abort, p, lane)) return -1;
+        return sh->last;
+    };
     uint32_t gt = tw;
-    int items_done = 0;
     int b = 0, kvh = 0, chunk = 0;
+    if (SPEC) {
+        // The item is known up front: fetch q while the first tiles load.
+        const int bh = (int)blockIdx.x % (p.B * p.Hkv);
+        chunk = (int)blockIdx.x / (p.B * p.Hkv);
+        b = bh / p.Hkv;
+        kvh = bh % p.Hkv;
+        st.load_query(p, b, kvh * G + hw * C::GW, lane);
+    }
     for (;; gt += C::NTW) {
         const int s = gt % C::STAGES;
         if (!wait_warp(full_bar + s, (gt / C::STAGES) & 1, abort, p, lane)) break;
         const int4 mt = meta[s];
         if (mt.x < 0) break;
-        if (mt.y < C::NTW) {
+        if (!SPEC && mt.y < C::NTW) {
             const int bh = mt.x % (p.B * p.Hkv);
             chunk = mt.x / (p.B * p.Hkv);
             b = bh / p.Hkv;
@@ -816,11 +966,8 @@ __global__ void __launch_bounds__(Cfg<T, D, G, SPEC, MMA>::kThreads, 1)
         if (!(mt.w & kLastTileFlag)) continue;
 
         // ---- end of this item: combine the warps' states into one partial.
-        if (items_done > 0 && !wait_warp(free_bar, (items_done - 1) & 1, abort, p, lane)) break;
         st.deposit(deposit + (hw * C::NTW + tw) * C::kSlotFloats, lane);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(dep_bar);
-        if (!wait_warp(dep_bar, items_done & 1, abort, p, lane)) break;
+        if (!sync_on(dep_bar, ph_dep)) break;
         {
             const int ctid = warp * 32 + lane;
             float* part_ml = SPEC ? p.spart_ml : p.mid_ml;
@@ -850,29 +997,21 @@ __global__ void __launch_bounds__(Cfg<T, D, G, SPEC, MMA>::kThreads, 1)
                 part_o[row * D + e] = O;
             }
         }
-        if (SPEC) __threadfence();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(free_bar);
+        __threadfence();
+        // Every consumer thread's partial is written (and the deposit slots
+        // are free again) once this sync passes.
+        if (!sync_on(free_bar, ph_free)) break;
         st.reset();
-        ++items_done;
-        if (!SPEC) continue;
+        const SeqGeom g = seq_geom(p, b, false);
+        const unsigned nmid = (unsigned)cdiv(g.mid_len, p.c2);
 
-        // ---- sink-set kernel: the CTA finishing last for (b, kv head)
-        // merges every item of that head into O_spec.
-        if (!wait_warp(free_bar, (items_done - 1) & 1, abort, p, lane)) break;
-        if (warp == 0 && lane == 0) {
-            const SeqGeom g = seq_geom(p, b, false);
+        if (SPEC) {
+            // ---- the CTA finishing last for (b, kv head) merges every
+            // sink-set item of that head into O_spec.
             const int nch = cdiv(spec_tiles(g, TT), p.c1 / TT);
-            unsigned* ticket = p.ctr + kCtrFixed + b * p.Hkv + kvh;
-            const unsigned t = atomicAdd(ticket, 1u);
-            sh->last = (t == (unsigned)(nch - 1)) ? nch : 0;
-            if (sh->last) atomicExch(ticket, 0u);
-            __threadfence();
-            mbar_arrive(tk_bar);
-        }
-        if (!wait_warp(tk_bar, 0, abort, p, lane)) break;
-        const int nch = sh->last;
-        if (nch > 0) {
+            const int last = ticket(p.ctr + ctr_spec(p.B, p.Hkv, b, kvh), (unsigned)nch);
+            if (last < 0) break;
+            if (!last) continue;
             // Stage every item's (m, l) in shared memory (the deposit area is
             // free now), then each thread merges its outputs.
             float2* ml = reinterpret_cast<float2*>(deposit);
@@ -881,9 +1020,7 @@ __global__ void __launch_bounds__(Cfg<T, D, G, SPEC, MMA>::kThreads, 1)
                 const size_t r = ((size_t)b * p.Hq + kvh * G + i / nch) * p.n1 + i % nch;
                 ml[i] = __ldcg(reinterpret_cast<const float2*>(p.spart_ml) + r);
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(dep_bar);
-            if (!wait_warp(dep_bar, items_done & 1, abort, p, lane)) break;
+            if (!sync_on(dep_bar, ph_dep)) break;
             for (int idx = ctid; idx < G * D; idx += C::NCW * 32) {
                 const int hh = idx / D;
                 const int e = idx % D;
@@ -904,102 +1041,15 @@ __global__ void __launch_bounds__(Cfg<T, D, G, SPEC, MMA>::kThreads, 1)
                 p.spec_o[bh * D + e] = O;
                 p.out_spec[bh * D + e] = __fdiv_rn(O, L);
             }
-        }
-        // A sink-set CTA owns exactly one item; its end marker follows.
-    }
-}
-
-// ------------------------------------------------------- merge + verify
-
-// One CTA per (query head, sequence); thread e owns output element e.
-// O_exact merges the sink-set partial with the sequence's middle partials;
-// O_spec is rebuilt from the same sink-set partial with the same division,
-// so the two are bit-identical when the middle is empty.  The per-head
-// squared distance and squared norm are reduced in a fixed order; the CTA
-// finishing last for the sequence sums them over heads (in head order) and
-// writes rel_l2 and the commit flag.
-template <int D>
-__global__ void __launch_bounds__(D) merge_kernel(const __grid_constant__ Params p) {
-    const int h = blockIdx.x;
-    const int b = blockIdx.y;
-    const int e = threadIdx.x;
-    const SeqGeom g = seq_geom(p, b, false);
-    const int nmid = cdiv(g.mid_len, p.c2);
-    const size_t bh = (size_t)b * p.Hq + h;
-    const float2* mid_ml = reinterpret_cast<const float2*>(p.mid_ml) + bh * p.n2;
-    const float* mid_o = p.mid_o + bh * p.n2 * D + e;
-    __shared__ float red[2][D / 32];
-
-    const float2 sml = *reinterpret_cast<const float2*>(p.spec_ml + bh * 2);
-    const float os = p.spec_o[bh * D + e];
-    const float o_spec = __fdiv_rn(os, sml.y);
-
-    // Merged max: every thread takes a strided share of the middle partials,
-    // then a block reduction.
-    float M = sml.x;
-    for (int c = e; c < nmid; c += D) M = fmaxf(M, __ldg(&mid_ml[c].x));
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    if ((e & 31) == 0) red[0][e >> 5] = M;
-    __syncthreads();
-#pragma unroll
-    for (int w = 0; w < D / 32; ++w) M = fmaxf(M, red[0][w]);
-    __syncthreads();
-
-    const float f0 = merge_weight(sml.x, M);
-    float acc = f0 * os;
-    float lsum = f0 * sml.y;
-#pragma unroll 8
-    for (int c = 0; c < nmid; ++c) {
-        const float2 ml = __ldg(&mid_ml[c]);
-        const float f = merge_weight(ml.x, M);
-        lsum = fmaf(f, ml.y, lsum);
-        acc = fmaf(f, __ldg(mid_o + (size_t)c * D), acc);
-    }
-    const float o_exact = __fdiv_rn(acc, lsum);
-    p.out_exact[bh * D + e] = o_exact;
-
-    const float diff = o_exact - o_spec;
-    float dd = diff * diff;
-    float nn = o_exact * o_exact;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        dd += __shfl_xor_sync(0xffffffffu, dd, o);
-        nn += __shfl_xor_sync(0xffffffffu, nn, o);
-    }
-    if ((e & 31) == 0) {
-        red[0][e >> 5] = dd;
-        red[1][e >> 5] = nn;
-    }
-    __syncthreads();
-    if (e == 0) {
-        float sd = 0.f, sn = 0.f;
-        for (int w = 0; w < D / 32; ++w) {
-            sd += red[0][w];
-            sn += red[1][w];
-        }
-        p.dn[bh * 2] = sd;
-        p.dn[bh * 2 + 1] = sn;
-        __threadfence();
-        unsigned* ticket = p.ctr + kCtrFixed + p.B * p.Hkv + b;
-        const unsigned t = atomicAdd(ticket, 1u);
-        if (t == (unsigned)(p.Hq - 1)) {
-            atomicExch(ticket, 0u);
             __threadfence();
-            double D2 = 0.0, N2 = 0.0;
-            for (int hh = 0; hh < p.Hq; ++hh) {
-                D2 += (double)__ldcg(p.dn + ((size_t)b * p.Hq + hh) * 2);
-                N2 += (double)__ldcg(p.dn + ((size_t)b * p.Hq + hh) * 2 + 1);
-            }
-            double r;
-            if (N2 == 0.0) {
-                r = D2 == 0.0 ? 0.0 : (double)INFINITY;
-            } else {
-                r = sqrt(D2 / N2);
-            }
-            p.rel_l2[b] = (float)r;
-            p.commit[b] = r <= (double)p.lambda ? 1 : 0;
+            if (!sync_on(free_bar, ph_free)) break;
         }
+        // ---- one more piece of (b, kv head) is complete: the sink-set merge
+        // (from the sink-set kernel) or a middle item.  The last of the
+        // 1 + nmid pieces finishes the head group.
+        const int fin = ticket(p.ctr + ctr_fin(p.B, p.Hkv, b, kvh), 1u + nmid);
+        if (fin < 0) break;
+        if (fin) finish_group<D, G>(p, b, kvh, (int)nmid, warp, C::NCW, lane);
     }
 }
 
