@@ -76,9 +76,11 @@ typedef enum {
  * q, k_cache and v_cache share `dtype`.  Supported: head_dim in {64, 128};
  * n_q_heads / n_kv_heads in {1, 2, 4, 8}.
  * batch * n_kv_heads * max_seq_len must stay below 2^31.
- * split_tokens: tokens per work item of the exact-attention split (rounded
- * up to the engine's tile, 16 or 32 tokens); 0 lets the library choose from
- * the GPU's SM count.
+ * split_tokens: tokens per work item of the exact-attention split of the
+ * longest sequence (rounded up to the engine's tile, 16 or 32 tokens;
+ * shorter sequences get proportionally shorter items); 0 lets the library
+ * choose (guided self-scheduling: items shrink towards the end of the
+ * queue; at most 256 items per sequence and KV head).
  */
 typedef struct {
     int batch;
@@ -159,7 +161,8 @@ alspec_status alspec_decode(const alspec_desc* desc,
  * Work plan the library would use (host only, no CUDA call except the SM
  * count query).  info[] receives, in order:
  *   0 tokens per sink-set work item      1 sink-set items per (b, kv head)
- *   2 tokens per exact-path work item    3 exact-path items per (b, kv head)
+ *   2 tokens in the first exact-path item of the longest sequence
+ *   3 exact-path items per (b, kv head)
  *   4 persistent CTAs of the exact path  5 threads per CTA
  *   6 dynamic shared memory per CTA      7 pipeline stages
  *   8 engine (alspec_engine, resolved)
@@ -168,6 +171,18 @@ alspec_status alspec_decode(const alspec_desc* desc,
  */
 alspec_status alspec_query_plan(const alspec_desc* desc, int n_sink, int window,
                                 int* info, int n_info);
+
+/*
+ * Chunk table of the exact-path (middle) split (host only).  The middle of
+ * sequence b -- rows [min(S, L_b), max(min(S, L_b), L_b - W)) -- is tiled in
+ * T-row tiles (T = 32 for the tensor-core engine, 16 for the CUDA-core
+ * engine; *tile receives T); with m_b tiles in it, chunk c covers tiles
+ * [(m_b * fq[c]) >> 24, (m_b * fq[c + 1]) >> 24).  fq receives n2 + 1
+ * entries (fq[0] = 0, fq[n2] = 1 << 24); capacity is the length of fq.
+ * *n2 receives the chunk count.
+ */
+alspec_status alspec_query_chunks(const alspec_desc* desc, int n_sink, int window,
+                                  uint32_t* fq, int capacity, int* n2, int* tile);
 
 /*
  * Read (and clear) the device error word of a workspace: a bitwise OR of

@@ -58,6 +58,8 @@ SIGNATURES = {
                            _vp, _vp, ctypes.POINTER(_vp)]),
     "alspec_query_plan": (_i, [_descp, _i, _i, ctypes.POINTER(_i), _i]),
     "alspec_get_device_error": (_i, [_vp, _sz, _vp, _u32p]),
+    "alspec_query_chunks": (_i, [_descp, _i, _i, _u32p, _i, ctypes.POINTER(_i),
+                                 ctypes.POINTER(_i)]),
     "alspec_graph_begin": (_i, [_vp]),
     "alspec_graph_end": (_i, [_vp, ctypes.POINTER(_vp)]),
     "alspec_graph_launch": (_i, [_vp, _vp]),
@@ -122,6 +124,16 @@ def alspec_query_plan(desc: alspec_desc, n_sink: int, window: int):
     st = int(_lib.alspec_query_plan(ctypes.byref(desc), n_sink, window, info, 9))
     keys = ("c1", "n1", "c2", "n2", "grid2", "threads", "smem", "stages", "engine")
     return st, dict(zip(keys, list(info)))
+
+
+def alspec_query_chunks(desc: alspec_desc, n_sink: int, window: int):
+    """(status, fq list of n2 + 1 fractions in 1/2^24, tile rows)."""
+    cap = 257
+    fq = (ctypes.c_uint32 * cap)()
+    n2, tile = ctypes.c_int(0), ctypes.c_int(0)
+    st = int(_lib.alspec_query_chunks(ctypes.byref(desc), n_sink, window, fq, cap,
+                                      ctypes.byref(n2), ctypes.byref(tile)))
+    return st, list(fq)[: n2.value + 1], tile.value
 
 
 def alspec_get_device_error(workspace: int, workspace_bytes: int, stream: int):

@@ -13,6 +13,7 @@
 #include <mutex>
 #include <set>
 #include <utility>
+#include <vector>
 
 #include "alspec.h"
 #include "attn_kernels.cuh"
@@ -22,6 +23,11 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 constexpr int kMaxSpecItems = 32;  // sink-set items per (sequence, KV head)
+
+// The sink-set kernel gets about 1/ALSPEC_SPEC_SM_DIV of the SMs.
+#ifndef ALSPEC_SPEC_SM_DIV
+#define ALSPEC_SPEC_SM_DIV 4
+#endif
 constexpr size_t kAlign = 256;
 
 thread_local cudaError_t t_last_error = cudaSuccess;
@@ -96,8 +102,10 @@ int sm_count_for_plan() {
 struct Plan {
     int engine;   // ALSPEC_ENGINE_CUDA_CORES or ALSPEC_ENGINE_TENSOR_CORES
     int tt;       // tokens per pipeline tile of that engine
-    int c1, n1, c2, n2;
-    int grid2;
+    int c1, n1;   // sink-set item tokens and items per (sequence, KV head)
+    int c2, n2;   // first middle chunk (tokens, longest sequence) and chunks per head
+    unsigned fq[kMaxChunks + 1];
+    int grid1, grid2;
     int threads, smem, stages;
     size_t off_ctr, off_spart_ml, off_spart_o, off_spec_ml, off_spec_o, off_mid_ml, off_mid_o,
         off_dn, total;
@@ -133,13 +141,18 @@ alspec_status check_desc(const alspec_desc* d, int S, int W) {
 
 void kernel_shape(int dtype, int D, int G, int engine, int* threads, int* smem, int* stages);
 
-// Item sizes: the sink-set list (at most S + W tokens per head, tiled as a
-// sink run and a window run) is cut so that all heads together use about a
-// quarter of the SMs -- few, long CTAs keep the sink-set kernel's fixed costs
-// and its merge short while the middle kernel takes the rest of the GPU; the
-// middle is cut so that the persistent grid (one CTA per SM) gets a couple
-// of items per CTA for a single sequence and more for batches, whose
-// lengths may differ.  Item sizes are multiples of the engine's tile.
+// Item sizes.  The sink-set list (at most S + W tokens per head, tiled as a
+// sink run and a window run) gets one item per head when it is short (at
+// most 64 tiles): that CTA publishes O_spec with no cross-CTA merge.  Long
+// sink sets are cut into a few items, with at most a quarter of the SMs for
+// the sink-set kernel overall.  The persistent middle kernel takes the
+// remaining SMs (at least three quarters), so both kernels start at once.
+// Middle chunks follow guided self-scheduling: with H heads sharing each
+// chunk index and P CTAs, chunk c takes H * r_c / (1.5 P) of what is left
+// of a head's middle (r_c), never less than 16 tiles; chunk boundaries are
+// fractions of each sequence's own middle, so ragged batches get the same
+// number of (proportionally smaller) items.  A caller-given split_tokens
+// instead cuts the longest middle into equal chunks of that size.
 void make_plan(const alspec_desc& d, int S, int W, int sms, Plan* pl) {
     pl->engine = resolve_engine(&d);
     const int TT = pl->engine == ALSPEC_ENGINE_TENSOR_CORES ? 32 : 16;
@@ -147,27 +160,53 @@ void make_plan(const alspec_desc& d, int S, int W, int sms, Plan* pl) {
     const int heads = d.batch * d.n_kv_heads;
     const int L = d.max_seq_len;
     const int tiles_max = ceil_div(std::min(S, L), TT) + ceil_div(std::min(W, L), TT);
-    const int per_head1 = std::min(kMaxSpecItems, std::max(1, sms / 4 / std::max(1, heads)));
-    const int tiles_per_item = std::max(1, ceil_div(tiles_max, per_head1));
+    const int room1 = std::max(1, sms / 4 / std::max(1, heads));
+    pl->n1 = std::min({kMaxSpecItems, room1, ceil_div(tiles_max, 64)});
+    pl->n1 = std::max(1, pl->n1);
+    const int tiles_per_item = ceil_div(tiles_max, pl->n1);
     pl->c1 = tiles_per_item * TT;
     pl->n1 = ceil_div(tiles_max, tiles_per_item);
+    pl->grid1 = heads * pl->n1;
 
     const int ns = std::min(S, L);
     const int mid_max = std::max(0, std::max(ns, L - W) - ns);
-    if (mid_max == 0) {
-        pl->c2 = TT;
-        pl->n2 = 0;
-    } else if (d.split_tokens > 0) {
-        pl->c2 = round_up(d.split_tokens, TT);
-        pl->n2 = ceil_div(mid_max, pl->c2);
-    } else {
-        const int target = (d.batch == 1 ? 2 : 8) * sms;
-        const int per_head2 = std::max(1, ceil_div(target, heads));
-        pl->c2 = round_up(std::max(1, ceil_div(mid_max, per_head2)), TT);
-        pl->n2 = ceil_div(mid_max, pl->c2);
+    const int mid_tiles = ceil_div(mid_max, TT);
+    const int P = std::max(sms - pl->grid1, (3 * sms + 3) / 4);
+    std::vector<double> sizes;  // chunk sizes as fractions of a head's middle
+    if (mid_tiles > 0) {
+        if (d.split_tokens > 0) {
+            const int ct = std::max(1, ceil_div(round_up(d.split_tokens, TT), TT));
+            const int n = std::min(kMaxChunks, ceil_div(mid_tiles, ct));
+            for (int c = 0; c < n; ++c) sizes.push_back((double)ct / mid_tiles);
+        } else {
+            const double smin = std::min(1.0, 16.0 / mid_tiles);
+            double r = 1.0;
+            while (r > 1e-9 && (int)sizes.size() < kMaxChunks) {
+                double s = std::max((double)heads * r / (1.5 * P), smin);
+                s = std::min(s, r);
+                sizes.push_back(s);
+                r -= s;
+            }
+        }
     }
+    pl->n2 = (int)sizes.size();
+    const double scale = (double)(1u << kFracBits);
+    double acc = 0.0;
+    pl->fq[0] = 0;
+    for (int c = 0; c < pl->n2; ++c) {
+        acc += sizes[c];
+        // Rounded up, so that the longest sequence gets its boundaries at
+        // exactly the intended tiles.
+        pl->fq[c + 1] = c + 1 == pl->n2 ? (1u << kFracBits)
+                                         : (unsigned)std::min(scale, std::ceil(acc * scale - 1e-6));
+        pl->fq[c + 1] = std::max(pl->fq[c + 1], pl->fq[c]);
+    }
+    for (int c = pl->n2 + 1; c <= kMaxChunks; ++c) pl->fq[c] = 1u << kFracBits;
+    pl->c2 = pl->n2 > 0
+                 ? (int)(((unsigned long long)mid_tiles * pl->fq[1]) >> kFracBits) * TT
+                 : 0;
     const long long items2 = (long long)heads * pl->n2;
-    pl->grid2 = (int)std::min<long long>(sms, items2);
+    pl->grid2 = (int)std::min<long long>(P, items2);
     const int G = d.n_q_heads / d.n_kv_heads;
     kernel_shape(d.dtype, d.head_dim, G, pl->engine, &pl->threads, &pl->smem, &pl->stages);
 
@@ -340,6 +379,20 @@ alspec_status alspec_query_plan(const alspec_desc* desc, int n_sink, int window,
     return ALSPEC_OK;
 }
 
+alspec_status alspec_query_chunks(const alspec_desc* desc, int n_sink, int window, uint32_t* fq,
+                                  int capacity, int* n2, int* tile) {
+    const alspec_status st = check_desc(desc, n_sink, window);
+    if (st != ALSPEC_OK) return st;
+    if (!fq || !n2 || !tile) return ALSPEC_ERR_INVALID_ARG;
+    Plan pl{};
+    make_plan(*desc, n_sink, window, sm_count_for_plan(), &pl);
+    if (capacity < pl.n2 + 1) return ALSPEC_ERR_INVALID_ARG;
+    for (int c = 0; c <= pl.n2; ++c) fq[c] = pl.fq[c];
+    *n2 = pl.n2;
+    *tile = pl.tt;
+    return ALSPEC_OK;
+}
+
 alspec_status alspec_decode(const alspec_desc* desc, const void* q, const void* k_cache,
                             const void* v_cache, const int32_t* seq_lens, int n_sink, int window,
                             float lambda, float* out_spec, float* out_exact, float* rel_l2,
@@ -385,8 +438,8 @@ alspec_status alspec_decode(const alspec_desc* desc, const void* q, const void* 
     p.lambda = lambda;
     p.c1 = pl.c1;
     p.n1 = pl.n1;
-    p.c2 = pl.c2;
     p.n2 = pl.n2;
+    std::memcpy(p.fq, pl.fq, sizeof p.fq);
     p.ctr = reinterpret_cast<unsigned*>(ws + pl.off_ctr);
     p.spart_ml = reinterpret_cast<float*>(ws + pl.off_spart_ml);
     p.spart_o = reinterpret_cast<float*>(ws + pl.off_spart_o);
@@ -410,7 +463,7 @@ alspec_status alspec_decode(const alspec_desc* desc, const void* q, const void* 
     // Fork: the sink-set kernel runs on the high-priority stream.
     if (!ok(cudaEventRecord(ds->fork, s)) || !ok(cudaStreamWaitEvent(ds->hi, ds->fork, 0)))
         return ALSPEC_ERR_CUDA;
-    const dim3 grid1(desc->batch * desc->n_kv_heads * pl.n1);
+    const dim3 grid1(pl.grid1);
     if ((st = launch(ks.spec, grid1, dim3(ks.threads_spec), ks.smem_spec, ds->hi, p, true,
                      ds->prio_hi)) != ALSPEC_OK)
         return st;
@@ -418,6 +471,9 @@ alspec_status alspec_decode(const alspec_desc* desc, const void* q, const void* 
         return ALSPEC_ERR_CUDA;
     if (!prof(1, ds->hi)) return ALSPEC_ERR_CUDA;
     if (!ok(cudaEventRecord(ds->join, ds->hi))) return ALSPEC_ERR_CUDA;
+#ifdef ALSPEC_SPEC_SERIAL
+    if (!ok(cudaStreamWaitEvent(s, ds->join, 0))) return ALSPEC_ERR_CUDA;
+#endif
     // The middle of every sequence on the caller's stream.
     if (!prof(2, s)) return ALSPEC_ERR_CUDA;
     if (pl.n2 > 0) {

@@ -92,6 +92,13 @@ __host__ __device__ __forceinline__ int ctr_words(int B, int Hkv) {
 
 constexpr int kLastTileFlag = 1;
 
+// Middle work items: every (sequence, KV head) middle is cut at fixed
+// fractions of its length into at most kMaxChunks chunks (guided
+// self-scheduling: large chunks first, shrinking towards the end, so the
+// queue drains on small items and the CTAs finish together).
+constexpr int kMaxChunks = 256;
+constexpr int kFracBits = 24;
+
 struct Params {
     CUtensorMap tmap_k;  // 2-D views [rows = B*Hkv*Lmax, d] (tensor-core engine)
     CUtensorMap tmap_v;
@@ -103,7 +110,9 @@ struct Params {
     float qscale;   // log2(e) / sqrt(d): scores come out in the log2 domain
     float lambda;
     int c1, n1;     // sink-set items: tokens per item, items per (b, kv head)
-    int c2, n2;     // middle items
+    int n2;         // middle chunks per (b, kv head)
+    unsigned fq[kMaxChunks + 1];  // chunk c covers middle tiles
+                                  // [mt * fq[c] >> 24, mt * fq[c+1] >> 24)
     unsigned* ctr;
     float* spart_ml;  // [B][Hq][n1][2]   sink-set item partials
     float* spart_o;   // [B][Hq][n1][D]
@@ -153,6 +162,24 @@ __host__ __device__ __forceinline__ int spec_tiles(const SeqGeom& g, int TT) {
     return cdiv(g.ns, TT) + cdiv(g.L - g.ws, TT);
 }
 
+// Middle tiles [t_lo, t_hi) of chunk c, for a middle of mid_tiles tiles.
+__device__ __forceinline__ void mid_chunk(const Params& p, int mid_tiles, int c, int& t_lo,
+                                          int& t_hi) {
+    t_lo = (int)(((unsigned long long)mid_tiles * p.fq[c]) >> kFracBits);
+    t_hi = (int)(((unsigned long long)mid_tiles * p.fq[c + 1]) >> kFracBits);
+}
+
+// Number of non-empty middle chunks of a middle of mid_tiles tiles.
+__device__ __forceinline__ int mid_pieces(const Params& p, int mid_tiles) {
+    int n = 0, prev = 0;
+    for (int c = 1; c <= p.n2; ++c) {
+        const int t = (int)(((unsigned long long)mid_tiles * p.fq[c]) >> kFracBits);
+        n += t > prev;
+        prev = t;
+    }
+    return n;
+}
+
 // One work item: a range of tiles of one (sequence, KV head).
 struct Item {
     int b, kvh, chunk, ntiles;
@@ -178,9 +205,11 @@ __device__ __forceinline__ Item decode_item(const Params& p, int item, bool flag
         it.ntiles = max(0, t1 - it.t0);
         it.lo = it.hi = 0;
     } else {
-        it.lo = g.ns + it.chunk * p.c2;
-        it.hi = min(it.lo + p.c2, g.ws);
-        it.ntiles = it.hi > it.lo ? cdiv(it.hi - it.lo, TT) : 0;
+        int tlo, thi;
+        mid_chunk(p, cdiv(g.mid_len, TT), it.chunk, tlo, thi);
+        it.lo = g.ns + tlo * TT;
+        it.hi = min(g.ns + thi * TT, g.ws);
+        it.ntiles = thi > tlo ? thi - tlo : 0;
         it.t0 = 0;
     }
     return it;
@@ -694,18 +723,23 @@ struct EngineOf<C, T, D, G, true> {
 // empty.  Each head's squared distance and squared norm are reduced in a
 // fixed order; the warp that completes the last head of the sequence sums
 // them over heads (fixed order, fp64) and writes rel_l2 and the flag.
-template <int D, int G>
-__device__ __noinline__ void finish_group(const Params& p, int b, int kvh, int nmid, int warp,
-                                          int nwarps, int lane) {
+template <int D, int G, int TT>
+__device__ __noinline__ void finish_group(const Params& p, int b, int kvh, int warp, int nwarps,
+                                          int lane) {
     constexpr int E = D / 32;  // output elements per lane
     const unsigned full = 0xffffffffu;
+    const int mid_tiles = cdiv(seq_geom(p, b, false).mid_len, TT);
     int mine = 0;
     for (int hh = warp; hh < G; hh += nwarps, ++mine) {
         const size_t bh = (size_t)b * p.Hq + kvh * G + hh;
         const float2 sml = __ldcg(reinterpret_cast<const float2*>(p.spec_ml) + bh);
         const float2* mml = reinterpret_cast<const float2*>(p.mid_ml) + bh * p.n2;
         float M = sml.x;
-        for (int c = lane; c < nmid; c += 32) M = fmaxf(M, __ldcg(&mml[c].x));
+        for (int c = lane; c < p.n2; c += 32) {
+            int tlo, thi;
+            mid_chunk(p, mid_tiles, c, tlo, thi);
+            if (thi > tlo) M = fmaxf(M, __ldcg(&mml[c].x));
+        }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(full, M, o));
         const float f0 = merge_weight(sml.x, M);
@@ -718,7 +752,10 @@ __device__ __noinline__ void finish_group(const Params& p, int b, int kvh, int n
         }
         const float* mo = p.mid_o + bh * p.n2 * D + lane;
 #pragma unroll 4
-        for (int c = 0; c < nmid; ++c) {
+        for (int c = 0; c < p.n2; ++c) {
+            int tlo, thi;
+            mid_chunk(p, mid_tiles, c, tlo, thi);
+            if (thi <= tlo) continue;  // empty chunk: never written
             const float2 ml = __ldcg(&mml[c]);
             const float f = merge_weight(ml.x, M);
             lsum = fmaf(f, ml.y, lsum);
@@ -989,7 +1026,19 @@ __global__ void __launch_bounds__(Cfg<T, D, G, SPEC, MMA>::kThreads, 1)
                     L = fmaf(f, ws[1], L);
                     O = fmaf(f, ws[2 + e], O);
                 }
-                const size_t row = ((size_t)b * p.Hq + kvh * G + hh) * per + chunk;
+                const size_t bh = (size_t)b * p.Hq + kvh * G + hh;
+                if (SPEC && per == 1) {
+                    // A single sink-set item per head is the whole sink set:
+                    // publish O_spec directly.
+                    if (e == 0) {
+                        p.spec_ml[bh * 2] = M;
+                        p.spec_ml[bh * 2 + 1] = L;
+                    }
+                    p.spec_o[bh * D + e] = O;
+                    p.out_spec[bh * D + e] = __fdiv_rn(O, L);
+                    continue;
+                }
+                const size_t row = bh * per + chunk;
                 if (e == 0) {
                     part_ml[row * 2] = M;
                     part_ml[row * 2 + 1] = L;
@@ -1003,9 +1052,9 @@ __global__ void __launch_bounds__(Cfg<T, D, G, SPEC, MMA>::kThreads, 1)
         if (!sync_on(free_bar, ph_free)) break;
         st.reset();
         const SeqGeom g = seq_geom(p, b, false);
-        const unsigned nmid = (unsigned)cdiv(g.mid_len, p.c2);
+        const unsigned nmid = (unsigned)mid_pieces(p, cdiv(g.mid_len, TT));
 
-        if (SPEC) {
+        if (SPEC && p.n1 > 1) {
             // ---- the CTA finishing last for (b, kv head) merges every
             // sink-set item of that head into O_spec.
             const int nch = cdiv(spec_tiles(g, TT), p.c1 / TT);
@@ -1049,7 +1098,7 @@ __global__ void __launch_bounds__(Cfg<T, D, G, SPEC, MMA>::kThreads, 1)
         // 1 + nmid pieces finishes the head group.
         const int fin = ticket(p.ctr + ctr_fin(p.B, p.Hkv, b, kvh), 1u + nmid);
         if (fin < 0) break;
-        if (fin) finish_group<D, G>(p, b, kvh, (int)nmid, warp, C::NCW, lane);
+        if (fin) finish_group<D, G, TT>(p, b, kvh, warp, C::NCW, lane);
     }
 }
 

@@ -56,8 +56,9 @@ def test_workspace_size_and_plan():
     assert st == 0
     assert plan["c1"] % 16 == 0 and plan["c2"] % 16 == 0
     assert plan["n1"] * plan["c1"] >= 1028 > (plan["n1"] - 1) * plan["c1"]
-    mid = 131072 - 4 - 1024
-    assert plan["n2"] * plan["c2"] >= mid > (plan["n2"] - 1) * plan["c2"]
+    # Middle chunks shrink along the queue (their coverage is checked in
+    # test_plan.py); the first one is the largest.
+    assert 1 <= plan["n2"] <= 256 and plan["c2"] % 32 == 0
     assert 0 < plan["smem"] <= 227 * 1024 and plan["threads"] % 32 == 0
     # A fixed split size is honoured, rounded up to the engine's tile:
     # 32 tokens for the tensor-core engine, 16 for the CUDA-core engine.
