@@ -47,6 +47,9 @@ def parse_args():
                     help="CPU-baseline budget (oracle time) on rank 0")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--split-tokens", type=int, default=0,
+                    help="exact-path item size for the longest sequence (0 = library's choice)")
+    ap.add_argument("--engine", default="auto", choices=["auto", "cuda_cores", "tensor_cores"])
     return ap.parse_args()
 
 
@@ -245,7 +248,8 @@ def run_alspec(args, wl):
         d["q"] = q_all[i]
         d["seq_lens"] = lens_all[i]
     kv_bytes = sum(workloads.kv_bytes(wl, d["lens"]) for d in layers)
-    dec = sfd.Decoder(wl.B, wl.Hq, wl.Hkv, wl.d, wl.L, wl.dtype, wl.S, wl.W, device=device)
+    dec = sfd.Decoder(wl.B, wl.Hq, wl.Hkv, wl.d, wl.L, wl.dtype, wl.S, wl.W, device=device,
+                      split_tokens=args.split_tokens, engine=args.engine)
     plan = dec.plan()
     out_spec = torch.empty(n_layers, wl.B, wl.Hq, wl.d, dtype=torch.float32, device=device)
     out_exact = torch.empty_like(out_spec)

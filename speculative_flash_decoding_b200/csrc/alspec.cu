@@ -482,9 +482,16 @@ alspec_status alspec_decode(const alspec_desc* desc, const void* q, const void* 
             return st;
     }
     if (!prof(3, s)) return ALSPEC_ERR_CUDA;
-    // Join: O_exact, rel_l2 and the flag are written by whichever of the two
-    // kernels completes a head group last.
+    // Join, then merge + relative L2 + flag.
     if (!ok(cudaStreamWaitEvent(s, ds->join, 0))) return ALSPEC_ERR_CUDA;
+    KernelFn mk = nullptr;
+    if (desc->head_dim == 128)
+        mk = pl.tt == 32 ? merge_kernel<128, 32> : merge_kernel<128, 16>;
+    else
+        mk = pl.tt == 32 ? merge_kernel<64, 32> : merge_kernel<64, 16>;
+    if ((st = launch(mk, dim3(desc->n_q_heads, desc->batch), dim3(desc->head_dim * kMergeParts),
+                     0, s, p, false, 0)) != ALSPEC_OK)
+        return st;
     if (!prof(4, s)) return ALSPEC_ERR_CUDA;
     return ALSPEC_OK;
 }

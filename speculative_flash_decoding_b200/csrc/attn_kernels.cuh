@@ -16,12 +16,10 @@
 //     items in the CTA that finishes last and writes O_spec;
 //   * the middle kernel (MID) is persistent: CTAs pull items from an atomic
 //     queue and stream the cache through shared memory;
-//   * whichever CTA -- of either kernel -- completes the last piece of a
-//     (sequence, KV head) merges the sink-set partial with the middle
-//     partials into O_exact for that head group, and the warp completing the
-//     last head of a sequence computes rel_l2 and the commit flag.  Both
-//     kernels only count completions with atomics; nothing waits on the
-//     other kernel.
+//   * the merge kernel, after both, combines the sink-set partial with the
+//     middle partials into O_exact (one CTA per query head, the chunks split
+//     over four thread groups), and the CTA finishing a sequence's last head
+//     computes rel_l2 and the commit flag.
 //
 // Inside a CTA one producer lane fills a ring of shared-memory stages with
 // K and V tiles through the TMA engine (mbarrier completion); consumer warps
@@ -57,20 +55,21 @@ namespace alspec {
 
 constexpr int kSmemLimit = 227 * 1024;
 
-// Stages per token slot of the tensor-core middle kernel: 2 slots of 16 KB
-// per consumer warp keep ~128 KB in flight per SM, enough for the HBM
-// bandwidth-latency product without queueing loads longer than necessary.
+// Stages per token slot of the tensor-core middle kernel: 3 stages of 16 KB
+// per consumer warp keep up to 192 KB in flight per SM -- well above the HBM
+// bandwidth-latency product -- so the producer keeps streaming through the
+// few microseconds an item's end (merging the warps' states) takes.
 #ifndef ALSPEC_MID_SPW
-#define ALSPEC_MID_SPW 2
+#define ALSPEC_MID_SPW 3
 #endif
 
 constexpr unsigned kErrSeqLen = 1u;   // ALSPEC_DEVERR_SEQ_LEN
 constexpr unsigned kErrTimeout = 2u;  // ALSPEC_DEVERR_TIMEOUT
 
 // Counter words at the head of the workspace.  Then, per (sequence, KV
-// head), the sink-set item tickets [B * Hkv] and the completion tickets
-// [B * Hkv]; then the per-sequence head tickets [B].  Whoever takes the last
-// ticket of a group resets it, so the words are zero between calls.
+// head), the sink-set item tickets [B * Hkv]; then the per-sequence head
+// tickets of the merge kernel [B].  Whoever takes the last ticket of a group
+// resets it, so the words are zero between calls.
 constexpr int kCtrQueue = 0;
 constexpr int kCtrDone = 1;
 constexpr int kCtrError = 2;
@@ -80,14 +79,11 @@ __host__ __device__ __forceinline__ int ctr_spec(int B, int Hkv, int b, int kvh)
     (void)B;
     return kCtrFixed + b * Hkv + kvh;
 }
-__host__ __device__ __forceinline__ int ctr_fin(int B, int Hkv, int b, int kvh) {
-    return kCtrFixed + B * Hkv + b * Hkv + kvh;
-}
 __host__ __device__ __forceinline__ int ctr_seq(int B, int Hkv, int b) {
-    return kCtrFixed + 2 * B * Hkv + b;
+    return kCtrFixed + B * Hkv + b;
 }
 __host__ __device__ __forceinline__ int ctr_words(int B, int Hkv) {
-    return kCtrFixed + 2 * B * Hkv + B;
+    return kCtrFixed + B * Hkv + B;
 }
 
 constexpr int kLastTileFlag = 1;
@@ -713,109 +709,6 @@ struct EngineOf<C, T, D, G, true> {
     using type = MmaEngine<C, D, G>;
 };
 
-// ------------------------------------------------------- merge + verify
-
-// Final merge for the G query heads of (sequence b, KV head kvh), run by the
-// consumer warps of the CTA that completed the group's last piece; warp w
-// takes heads w, w + nwarps, ...  O_exact merges the sink-set partial with
-// the nmid middle partials; O_spec is rebuilt from the same sink-set partial
-// with the same division, so the two are bit-identical when the middle is
-// empty.  Each head's squared distance and squared norm are reduced in a
-// fixed order; the warp that completes the last head of the sequence sums
-// them over heads (fixed order, fp64) and writes rel_l2 and the flag.
-template <int D, int G, int TT>
-__device__ __noinline__ void finish_group(const Params& p, int b, int kvh, int warp, int nwarps,
-                                          int lane) {
-    constexpr int E = D / 32;  // output elements per lane
-    const unsigned full = 0xffffffffu;
-    const int mid_tiles = cdiv(seq_geom(p, b, false).mid_len, TT);
-    int mine = 0;
-    for (int hh = warp; hh < G; hh += nwarps, ++mine) {
-        const size_t bh = (size_t)b * p.Hq + kvh * G + hh;
-        const float2 sml = __ldcg(reinterpret_cast<const float2*>(p.spec_ml) + bh);
-        const float2* mml = reinterpret_cast<const float2*>(p.mid_ml) + bh * p.n2;
-        float M = sml.x;
-        for (int c = lane; c < p.n2; c += 32) {
-            int tlo, thi;
-            mid_chunk(p, mid_tiles, c, tlo, thi);
-            if (thi > tlo) M = fmaxf(M, __ldcg(&mml[c].x));
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(full, M, o));
-        const float f0 = merge_weight(sml.x, M);
-        float os[E], acc[E];
-        float lsum = f0 * sml.y;
-#pragma unroll
-        for (int i = 0; i < E; ++i) {
-            os[i] = __ldcg(p.spec_o + bh * D + lane + 32 * i);
-            acc[i] = f0 * os[i];
-        }
-        const float* mo = p.mid_o + bh * p.n2 * D + lane;
-#pragma unroll 4
-        for (int c = 0; c < p.n2; ++c) {
-            int tlo, thi;
-            mid_chunk(p, mid_tiles, c, tlo, thi);
-            if (thi <= tlo) continue;  // empty chunk: never written
-            const float2 ml = __ldcg(&mml[c]);
-            const float f = merge_weight(ml.x, M);
-            lsum = fmaf(f, ml.y, lsum);
-#pragma unroll
-            for (int i = 0; i < E; ++i) acc[i] = fmaf(f, __ldcg(mo + (size_t)c * D + 32 * i), acc[i]);
-        }
-        float dd = 0.f, nn = 0.f;
-#pragma unroll
-        for (int i = 0; i < E; ++i) {
-            const float o_spec = __fdiv_rn(os[i], sml.y);
-            const float o_exact = __fdiv_rn(acc[i], lsum);
-            p.out_exact[bh * D + lane + 32 * i] = o_exact;
-            const float diff = o_exact - o_spec;
-            dd = fmaf(diff, diff, dd);
-            nn = fmaf(o_exact, o_exact, nn);
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            dd += __shfl_xor_sync(full, dd, o);
-            nn += __shfl_xor_sync(full, nn, o);
-        }
-        if (lane == 0) *reinterpret_cast<float2*>(p.dn + bh * 2) = make_float2(dd, nn);
-    }
-    if (mine == 0) return;
-    // Count this warp's heads towards the sequence.
-    int last = 0;
-    if (lane == 0) {
-        __threadfence();
-        unsigned* word = p.ctr + ctr_seq(p.B, p.Hkv, b);
-        const unsigned t = atomicAdd(word, (unsigned)mine);
-        last = t + (unsigned)mine == (unsigned)p.Hq;
-        if (last) {
-            atomicExch(word, 0u);
-            __threadfence();
-        }
-    }
-    if (!__shfl_sync(full, last, 0)) return;
-    double D2 = 0.0, N2 = 0.0;
-    for (int h = lane; h < p.Hq; h += 32) {
-        const float2 v = __ldcg(reinterpret_cast<const float2*>(p.dn) + (size_t)b * p.Hq + h);
-        D2 += (double)v.x;
-        N2 += (double)v.y;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        D2 += __shfl_xor_sync(full, D2, o);
-        N2 += __shfl_xor_sync(full, N2, o);
-    }
-    if (lane == 0) {
-        double r;
-        if (N2 == 0.0) {
-            r = D2 == 0.0 ? 0.0 : (double)INFINITY;
-        } else {
-            r = sqrt(D2 / N2);
-        }
-        p.rel_l2[b] = (float)r;
-        p.commit[b] = r <= (double)p.lambda ? 1 : 0;
-    }
-}
-
 // ------------------------------------------------------------ the kernel
 
 template <typename T, int D, int G, bool SPEC, bool MMA>
@@ -1046,15 +939,13 @@ __global__ void __launch_bounds__(Cfg<T, D, G, SPEC, MMA>::kThreads, 1)
                 part_o[row * D + e] = O;
             }
         }
-        __threadfence();
+        if (SPEC) __threadfence();  // partials are read by another CTA's merge
         // Every consumer thread's partial is written (and the deposit slots
         // are free again) once this sync passes.
         if (!sync_on(free_bar, ph_free)) break;
         st.reset();
-        const SeqGeom g = seq_geom(p, b, false);
-        const unsigned nmid = (unsigned)mid_pieces(p, cdiv(g.mid_len, TT));
-
         if (SPEC && p.n1 > 1) {
+            const SeqGeom g = seq_geom(p, b, false);
             // ---- the CTA finishing last for (b, kv head) merges every
             // sink-set item of that head into O_spec.
             const int nch = cdiv(spec_tiles(g, TT), p.c1 / TT);
@@ -1090,15 +981,146 @@ __global__ void __launch_bounds__(Cfg<T, D, G, SPEC, MMA>::kThreads, 1)
                 p.spec_o[bh * D + e] = O;
                 p.out_spec[bh * D + e] = __fdiv_rn(O, L);
             }
-            __threadfence();
             if (!sync_on(free_bar, ph_free)) break;
         }
-        // ---- one more piece of (b, kv head) is complete: the sink-set merge
-        // (from the sink-set kernel) or a middle item.  The last of the
-        // 1 + nmid pieces finishes the head group.
-        const int fin = ticket(p.ctr + ctr_fin(p.B, p.Hkv, b, kvh), 1u + nmid);
-        if (fin < 0) break;
-        if (fin) finish_group<D, G, TT>(p, b, kvh, warp, C::NCW, lane);
+    }
+}
+
+// ------------------------------------------------------- merge + verify
+
+constexpr int kMergeParts = 4;  // thread groups sharing a head's chunks
+
+// One CTA per (query head, sequence), D x 4 threads: thread (part, e) owns
+// output element e and the chunks c = part, part + 4, ...  O_exact merges the
+// sink-set partial with the sequence's non-empty middle partials; O_spec is
+// rebuilt from the same sink-set partial with the same division, so the two
+// are bit-identical when the middle is empty.  Each head's squared distance
+// and squared norm are reduced in a fixed order; the CTA finishing the last
+// head of a sequence sums them over heads (fixed order, fp64) and writes
+// rel_l2 and the commit flag.
+template <int D, int TT>
+__global__ void __launch_bounds__(D * kMergeParts) merge_kernel(const __grid_constant__ Params p) {
+    constexpr int NT = D * kMergeParts;
+    const int h = blockIdx.x;
+    const int b = blockIdx.y;
+    const int tid = threadIdx.x;
+    const int e = tid % D;
+    const int part = tid / D;
+    const size_t bh = (size_t)b * p.Hq + h;
+    const int mid_tiles = cdiv(seq_geom(p, b, false).mid_len, TT);
+    __shared__ int list[kMaxChunks];         // non-empty chunks, in order
+    __shared__ float wgt[kMaxChunks];        // their merge weights
+    __shared__ float red[NT / 32];
+    __shared__ float accs[kMergeParts][D];
+    __shared__ float lpart[kMergeParts];
+    __shared__ int nlist;
+    __shared__ int last;
+
+    // Non-empty chunks (warp 0, in chunk order) and the merged max.
+    const float2* mml = reinterpret_cast<const float2*>(p.mid_ml) + bh * p.n2;
+    const float2 sml = *reinterpret_cast<const float2*>(p.spec_ml + bh * 2);
+    if (tid < 32) {
+        int count = 0;
+        for (int c0 = 0; c0 < p.n2; c0 += 32) {
+            const int c = c0 + tid;
+            int tlo = 0, thi = 0;
+            if (c < p.n2) mid_chunk(p, mid_tiles, c, tlo, thi);
+            const bool ne = c < p.n2 && thi > tlo;
+            const unsigned m = __ballot_sync(0xffffffffu, ne);
+            if (ne) list[count + __popc(m & ((1u << tid) - 1u))] = c;
+            count += __popc(m);
+        }
+        if (tid == 0) nlist = count;
+    }
+    __syncthreads();
+    const int n = nlist;
+    float M = sml.x;
+    for (int i = tid; i < n; i += NT) M = fmaxf(M, __ldg(&mml[list[i]].x));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    if ((tid & 31) == 0) red[tid >> 5] = M;
+    __syncthreads();
+#pragma unroll
+    for (int w = 0; w < NT / 32; ++w) M = fmaxf(M, red[w]);
+    for (int i = tid; i < n; i += NT) wgt[i] = merge_weight(__ldg(&mml[list[i]].x), M);
+    __syncthreads();
+
+    // Weighted sums over this thread group's share of the chunks.
+    const float* mo = p.mid_o + bh * p.n2 * D + e;
+    float acc = 0.f, ls = 0.f;
+#pragma unroll 8
+    for (int i = part; i < n; i += kMergeParts) {
+        const int c = list[i];
+        acc = fmaf(wgt[i], __ldg(mo + (size_t)c * D), acc);
+        if (e == 0) ls = fmaf(wgt[i], __ldg(&mml[c].y), ls);
+    }
+    accs[part][e] = acc;
+    if (e == 0) lpart[part] = ls;
+    __syncthreads();
+    if (part == 0) {
+        const float os = p.spec_o[bh * D + e];
+        const float f0 = merge_weight(sml.x, M);
+        float a = f0 * os;
+        float l = f0 * sml.y;
+#pragma unroll
+        for (int q = 0; q < kMergeParts; ++q) {
+            a += accs[q][e];
+            l += lpart[q];
+        }
+        const float o_spec = __fdiv_rn(os, sml.y);
+        const float o_exact = __fdiv_rn(a, l);
+        p.out_exact[bh * D + e] = o_exact;
+        const float diff = o_exact - o_spec;
+        accs[0][e] = diff * diff;  // each thread only rewrites its own slot
+        accs[1][e] = o_exact * o_exact;
+    }
+    __syncthreads();
+    if (tid < 32) {
+        float dd = 0.f, nn = 0.f;
+        for (int i = tid; i < D; i += 32) {
+            dd += accs[0][i];
+            nn += accs[1][i];
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            dd += __shfl_xor_sync(0xffffffffu, dd, o);
+            nn += __shfl_xor_sync(0xffffffffu, nn, o);
+        }
+        if (tid == 0) {
+            *reinterpret_cast<float2*>(p.dn + bh * 2) = make_float2(dd, nn);
+            __threadfence();
+            unsigned* word = p.ctr + ctr_seq(p.B, p.Hkv, b);
+            const unsigned t = atomicAdd(word, 1u);
+            last = t == (unsigned)(p.Hq - 1);
+            if (last) {
+                atomicExch(word, 0u);
+                __threadfence();
+            }
+        }
+        if (__shfl_sync(0xffffffffu, tid == 0 ? last : 0, 0)) {
+            double D2 = 0.0, N2 = 0.0;
+            for (int hh = tid; hh < p.Hq; hh += 32) {
+                const float2 v =
+                    __ldcg(reinterpret_cast<const float2*>(p.dn) + (size_t)b * p.Hq + hh);
+                D2 += (double)v.x;
+                N2 += (double)v.y;
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                D2 += __shfl_xor_sync(0xffffffffu, D2, o);
+                N2 += __shfl_xor_sync(0xffffffffu, N2, o);
+            }
+            if (tid == 0) {
+                double r;
+                if (N2 == 0.0) {
+                    r = D2 == 0.0 ? 0.0 : (double)INFINITY;
+                } else {
+                    r = sqrt(D2 / N2);
+                }
+                p.rel_l2[b] = (float)r;
+                p.commit[b] = r <= (double)p.lambda ? 1 : 0;
+            }
+        }
     }
 }
 
