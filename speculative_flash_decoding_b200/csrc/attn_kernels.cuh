@@ -158,22 +158,13 @@ __host__ __device__ __forceinline__ int spec_tiles(const SeqGeom& g, int TT) {
     return cdiv(g.ns, TT) + cdiv(g.L - g.ws, TT);
 }
 
+__device__ __forceinline__ int per_spec_items(const Params& p) { return p.n1; }
+
 // Middle tiles [t_lo, t_hi) of chunk c, for a middle of mid_tiles tiles.
 __device__ __forceinline__ void mid_chunk(const Params& p, int mid_tiles, int c, int& t_lo,
                                           int& t_hi) {
     t_lo = (int)(((unsigned long long)mid_tiles * p.fq[c]) >> kFracBits);
     t_hi = (int)(((unsigned long long)mid_tiles * p.fq[c + 1]) >> kFracBits);
-}
-
-// Number of non-empty middle chunks of a middle of mid_tiles tiles.
-__device__ __forceinline__ int mid_pieces(const Params& p, int mid_tiles) {
-    int n = 0, prev = 0;
-    for (int c = 1; c <= p.n2; ++c) {
-        const int t = (int)(((unsigned long long)mid_tiles * p.fq[c]) >> kFracBits);
-        n += t > prev;
-        prev = t;
-    }
-    return n;
 }
 
 // One work item: a range of tiles of one (sequence, KV head).
@@ -939,7 +930,7 @@ __global__ void __launch_bounds__(Cfg<T, D, G, SPEC, MMA>::kThreads, 1)
                 part_o[row * D + e] = O;
             }
         }
-        if (SPEC) __threadfence();  // partials are read by another CTA's merge
+        if (SPEC && per_spec_items(p) > 1) __threadfence();  // read by another CTA's merge
         // Every consumer thread's partial is written (and the deposit slots
         // are free again) once this sync passes.
         if (!sync_on(free_bar, ph_free)) break;
@@ -1016,39 +1007,41 @@ __global__ void __launch_bounds__(D * kMergeParts) merge_kernel(const __grid_con
     __shared__ int nlist;
     __shared__ int last;
 
-    // Non-empty chunks (warp 0, in chunk order) and the merged max.
+    // Non-empty chunks, in chunk order.  Thread 0 walks the chunk table with
+    // uniform indices (the table lives in parameter space, where lanes
+    // reading different entries would serialize).
     const float2* mml = reinterpret_cast<const float2*>(p.mid_ml) + bh * p.n2;
     const float2 sml = *reinterpret_cast<const float2*>(p.spec_ml + bh * 2);
-    if (tid < 32) {
-        int count = 0;
-        for (int c0 = 0; c0 < p.n2; c0 += 32) {
-            const int c = c0 + tid;
-            int tlo = 0, thi = 0;
-            if (c < p.n2) mid_chunk(p, mid_tiles, c, tlo, thi);
-            const bool ne = c < p.n2 && thi > tlo;
-            const unsigned m = __ballot_sync(0xffffffffu, ne);
-            if (ne) list[count + __popc(m & ((1u << tid) - 1u))] = c;
-            count += __popc(m);
+    if (tid == 0) {
+        int count = 0, prev = 0;
+#pragma unroll 8
+        for (int c = 0; c < p.n2; ++c) {
+            const int t = (int)(((unsigned long long)mid_tiles * p.fq[c + 1]) >> kFracBits);
+            if (t > prev) list[count++] = c;
+            prev = t;
         }
-        if (tid == 0) nlist = count;
+        nlist = count;
     }
     __syncthreads();
     const int n = nlist;
     float M = sml.x;
-    for (int i = tid; i < n; i += NT) M = fmaxf(M, __ldg(&mml[list[i]].x));
+    for (int i = tid; i < n; i += NT) {
+        wgt[i] = __ldg(&mml[list[i]].x);  // the chunk's max, turned into a weight below
+        M = fmaxf(M, wgt[i]);
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     if ((tid & 31) == 0) red[tid >> 5] = M;
     __syncthreads();
 #pragma unroll
     for (int w = 0; w < NT / 32; ++w) M = fmaxf(M, red[w]);
-    for (int i = tid; i < n; i += NT) wgt[i] = merge_weight(__ldg(&mml[list[i]].x), M);
+    for (int i = tid; i < n; i += NT) wgt[i] = merge_weight(wgt[i], M);
     __syncthreads();
 
     // Weighted sums over this thread group's share of the chunks.
     const float* mo = p.mid_o + bh * p.n2 * D + e;
     float acc = 0.f, ls = 0.f;
-#pragma unroll 8
+#pragma unroll 16
     for (int i = part; i < n; i += kMergeParts) {
         const int c = list[i];
         acc = fmaf(wgt[i], __ldg(mo + (size_t)c * D), acc);
