@@ -980,38 +980,43 @@ __global__ void __launch_bounds__(Cfg<T, D, G, SPEC, MMA>::kThreads, 1)
 // ------------------------------------------------------- merge + verify
 
 constexpr int kMergeParts = 4;  // thread groups sharing a head's chunks
+constexpr int kMergeBatch = 8;  // chunk loads each thread keeps in flight
 
 // One CTA per (query head, sequence), D x 4 threads: thread (part, e) owns
-// output element e and the chunks c = part, part + 4, ...  O_exact merges the
-// sink-set partial with the sequence's non-empty middle partials; O_spec is
-// rebuilt from the same sink-set partial with the same division, so the two
-// are bit-identical when the middle is empty.  Each head's squared distance
-// and squared norm are reduced in a fixed order; the CTA finishing the last
-// head of a sequence sums them over heads (fixed order, fp64) and writes
-// rel_l2 and the commit flag.
+// output element e and the chunks list[part], list[part + 4], ...  O_exact
+// merges the sink-set partial with the sequence's non-empty middle partials;
+// O_spec is rebuilt from the same sink-set partial with the same division,
+// so the two are bit-identical when the middle is empty.  Each head's
+// squared distance and squared norm are reduced in a fixed order; the CTA
+// finishing the last head of a sequence sums them over heads (fixed order,
+// fp64) and writes rel_l2 and the commit flag.
 template <int D, int TT>
 __global__ void __launch_bounds__(D * kMergeParts) merge_kernel(const __grid_constant__ Params p) {
     constexpr int NT = D * kMergeParts;
+    constexpr int NW = NT / 32;
     const int h = blockIdx.x;
     const int b = blockIdx.y;
     const int tid = threadIdx.x;
     const int e = tid % D;
     const int part = tid / D;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
     const size_t bh = (size_t)b * p.Hq + h;
-    const int mid_tiles = cdiv(seq_geom(p, b, false).mid_len, TT);
-    __shared__ int list[kMaxChunks];         // non-empty chunks, in order
-    __shared__ float wgt[kMaxChunks];        // their merge weights
-    __shared__ float red[NT / 32];
+    __shared__ int list[kMaxChunks];      // non-empty chunks, in order
+    __shared__ float2 cml[kMaxChunks];    // their (m, l), then (weight, weighted l)
+    __shared__ float red[2][NW];
     __shared__ float accs[kMergeParts][D];
-    __shared__ float lpart[kMergeParts];
     __shared__ int nlist;
     __shared__ int last;
 
-    // Non-empty chunks, in chunk order.  Thread 0 walks the chunk table with
-    // uniform indices (the table lives in parameter space, where lanes
-    // reading different entries would serialize).
+    // Loads that do not depend on the chunk list go out first.
+    const float2 sml = __ldg(reinterpret_cast<const float2*>(p.spec_ml) + bh);
+    const float os = __ldg(p.spec_o + bh * D + e);
+    const int mid_tiles = cdiv(seq_geom(p, b, false).mid_len, TT);
     const float2* mml = reinterpret_cast<const float2*>(p.mid_ml) + bh * p.n2;
-    const float2 sml = *reinterpret_cast<const float2*>(p.spec_ml + bh * 2);
+
+    // Non-empty chunks, in chunk order (thread 0 walks the table with
+    // uniform indices; the table lives in parameter space).
     if (tid == 0) {
         int count = 0, prev = 0;
 #pragma unroll 8
@@ -1026,51 +1031,64 @@ __global__ void __launch_bounds__(D * kMergeParts) merge_kernel(const __grid_con
     const int n = nlist;
     float M = sml.x;
     for (int i = tid; i < n; i += NT) {
-        wgt[i] = __ldg(&mml[list[i]].x);  // the chunk's max, turned into a weight below
-        M = fmaxf(M, wgt[i]);
+        cml[i] = __ldg(&mml[list[i]]);
+        M = fmaxf(M, cml[i].x);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    if ((tid & 31) == 0) red[tid >> 5] = M;
+    if (lane == 0) red[0][warp] = M;
     __syncthreads();
 #pragma unroll
-    for (int w = 0; w < NT / 32; ++w) M = fmaxf(M, red[w]);
-    for (int i = tid; i < n; i += NT) wgt[i] = merge_weight(wgt[i], M);
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, red[0][w]);
+    // Weights, and the normaliser: sum of weight * l in a fixed order.
+    float lsum = 0.f;
+    for (int i = tid; i < n; i += NT) {
+        const float w = merge_weight(cml[i].x, M);
+        cml[i].x = w;
+        lsum = fmaf(w, cml[i].y, lsum);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
+    if (lane == 0) red[1][warp] = lsum;
     __syncthreads();
 
-    // Weighted sums over this thread group's share of the chunks.
+    // Weighted value rows: batches of independent loads.
     const float* mo = p.mid_o + bh * p.n2 * D + e;
-    float acc = 0.f, ls = 0.f;
-#pragma unroll 16
-    for (int i = part; i < n; i += kMergeParts) {
-        const int c = list[i];
-        acc = fmaf(wgt[i], __ldg(mo + (size_t)c * D), acc);
-        if (e == 0) ls = fmaf(wgt[i], __ldg(&mml[c].y), ls);
+    float acc = 0.f;
+    for (int i0 = part; i0 < n; i0 += kMergeParts * kMergeBatch) {
+        float v[kMergeBatch];
+#pragma unroll
+        for (int u = 0; u < kMergeBatch; ++u) {
+            const int i = i0 + u * kMergeParts;
+            v[u] = i < n ? __ldg(mo + (size_t)list[i] * D) : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < kMergeBatch; ++u) {
+            const int i = i0 + u * kMergeParts;
+            if (i < n) acc = fmaf(cml[i].x, v[u], acc);
+        }
     }
     accs[part][e] = acc;
-    if (e == 0) lpart[part] = ls;
     __syncthreads();
     if (part == 0) {
-        const float os = p.spec_o[bh * D + e];
         const float f0 = merge_weight(sml.x, M);
         float a = f0 * os;
         float l = f0 * sml.y;
 #pragma unroll
-        for (int q = 0; q < kMergeParts; ++q) {
-            a += accs[q][e];
-            l += lpart[q];
-        }
+        for (int q = 0; q < kMergeParts; ++q) a += accs[q][e];
+#pragma unroll
+        for (int w = 0; w < NW; ++w) l += red[1][w];
         const float o_spec = __fdiv_rn(os, sml.y);
         const float o_exact = __fdiv_rn(a, l);
         p.out_exact[bh * D + e] = o_exact;
         const float diff = o_exact - o_spec;
-        accs[0][e] = diff * diff;  // each thread only rewrites its own slot
+        accs[0][e] = diff * diff;  // each thread only rewrites its own column
         accs[1][e] = o_exact * o_exact;
     }
     __syncthreads();
-    if (tid < 32) {
+    if (warp == 0) {
         float dd = 0.f, nn = 0.f;
-        for (int i = tid; i < D; i += 32) {
+        for (int i = lane; i < D; i += 32) {
             dd += accs[0][i];
             nn += accs[1][i];
         }
@@ -1079,7 +1097,7 @@ __global__ void __launch_bounds__(D * kMergeParts) merge_kernel(const __grid_con
             dd += __shfl_xor_sync(0xffffffffu, dd, o);
             nn += __shfl_xor_sync(0xffffffffu, nn, o);
         }
-        if (tid == 0) {
+        if (lane == 0) {
             *reinterpret_cast<float2*>(p.dn + bh * 2) = make_float2(dd, nn);
             __threadfence();
             unsigned* word = p.ctr + ctr_seq(p.B, p.Hkv, b);
@@ -1090,9 +1108,9 @@ __global__ void __launch_bounds__(D * kMergeParts) merge_kernel(const __grid_con
                 __threadfence();
             }
         }
-        if (__shfl_sync(0xffffffffu, tid == 0 ? last : 0, 0)) {
+        if (__shfl_sync(0xffffffffu, lane == 0 ? last : 0, 0)) {
             double D2 = 0.0, N2 = 0.0;
-            for (int hh = tid; hh < p.Hq; hh += 32) {
+            for (int hh = lane; hh < p.Hq; hh += 32) {
                 const float2 v =
                     __ldcg(reinterpret_cast<const float2*>(p.dn) + (size_t)b * p.Hq + hh);
                 D2 += (double)v.x;
@@ -1103,7 +1121,7 @@ __global__ void __launch_bounds__(D * kMergeParts) merge_kernel(const __grid_con
                 D2 += __shfl_xor_sync(0xffffffffu, D2, o);
                 N2 += __shfl_xor_sync(0xffffffffu, N2, o);
             }
-            if (tid == 0) {
+            if (lane == 0) {
                 double r;
                 if (N2 == 0.0) {
                     r = D2 == 0.0 ? 0.0 : (double)INFINITY;
