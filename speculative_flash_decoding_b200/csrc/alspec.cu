@@ -325,20 +325,31 @@ alspec_status ensure_smem_attr(DeviceState* ds, KernelFn fn, int bytes) {
     return ALSPEC_OK;
 }
 
+enum LaunchFlags { kLaunchHighPriority = 1, kLaunchProgrammatic = 2 };
+
 alspec_status launch(KernelFn fn, dim3 grid, dim3 block, int smem, cudaStream_t stream,
-                     const Params& p, bool high_priority, int prio) {
+                     const Params& p, int flags, int prio) {
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = grid;
     cfg.blockDim = block;
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    if (high_priority) {
-        attr[0].id = cudaLaunchAttributePriority;
-        attr[0].val.priority = prio;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
+    cudaLaunchAttribute attr[2];
+    int n = 0;
+    if (flags & kLaunchHighPriority) {
+        attr[n].id = cudaLaunchAttributePriority;
+        attr[n].val.priority = prio;
+        ++n;
     }
+    if (flags & kLaunchProgrammatic) {
+        // May start before the preceding kernel in the stream completes; the
+        // kernel waits for it (griddepcontrol.wait) before using its output.
+        attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[n].val.programmaticStreamSerializationAllowed = 1;
+        ++n;
+    }
+    cfg.attrs = n ? attr : nullptr;
+    cfg.numAttrs = n;
     return ok(cudaLaunchKernelEx(&cfg, fn, p)) ? ALSPEC_OK : ALSPEC_ERR_CUDA;
 }
 
@@ -464,8 +475,8 @@ alspec_status alspec_decode(const alspec_desc* desc, const void* q, const void* 
     if (!ok(cudaEventRecord(ds->fork, s)) || !ok(cudaStreamWaitEvent(ds->hi, ds->fork, 0)))
         return ALSPEC_ERR_CUDA;
     const dim3 grid1(pl.grid1);
-    if ((st = launch(ks.spec, grid1, dim3(ks.threads_spec), ks.smem_spec, ds->hi, p, true,
-                     ds->prio_hi)) != ALSPEC_OK)
+    if ((st = launch(ks.spec, grid1, dim3(ks.threads_spec), ks.smem_spec, ds->hi, p,
+                     kLaunchHighPriority, ds->prio_hi)) != ALSPEC_OK)
         return st;
     if (spec_event && !ok(record_event(static_cast<cudaEvent_t>(spec_event), ds->hi)))
         return ALSPEC_ERR_CUDA;
@@ -477,8 +488,8 @@ alspec_status alspec_decode(const alspec_desc* desc, const void* q, const void* 
     // The middle of every sequence on the caller's stream.
     if (!prof(2, s)) return ALSPEC_ERR_CUDA;
     if (pl.n2 > 0) {
-        if ((st = launch(ks.mid, dim3(pl.grid2), dim3(ks.threads_mid), ks.smem_mid, s, p, false,
-                         0)) != ALSPEC_OK)
+        if ((st = launch(ks.mid, dim3(pl.grid2), dim3(ks.threads_mid), ks.smem_mid, s, p, 0, 0)) !=
+            ALSPEC_OK)
             return st;
     }
     if (!prof(3, s)) return ALSPEC_ERR_CUDA;
@@ -489,8 +500,11 @@ alspec_status alspec_decode(const alspec_desc* desc, const void* q, const void* 
         mk = pl.tt == 32 ? merge_kernel<128, 32> : merge_kernel<128, 16>;
     else
         mk = pl.tt == 32 ? merge_kernel<64, 32> : merge_kernel<64, 16>;
+    // Programmatic launch right behind the middle kernel (when there is one
+    // and no profiling event sits between them).
+    const bool pdl = pl.n2 > 0 && !prof_events;
     if ((st = launch(mk, dim3(desc->n_q_heads, desc->batch), dim3(desc->head_dim * kMergeParts),
-                     0, s, p, false, 0)) != ALSPEC_OK)
+                     0, s, p, pdl ? kLaunchProgrammatic : 0, 0)) != ALSPEC_OK)
         return st;
     if (!prof(4, s)) return ALSPEC_ERR_CUDA;
     return ALSPEC_OK;

@@ -737,6 +737,9 @@ __global__ void __launch_bounds__(Cfg<T, D, G, SPEC, MMA>::kThreads, 1)
         sh->last = 0;
         fence_barrier_init();
     }
+    // The merge kernel that follows this (middle) kernel may be resident
+    // already: it only prepares until this grid has completed.
+    if (!SPEC) pdl_launch_dependents();
     __syncthreads();
 
     if (warp == C::NCW) {
@@ -1009,9 +1012,6 @@ __global__ void __launch_bounds__(D * kMergeParts) merge_kernel(const __grid_con
     __shared__ int nlist;
     __shared__ int last;
 
-    // Loads that do not depend on the chunk list go out first.
-    const float2 sml = __ldg(reinterpret_cast<const float2*>(p.spec_ml) + bh);
-    const float os = __ldg(p.spec_o + bh * D + e);
     const int mid_tiles = cdiv(seq_geom(p, b, false).mid_len, TT);
     const float2* mml = reinterpret_cast<const float2*>(p.mid_ml) + bh * p.n2;
 
@@ -1027,11 +1027,16 @@ __global__ void __launch_bounds__(D * kMergeParts) merge_kernel(const __grid_con
         }
         nlist = count;
     }
+    // Everything above only read inputs; the partials are written by the
+    // kernels this one follows, which may still be running.
+    pdl_wait_prerequisite();
+    const float2 sml = __ldcg(reinterpret_cast<const float2*>(p.spec_ml) + bh);
+    const float os = __ldcg(p.spec_o + bh * D + e);
     __syncthreads();
     const int n = nlist;
     float M = sml.x;
     for (int i = tid; i < n; i += NT) {
-        cml[i] = __ldg(&mml[list[i]]);
+        cml[i] = __ldcg(&mml[list[i]]);
         M = fmaxf(M, cml[i].x);
     }
 #pragma unroll
@@ -1060,7 +1065,7 @@ __global__ void __launch_bounds__(D * kMergeParts) merge_kernel(const __grid_con
 #pragma unroll
         for (int u = 0; u < kMergeBatch; ++u) {
             const int i = i0 + u * kMergeParts;
-            v[u] = i < n ? __ldg(mo + (size_t)list[i] * D) : 0.f;
+            v[u] = i < n ? __ldcg(mo + (size_t)list[i] * D) : 0.f;
         }
 #pragma unroll
         for (int u = 0; u < kMergeBatch; ++u) {
