@@ -221,6 +221,38 @@ int alspec_version(void);
  */
 int alspec_last_cuda_error(void);
 
+/*
+ * Allocation-free variant of alspec_decode (the paper has no counterpart;
+ * this is a deployment convenience).  Some callers cannot allocate device
+ * memory at all -- for example code running inside a host framework that
+ * owns every allocation, or a callback that must not call cudaMalloc -- and
+ * so cannot provide the workspace alspec_decode needs.  This entry point
+ * takes the same inputs and outputs but no workspace: its scratch space is
+ * a fixed array of ALSPEC_NOALLOC_SCRATCH_BYTES (8 MiB) in the library's
+ * own device memory, which every GPU that loads the library holds until the
+ * process exits.  It never calls cudaMalloc or cudaFree.
+ *
+ *   - A problem whose workspace (alspec_workspace_size) is larger than
+ *     ALSPEC_NOALLOC_SCRATCH_BYTES is rejected with ALSPEC_ERR_WORKSPACE
+ *     before anything is launched.
+ *   - The first call on a device looks up the device address of the array
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     outside any stream capture.
+ *   - Each call clears the array's counters on `stream`, then runs exactly
+ *     what alspec_decode runs.  All calls on a device share the one array:
+ *     calls that overlap on the GPU (different streams without ordering
+ *     between them) race and corrupt each other's results.  Calls ordered
+ *     on one stream are fine.
+ *   - There is no spec_event and no profiling events; the device error word
+ *     is not readable (use alspec_decode with a workspace for that).
+ */
+#define ALSPEC_NOALLOC_SCRATCH_BYTES (8u << 20)
+alspec_status alspec_decode_noalloc(const alspec_desc* desc,
+                                    const void* q, const void* k_cache, const void* v_cache,
+                                    const int32_t* seq_lens, int n_sink, int window,
+                                    float lambda, float* out_spec, float* out_exact,
+                                    float* rel_l2, uint8_t* commit, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

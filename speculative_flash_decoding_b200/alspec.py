@@ -68,7 +68,11 @@ SIGNATURES = {
     "alspec_status_string": (ctypes.c_char_p, [_i]),
     "alspec_version": (_i, []),
     "alspec_last_cuda_error": (_i, []),
+    "alspec_decode_noalloc": (_i, [_descp, _vp, _vp, _vp, _vp, _i, _i, _f, _vp, _vp, _vp, _vp,
+                                   _vp]),
 }
+
+ALSPEC_NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
 def _load():
@@ -117,6 +121,17 @@ def alspec_decode(desc: alspec_desc, q: int, k_cache: int, v_cache: int, seq_len
     return int(_lib.alspec_decode(ctypes.byref(desc), q, k_cache, v_cache, seq_lens, n_sink,
                                   window, lam, out_spec, out_exact, rel_l2, commit, workspace,
                                   workspace_bytes, stream, spec_event or None, prof))
+
+
+def alspec_decode_noalloc(desc: alspec_desc, q: int, k_cache: int, v_cache: int, seq_lens: int,
+                          n_sink: int, window: int, lam: float, out_spec: int, out_exact: int,
+                          rel_l2: int, commit: int, stream: int) -> int:
+    """alspec_decode without a workspace: for callers that cannot allocate
+    device memory.  Uses the library's fixed 8 MiB device scratch array
+    (shared by all calls on a device -- calls must not overlap on the GPU)."""
+    return int(_lib.alspec_decode_noalloc(ctypes.byref(desc), q, k_cache, v_cache, seq_lens,
+                                          n_sink, window, lam, out_spec, out_exact, rel_l2,
+                                          commit, stream))
 
 
 def alspec_query_plan(desc: alspec_desc, n_sink: int, window: int):

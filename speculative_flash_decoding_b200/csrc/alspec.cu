@@ -602,3 +602,56 @@ int alspec_version(void) { return 100; }
 int alspec_last_cuda_error(void) { return (int)t_last_error; }
 
 }  // extern "C"
+
+// ------------------------------------------------------------ no-alloc path
+
+namespace {
+
+// Scratch space of alspec_decode_noalloc: a fixed array in this library's
+// device memory (zero at load), used in place of a caller's workspace.  In
+// host code the name is only a host-side stand-in; kernels get the device
+// address looked up below.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[ALSPEC_NOALLOC_SCRATCH_BYTES];
+
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device, looked up once
+// per device (with that device current).
+alspec_status noalloc_scratch(void** out) {
+    int dev = 0;
+    if (!ok(cudaGetDevice(&dev)) || dev < 0 || dev >= kMaxDevices) return ALSPEC_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (!g_noalloc_ptr[dev]) {
+        void* ptr = nullptr;
+        if (!ok(cudaGetSymbolAddress(&ptr, g_noalloc_scratch)) || !ptr) return ALSPEC_ERR_CUDA;
+        g_noalloc_ptr[dev] = ptr;
+    }
+    *out = g_noalloc_ptr[dev];
+    return ALSPEC_OK;
+}
+
+}  // namespace
+
+extern "C" alspec_status alspec_decode_noalloc(const alspec_desc* desc, const void* q,
+                                               const void* k_cache, const void* v_cache,
+                                               const int32_t* seq_lens, int n_sink, int window,
+                                               float lambda, float* out_spec, float* out_exact,
+                                               float* rel_l2, uint8_t* commit, void* stream) {
+    const size_t need = alspec_workspace_size(desc, n_sink, window);
+    if (need == 0) {
+        const alspec_status st = check_desc(desc, n_sink, window);
+        return st != ALSPEC_OK ? st : ALSPEC_ERR_INVALID_ARG;
+    }
+    if (need > ALSPEC_NOALLOC_SCRATCH_BYTES) return ALSPEC_ERR_WORKSPACE;
+    void* scratch = nullptr;
+    alspec_status st = noalloc_scratch(&scratch);
+    if (st != ALSPEC_OK) return st;
+    // The counters at the head of the scratch must start at zero; the rest
+    // of it is written before it is read within a call.
+    const size_t counters = (size_t)ctr_words(desc->batch, desc->n_kv_heads) * sizeof(unsigned);
+    if (!ok(cudaMemsetAsync(scratch, 0, counters, static_cast<cudaStream_t>(stream))))
+        return ALSPEC_ERR_CUDA;
+    return alspec_decode(desc, q, k_cache, v_cache, seq_lens, n_sink, window, lambda, out_spec,
+                         out_exact, rel_l2, commit, scratch, ALSPEC_NOALLOC_SCRATCH_BYTES, stream,
+                         nullptr, nullptr);
+}
