@@ -22,7 +22,7 @@ namespace alspec {
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr int kMaxSpecItems = 32;  // sink-set items per (sequence, KV head)
+constexpr int kMaxSpecItems = 8;  // sink-set CTAs per (sequence, KV head): a portable cluster
 
 // The sink-set kernel gets about 1/ALSPEC_SPEC_SM_DIV of the SMs.
 #ifndef ALSPEC_SPEC_SM_DIV
@@ -102,13 +102,12 @@ int sm_count_for_plan() {
 struct Plan {
     int engine;   // ALSPEC_ENGINE_CUDA_CORES or ALSPEC_ENGINE_TENSOR_CORES
     int tt;       // tokens per pipeline tile of that engine
-    int c1, n1;   // sink-set item tokens and items per (sequence, KV head)
+    int c1, n1;   // sink-set tokens per CTA and CTAs (one cluster) per (sequence, KV head)
     int c2, n2;   // first middle chunk (tokens, longest sequence) and chunks per head
     unsigned fq[kMaxChunks + 1];
     int grid1, grid2;
     int threads, smem, stages;
-    size_t off_ctr, off_spart_ml, off_spart_o, off_spec_ml, off_spec_o, off_mid_ml, off_mid_o,
-        off_dn, total;
+    size_t off_ctr, off_spec_ml, off_spec_o, off_mid_ml, off_mid_o, off_dn, total;
 };
 
 bool supported_g(int g) { return g == 1 || g == 2 || g == 4 || g == 8; }
@@ -160,18 +159,22 @@ void make_plan(const alspec_desc& d, int S, int W, int sms, Plan* pl) {
     const int heads = d.batch * d.n_kv_heads;
     const int L = d.max_seq_len;
     const int tiles_max = ceil_div(std::min(S, L), TT) + ceil_div(std::min(W, L), TT);
-    const int room1 = std::max(1, sms / 4 / std::max(1, heads));
-    pl->n1 = std::min({kMaxSpecItems, room1, ceil_div(tiles_max, 64)});
-    pl->n1 = std::max(1, pl->n1);
+    // CTAs per head for the sink set (one thread-block cluster): about 8
+    // tiles each, at most 8 (the portable cluster size), and all heads
+    // together within half of the SMs.
+    const int room1 = std::max(1, sms / 2 / std::max(1, heads));
+    pl->n1 = std::max(1, std::min({kMaxSpecItems, room1, ceil_div(tiles_max, 8)}));
     const int tiles_per_item = ceil_div(tiles_max, pl->n1);
     pl->c1 = tiles_per_item * TT;
-    pl->n1 = ceil_div(tiles_max, tiles_per_item);
     pl->grid1 = heads * pl->n1;
 
     const int ns = std::min(S, L);
     const int mid_max = std::max(0, std::max(ns, L - W) - ns);
     const int mid_tiles = ceil_div(mid_max, TT);
-    const int P = std::max(sms - pl->grid1, (3 * sms + 3) / 4);
+    // The persistent middle kernel takes every SM: CTAs that find an SM
+    // busy with the (short) sink-set kernel start when it is done, and the
+    // atomic queue balances the work.
+    const int P = sms;
     std::vector<double> sizes;  // chunk sizes as fractions of a head's middle
     if (mid_tiles > 0) {
         if (d.split_tokens > 0) {
@@ -211,7 +214,7 @@ void make_plan(const alspec_desc& d, int S, int W, int sms, Plan* pl) {
     kernel_shape(d.dtype, d.head_dim, G, pl->engine, &pl->threads, &pl->smem, &pl->stages);
 
     const size_t B = d.batch, Hq = d.n_q_heads, D = d.head_dim;
-    const size_t n1 = pl->n1, n2 = std::max(pl->n2, 1);
+    const size_t n2 = std::max(pl->n2, 1);
     size_t off = 0;
     auto take = [&](size_t bytes) {
         const size_t o = off;
@@ -219,8 +222,6 @@ void make_plan(const alspec_desc& d, int S, int W, int sms, Plan* pl) {
         return o;
     };
     pl->off_ctr = take((size_t)ctr_words(d.batch, d.n_kv_heads) * sizeof(unsigned));
-    pl->off_spart_ml = take(B * Hq * n1 * 2 * sizeof(float));
-    pl->off_spart_o = take(B * Hq * n1 * D * sizeof(float));
     pl->off_spec_ml = take(B * Hq * 2 * sizeof(float));
     pl->off_spec_o = take(B * Hq * D * sizeof(float));
     pl->off_mid_ml = take(B * Hq * n2 * 2 * sizeof(float));
@@ -328,14 +329,21 @@ alspec_status ensure_smem_attr(DeviceState* ds, KernelFn fn, int bytes) {
 enum LaunchFlags { kLaunchHighPriority = 1, kLaunchProgrammatic = 2 };
 
 alspec_status launch(KernelFn fn, dim3 grid, dim3 block, int smem, cudaStream_t stream,
-                     const Params& p, int flags, int prio) {
+                     const Params& p, int flags, int prio, int cluster = 1) {
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = grid;
     cfg.blockDim = block;
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[2];
+    cudaLaunchAttribute attr[3];
     int n = 0;
+    if (cluster > 1) {
+        attr[n].id = cudaLaunchAttributeClusterDimension;
+        attr[n].val.clusterDim.x = cluster;
+        attr[n].val.clusterDim.y = 1;
+        attr[n].val.clusterDim.z = 1;
+        ++n;
+    }
     if (flags & kLaunchHighPriority) {
         attr[n].id = cudaLaunchAttributePriority;
         attr[n].val.priority = prio;
@@ -452,8 +460,6 @@ alspec_status alspec_decode(const alspec_desc* desc, const void* q, const void* 
     p.n2 = pl.n2;
     std::memcpy(p.fq, pl.fq, sizeof p.fq);
     p.ctr = reinterpret_cast<unsigned*>(ws + pl.off_ctr);
-    p.spart_ml = reinterpret_cast<float*>(ws + pl.off_spart_ml);
-    p.spart_o = reinterpret_cast<float*>(ws + pl.off_spart_o);
     p.spec_ml = reinterpret_cast<float*>(ws + pl.off_spec_ml);
     p.spec_o = reinterpret_cast<float*>(ws + pl.off_spec_o);
     p.mid_ml = reinterpret_cast<float*>(ws + pl.off_mid_ml);
@@ -476,7 +482,7 @@ alspec_status alspec_decode(const alspec_desc* desc, const void* q, const void* 
         return ALSPEC_ERR_CUDA;
     const dim3 grid1(pl.grid1);
     if ((st = launch(ks.spec, grid1, dim3(ks.threads_spec), ks.smem_spec, ds->hi, p,
-                     kLaunchHighPriority, ds->prio_hi)) != ALSPEC_OK)
+                     kLaunchHighPriority, ds->prio_hi, pl.n1)) != ALSPEC_OK)
         return st;
     if (spec_event && !ok(record_event(static_cast<cudaEvent_t>(spec_event), ds->hi)))
         return ALSPEC_ERR_CUDA;

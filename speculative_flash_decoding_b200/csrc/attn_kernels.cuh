@@ -12,8 +12,10 @@
 // of value rows -- and partials are merged with the log-sum-exp rule.  The
 // sink-set tokens and the middle tokens are separate item lists, so both
 // outputs come from one read of every cache row:
-//   * the sink-set kernel (SPEC) reads only the S + W tokens, merges its
-//     items in the CTA that finishes last and writes O_spec;
+//   * the sink-set kernel (SPEC) reads only the S + W tokens; the CTAs of one
+//     (sequence, KV head) form a thread-block cluster, each streams a slice
+//     of the sink set, and they merge their partials through distributed
+//     shared memory and write O_spec;
 //   * the middle kernel (MID) is persistent: CTAs pull items from an atomic
 //     queue and stream the cache through shared memory;
 //   * the merge kernel, after both, combines the sink-set partial with the
@@ -66,8 +68,7 @@ constexpr int kSmemLimit = 227 * 1024;
 constexpr unsigned kErrSeqLen = 1u;   // ALSPEC_DEVERR_SEQ_LEN
 constexpr unsigned kErrTimeout = 2u;  // ALSPEC_DEVERR_TIMEOUT
 
-// Counter words at the head of the workspace.  Then, per (sequence, KV
-// head), the sink-set item tickets [B * Hkv]; then the per-sequence head
+// Counter words at the head of the workspace, then the per-sequence head
 // tickets of the merge kernel [B].  Whoever takes the last ticket of a group
 // resets it, so the words are zero between calls.
 constexpr int kCtrQueue = 0;
@@ -75,15 +76,13 @@ constexpr int kCtrDone = 1;
 constexpr int kCtrError = 2;
 constexpr int kCtrFixed = 4;
 
-__host__ __device__ __forceinline__ int ctr_spec(int B, int Hkv, int b, int kvh) {
-    (void)B;
-    return kCtrFixed + b * Hkv + kvh;
-}
 __host__ __device__ __forceinline__ int ctr_seq(int B, int Hkv, int b) {
-    return kCtrFixed + B * Hkv + b;
+    (void)Hkv;
+    return kCtrFixed + b;
 }
 __host__ __device__ __forceinline__ int ctr_words(int B, int Hkv) {
-    return kCtrFixed + B * Hkv + B;
+    (void)Hkv;
+    return kCtrFixed + B;
 }
 
 constexpr int kLastTileFlag = 1;
@@ -105,13 +104,11 @@ struct Params {
     int B, Hq, Hkv, Lmax, S, W;
     float qscale;   // log2(e) / sqrt(d): scores come out in the log2 domain
     float lambda;
-    int c1, n1;     // sink-set items: tokens per item, items per (b, kv head)
+    int c1, n1;     // sink-set items: tokens per item, CTAs (cluster size) per (b, kv head)
     int n2;         // middle chunks per (b, kv head)
     unsigned fq[kMaxChunks + 1];  // chunk c covers middle tiles
                                   // [mt * fq[c] >> 24, mt * fq[c+1] >> 24)
     unsigned* ctr;
-    float* spart_ml;  // [B][Hq][n1][2]   sink-set item partials
-    float* spart_o;   // [B][Hq][n1][D]
     float* spec_ml;   // [B][Hq][2]       merged sink-set partial
     float* spec_o;    // [B][Hq][D]
     float* mid_ml;    // [B][Hq][n2][2]   middle item partials
@@ -158,8 +155,6 @@ __host__ __device__ __forceinline__ int spec_tiles(const SeqGeom& g, int TT) {
     return cdiv(g.ns, TT) + cdiv(g.L - g.ws, TT);
 }
 
-__device__ __forceinline__ int per_spec_items(const Params& p) { return p.n1; }
-
 // Middle tiles [t_lo, t_hi) of chunk c, for a middle of mid_tiles tiles.
 __device__ __forceinline__ void mid_chunk(const Params& p, int mid_tiles, int c, int& t_lo,
                                           int& t_hi) {
@@ -177,8 +172,10 @@ struct Item {
 template <bool SPEC, int TT>
 __device__ __forceinline__ Item decode_item(const Params& p, int item, bool flag) {
     Item it;
-    const int bh = item % (p.B * p.Hkv);
-    it.chunk = item / (p.B * p.Hkv);
+    // Sink-set items of one head are consecutive (one cluster); middle items
+    // are chunk-major across heads.
+    const int bh = SPEC ? item / p.n1 : item % (p.B * p.Hkv);
+    it.chunk = SPEC ? item % p.n1 : item / (p.B * p.Hkv);
     it.b = bh / p.Hkv;
     it.kvh = bh % p.Hkv;
     const SeqGeom g = seq_geom(p, it.b, flag);
@@ -277,30 +274,31 @@ struct Cfg {
     static constexpr int kDepositBytes = NCW * kSlotFloats * 4;
     static constexpr int kSpwMax = SPEC ? 3 : (MMA ? ALSPEC_MID_SPW : 4);
     static constexpr int kSpwBudget =
-        (kSmemLimit - 1024 - kDepositBytes - 4096) / (NTW * kStageBytes);
+        (kSmemLimit - 1024 - kDepositBytes - 4096 - (SPEC ? G * (D + 2) * 4 : 0)) /
+        (NTW * kStageBytes);
     static constexpr int SPW = kSpwBudget < 1 ? 1 : (kSpwBudget > kSpwMax ? kSpwMax : kSpwBudget);
     static constexpr int STAGES = NTW * SPW;
     // Dynamic shared memory layout (offsets from a 1024-byte aligned base).
     static constexpr int kOffDeposit = STAGES * kStageBytes;
     static constexpr int kOffMeta = kOffDeposit + kDepositBytes;
     static constexpr int kOffBar = kOffMeta + STAGES * 16;
-    static constexpr int kNumBars = 2 * STAGES + 4;
+    static constexpr int kNumBars = 2 * STAGES + 2;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-    static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
+    // Sink-set kernel: this CTA's merged partial, read by its cluster peers.
+    static constexpr int kOffCPart = kOffMisc + 16;
+    static constexpr int kCPartBytes = SPEC ? G * (D + 2) * 4 : 0;
+    static constexpr int kSmemBytes = kOffCPart + kCPartBytes + 1024;  // + alignment slack
     static_assert(kRowBytes % 128 == 0, "row must be a multiple of 128 bytes");
     static_assert(G == 1 || G == 2 || G == 4 || G == 8, "group size");
     static_assert(!MMA || (sizeof(T) == 2 && G <= 8), "tensor-core engine: bf16, g <= 8");
     static_assert(kSmemBytes <= kSmemLimit, "shared memory budget");
     static_assert(NTW >= 1 && NCW <= 8, "warp split");
-    // The sink-set merge reuses the deposit area for (m, l) of G x 32 items.
-    static_assert(kDepositBytes >= G * 32 * 8, "deposit area too small");
 };
 
 // ---------------------------------------------------------------- waiting
 
 struct Shared {
     int abort;
-    int last;
 };
 
 // Producer-side bounded wait (one thread).
@@ -700,51 +698,58 @@ struct EngineOf<C, T, D, G, true> {
     using type = MmaEngine<C, D, G>;
 };
 
-// ------------------------------------------------------------ the kernel
-
-template <typename T, int D, int G, bool SPEC, bool MMA>
-__global__ void __launch_bounds__(Cfg<T, D, G, SPEC, MMA>::kThreads, 1)
-    attn_kernel(const __grid_constant__ Params p) {
-    using C = Cfg<T, D, G, SPEC, MMA>;
-    using Engine = typename EngineOf<C, T, D, G, MMA>::type;
-    constexpr int TT = C::TT;
-    extern __shared__ unsigned char smem_raw[];
-    unsigned char* smem = reinterpret_cast<unsigned char*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    float* deposit = reinterpret_cast<float*>(smem + C::kOffDeposit);
-    int4* meta = reinterpret_cast<int4*>(smem + C::kOffMeta);
-    uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
-    uint64_t* empty_bar = full_bar + C::STAGES;
-    uint64_t* dep_bar = empty_bar + C::STAGES;  // consumer warps: phase sync
-    uint64_t* free_bar = dep_bar + 1;           // consumer warps: writes done
-    uint64_t* tk_bar = dep_bar + 2;             // ticket result published
-    Shared* sh = reinterpret_cast<Shared*>(smem + C::kOffMisc);
-    volatile int* abort = &sh->abort;
-
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-    const int n_items = p.B * p.Hkv * (SPEC ? p.n1 : p.n2);
-
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < C::STAGES; ++s) {
-            mbar_init(full_bar + s, 1);
-            mbar_init(empty_bar + s, C::NHW);
+// Sink-set kernel, several CTAs per head: the CTAs of a cluster hold their
+// partials in shared memory; after a cluster barrier CTA r merges outputs
+// [r * G * D / n1, (r + 1) * G * D / n1) from every CTA's partial (fixed
+// rank order) and writes them; a second barrier keeps every CTA's shared
+// memory alive until its peers have read it.  Every thread of every CTA
+// reaches both barriers (all waits before them are bounded).
+template <int D, int G, int NCW>
+__device__ __forceinline__ void cluster_merge(const Params& p, float* cpart, int warp, int lane) {
+    cluster_sync();
+    const int n = p.n1;
+    const int rank = (int)cluster_ctarank();
+    const int bh0 = (int)blockIdx.x / n;
+    const int b = bh0 / p.Hkv;
+    const int kvh = bh0 % p.Hkv;
+    if (warp < NCW) {
+        const int per = (G * D + n - 1) / n;
+        const uint32_t local = smem_addr(cpart);
+        for (int idx = rank * per + warp * 32 + lane; idx < min(G * D, (rank + 1) * per);
+             idx += NCW * 32) {
+            const int hh = idx / D;
+            const int e = idx % D;
+            const uint32_t off = (uint32_t)(hh * (D + 2)) * 4u;
+            float M = -INFINITY;
+            for (int j = 0; j < n; ++j) M = fmaxf(M, ld_dsmem(dsmem_addr(local + off, j)));
+            float L = 0.f, O = 0.f;
+            for (int j = 0; j < n; ++j) {
+                const uint32_t base = dsmem_addr(local + off, j);
+                const float f = merge_weight(ld_dsmem(base), M);
+                L = fmaf(f, ld_dsmem(base + 4u), L);
+                O = fmaf(f, ld_dsmem(base + 8u + 4u * e), O);
+            }
+            const size_t bh = (size_t)b * p.Hq + kvh * G + hh;
+            if (e == 0) {
+                p.spec_ml[bh * 2] = M;
+                p.spec_ml[bh * 2 + 1] = L;
+            }
+            p.spec_o[bh * D + e] = O;
+            p.out_spec[bh * D + e] = __fdiv_rn(O, L);
         }
-        mbar_init(dep_bar, C::NCW);
-        mbar_init(free_bar, C::NCW);
-        mbar_init(tk_bar, 1);
-        sh->abort = 0;
-        sh->last = 0;
-        fence_barrier_init();
     }
-    // The merge kernel that follows this (middle) kernel may be resident
-    // already: it only prepares until this grid has completed.
-    if (!SPEC) pdl_launch_dependents();
-    __syncthreads();
+    cluster_sync();
+}
 
-    if (warp == C::NCW) {
-        // ---------------------------------------------------- producer
-        if (lane != 0) return;
+// Producer lane: pull items, fill the stage ring, send end markers.
+template <typename T, int D, int G, bool SPEC, bool MMA>
+__device__ __forceinline__ void produce(const Params& p, unsigned char* smem, int4* meta,
+                                        uint64_t* full_bar, uint64_t* empty_bar,
+                                        volatile int* abort) {
+    using C = Cfg<T, D, G, SPEC, MMA>;
+    constexpr int TT = C::TT;
+    const int n_items = p.B * p.Hkv * (SPEC ? p.n1 : p.n2);
+    {
         if (MMA) {
             prefetch_tmap(&p.tmap_k);
             prefetch_tmap(&p.tmap_v);
@@ -830,9 +835,21 @@ __global__ void __launch_bounds__(Cfg<T, D, G, SPEC, MMA>::kThreads, 1)
                 atomicExch(p.ctr + kCtrDone, 0u);
             }
         }
-        return;
     }
+}
 
+// Consumer warps: compute tiles; at each item's end merge the warps' states
+// and write the item's partial (or, for the sink set, O_spec / this CTA's
+// share of it).
+template <typename T, int D, int G, bool SPEC, bool MMA>
+__device__ __forceinline__ void consume(const Params& p, unsigned char* smem, float* deposit,
+                                        float* cpart, int4* meta, uint64_t* full_bar,
+                                        uint64_t* empty_bar, uint64_t* dep_bar, uint64_t* free_bar,
+                                        volatile int* abort) {
+    using C = Cfg<T, D, G, SPEC, MMA>;
+    using Engine = typename EngineOf<C, T, D, G, MMA>::type;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
     // -------------------------------------------------------- consumers
     const int hw = warp / C::NTW;   // which GW heads of the group
     const int tw = warp % C::NTW;   // which token slot of the round
@@ -840,31 +857,18 @@ __global__ void __launch_bounds__(Cfg<T, D, G, SPEC, MMA>::kThreads, 1)
     st.reset();
     // Phase counters of the consumer-only barriers (all consumer warps run
     // the same sequence of syncs, so the counters agree across warps).
-    uint32_t ph_dep = 0, ph_free = 0, ph_tk = 0;
+    uint32_t ph_dep = 0, ph_free = 0;
     auto sync_on = [&](uint64_t* bar, uint32_t& ph) {
         __syncwarp();
         if (lane == 0) mbar_arrive(bar);
         return wait_warp(bar, (ph++) & 1, abort, p, lane);
     };
-    // Ticket taken by one thread; the result reaches every consumer warp.
-    auto ticket = [&](unsigned* word, unsigned total) {
-        if (warp == 0 && lane == 0) {
-            const unsigned t = atomicAdd(word, 1u);
-            const int last = t == total - 1;
-            if (last) atomicExch(word, 0u);
-            __threadfence();
-            sh->last = last;
-            mbar_arrive(tk_bar);
-        }
-        if (!wait_warp(tk_bar, (ph_tk++) & 1, abort, p, lane)) return -1;
-        return sh->last;
-    };
     uint32_t gt = tw;
     int b = 0, kvh = 0, chunk = 0;
     if (SPEC) {
         // The item is known up front: fetch q while the first tiles load.
-        const int bh = (int)blockIdx.x % (p.B * p.Hkv);
-        chunk = (int)blockIdx.x / (p.B * p.Hkv);
+        const int bh = (int)blockIdx.x / p.n1;
+        chunk = (int)blockIdx.x % p.n1;
         b = bh / p.Hkv;
         kvh = bh % p.Hkv;
         st.load_query(p, b, kvh * G + hw * C::GW, lane);
@@ -894,8 +898,8 @@ __global__ void __launch_bounds__(Cfg<T, D, G, SPEC, MMA>::kThreads, 1)
         if (!sync_on(dep_bar, ph_dep)) break;
         {
             const int ctid = warp * 32 + lane;
-            float* part_ml = SPEC ? p.spart_ml : p.mid_ml;
-            float* part_o = SPEC ? p.spart_o : p.mid_o;
+            float* part_ml = p.mid_ml;
+            float* part_o = p.mid_o;
             const int per = SPEC ? p.n1 : p.n2;
             for (int idx = ctid; idx < G * D; idx += C::NCW * 32) {
                 const int hh = idx / D;
@@ -914,15 +918,24 @@ __global__ void __launch_bounds__(Cfg<T, D, G, SPEC, MMA>::kThreads, 1)
                     O = fmaf(f, ws[2 + e], O);
                 }
                 const size_t bh = (size_t)b * p.Hq + kvh * G + hh;
-                if (SPEC && per == 1) {
-                    // A single sink-set item per head is the whole sink set:
-                    // publish O_spec directly.
-                    if (e == 0) {
-                        p.spec_ml[bh * 2] = M;
-                        p.spec_ml[bh * 2 + 1] = L;
+                if (SPEC) {
+                    if (per == 1) {
+                        // A single sink-set item per head is the whole sink
+                        // set: publish O_spec directly.
+                        if (e == 0) {
+                            p.spec_ml[bh * 2] = M;
+                            p.spec_ml[bh * 2 + 1] = L;
+                        }
+                        p.spec_o[bh * D + e] = O;
+                        p.out_spec[bh * D + e] = __fdiv_rn(O, L);
+                    } else {
+                        // Keep this CTA's partial for the cluster merge.
+                        if (e == 0) {
+                            cpart[hh * (D + 2)] = M;
+                            cpart[hh * (D + 2) + 1] = L;
+                        }
+                        cpart[hh * (D + 2) + 2 + e] = O;
                     }
-                    p.spec_o[bh * D + e] = O;
-                    p.out_spec[bh * D + e] = __fdiv_rn(O, L);
                     continue;
                 }
                 const size_t row = bh * per + chunk;
@@ -933,51 +946,67 @@ __global__ void __launch_bounds__(Cfg<T, D, G, SPEC, MMA>::kThreads, 1)
                 part_o[row * D + e] = O;
             }
         }
-        if (SPEC && per_spec_items(p) > 1) __threadfence();  // read by another CTA's merge
         // Every consumer thread's partial is written (and the deposit slots
         // are free again) once this sync passes.
         if (!sync_on(free_bar, ph_free)) break;
         st.reset();
-        if (SPEC && p.n1 > 1) {
-            const SeqGeom g = seq_geom(p, b, false);
-            // ---- the CTA finishing last for (b, kv head) merges every
-            // sink-set item of that head into O_spec.
-            const int nch = cdiv(spec_tiles(g, TT), p.c1 / TT);
-            const int last = ticket(p.ctr + ctr_spec(p.B, p.Hkv, b, kvh), (unsigned)nch);
-            if (last < 0) break;
-            if (!last) continue;
-            // Stage every item's (m, l) in shared memory (the deposit area is
-            // free now), then each thread merges its outputs.
-            float2* ml = reinterpret_cast<float2*>(deposit);
-            const int ctid = warp * 32 + lane;
-            for (int i = ctid; i < G * nch; i += C::NCW * 32) {
-                const size_t r = ((size_t)b * p.Hq + kvh * G + i / nch) * p.n1 + i % nch;
-                ml[i] = __ldcg(reinterpret_cast<const float2*>(p.spart_ml) + r);
-            }
-            if (!sync_on(dep_bar, ph_dep)) break;
-            for (int idx = ctid; idx < G * D; idx += C::NCW * 32) {
-                const int hh = idx / D;
-                const int e = idx % D;
-                const size_t bh = (size_t)b * p.Hq + kvh * G + hh;
-                float M = -INFINITY;
-                for (int c = 0; c < nch; ++c) M = fmaxf(M, ml[hh * nch + c].x);
-                float L = 0.f, O = 0.f;
-#pragma unroll 8
-                for (int c = 0; c < nch; ++c) {
-                    const float f = merge_weight(ml[hh * nch + c].x, M);
-                    L = fmaf(f, ml[hh * nch + c].y, L);
-                    O = fmaf(f, __ldcg(p.spart_o + (bh * p.n1 + c) * D + e), O);
-                }
-                if (e == 0) {
-                    p.spec_ml[bh * 2] = M;
-                    p.spec_ml[bh * 2 + 1] = L;
-                }
-                p.spec_o[bh * D + e] = O;
-                p.out_spec[bh * D + e] = __fdiv_rn(O, L);
-            }
-            if (!sync_on(free_bar, ph_free)) break;
-        }
     }
+}
+// ------------------------------------------------------------ the kernel
+
+template <typename T, int D, int G, bool SPEC, bool MMA>
+__global__ void __launch_bounds__(Cfg<T, D, G, SPEC, MMA>::kThreads, 1)
+    attn_kernel(const __grid_constant__ Params p) {
+    using C = Cfg<T, D, G, SPEC, MMA>;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* smem = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    float* deposit = reinterpret_cast<float*>(smem + C::kOffDeposit);
+    int4* meta = reinterpret_cast<int4*>(smem + C::kOffMeta);
+    uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+    uint64_t* empty_bar = full_bar + C::STAGES;
+    uint64_t* dep_bar = empty_bar + C::STAGES;  // consumer warps: phase sync
+    uint64_t* free_bar = dep_bar + 1;           // consumer warps: writes done
+    Shared* sh = reinterpret_cast<Shared*>(smem + C::kOffMisc);
+    volatile int* abort = &sh->abort;
+    float* cpart = reinterpret_cast<float*>(smem + C::kOffCPart);
+    // Sink-set kernel with several CTAs per head: those CTAs are one cluster.
+    const bool clustered = SPEC && p.n1 > 1;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(full_bar + s, 1);
+            mbar_init(empty_bar + s, C::NHW);
+        }
+        mbar_init(dep_bar, C::NCW);
+        mbar_init(free_bar, C::NCW);
+        sh->abort = 0;
+        fence_barrier_init();
+    }
+    if (clustered) {
+        // An empty partial (m = -inf, l = 0, o = 0): a CTA whose slice of a
+        // short sink set has no tiles contributes nothing to the merge.
+        for (int i = threadIdx.x; i < G * (D + 2); i += C::kThreads)
+            cpart[i] = i % (D + 2) == 0 ? -INFINITY : 0.f;
+    }
+    // The merge kernel that follows this (middle) kernel may be resident
+    // already: it only prepares until this grid has completed.
+    if (!SPEC) pdl_launch_dependents();
+    __syncthreads();
+
+    if (warp == C::NCW) {
+        // ---------------------------------------------------- producer
+        if (lane == 0) produce<T, D, G, SPEC, MMA>(p, smem, meta, full_bar, empty_bar, abort);
+        if (!clustered) return;
+        __syncwarp();  // the warp waits for its producer lane, then joins the cluster merge
+    } else {
+        consume<T, D, G, SPEC, MMA>(p, smem, deposit, cpart, meta, full_bar, empty_bar, dep_bar,
+                                    free_bar, abort);
+    }
+    if (clustered) cluster_merge<D, G, C::NCW>(p, cpart, warp, lane);
 }
 
 // ------------------------------------------------------- merge + verify

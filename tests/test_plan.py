@@ -40,7 +40,12 @@ def tiles_of(B, Hq, Hkv, d, Lmax, dtype, S, W, lens, split=0, engine="auto"):
     for spec in (True, False):
         per = n1 if spec else n2
         for item in range(B * Hkv * per):
-            bh, chunk = item % (B * Hkv), item // (B * Hkv)
+            # Sink-set CTAs of one head are consecutive (one cluster); middle
+            # items are chunk-major across heads.
+            if spec:
+                bh, chunk = item // n1, item % n1
+            else:
+                bh, chunk = item % (B * Hkv), item // (B * Hkv)
             b, kvh = bh // Hkv, bh % Hkv
             L = lens[b]
             ns, ws = geom(L, S, W)
@@ -124,9 +129,9 @@ def test_guided_chunks_shrink_and_fill_the_grid():
     sizes = [b - a for a, b in zip(fq, fq[1:])]
     assert sizes[0] >= sizes[-1] * 4          # large chunks first, small at the end
     assert all(x >= y - 2 for x, y in zip(sizes, sizes[1:]))  # non-increasing (rounding)
-    # The sink-set kernel (one CTA per head here) and the middle kernel fit
-    # on the GPU together.
-    assert plan["n1"] == 1 and plan["grid2"] + 8 <= 148
+    # The sink-set kernel runs as a cluster of a few CTAs per head (8 heads
+    # here) within half of the GPU; the middle kernel takes every SM.
+    assert 1 < plan["n1"] <= 8 and 8 * plan["n1"] <= 74 and plan["grid2"] == 148
 
 
 def test_query_chunks_rejects_small_buffer():
