@@ -24,9 +24,8 @@ namespace {
 constexpr int kMaxDevices = 64;
 constexpr int kMaxSpecItems = 8;  // sink-set CTAs per (sequence, KV head): a portable cluster
 
-// The sink-set kernel gets about 1/ALSPEC_SPEC_SM_DIV of the SMs.
-#ifndef ALSPEC_SPEC_SM_DIV
-#define ALSPEC_SPEC_SM_DIV 4
+#ifndef ALSPEC_MID_SM_RESERVE
+#define ALSPEC_MID_SM_RESERVE 0
 #endif
 constexpr size_t kAlign = 256;
 
@@ -171,10 +170,10 @@ void make_plan(const alspec_desc& d, int S, int W, int sms, Plan* pl) {
     const int ns = std::min(S, L);
     const int mid_max = std::max(0, std::max(ns, L - W) - ns);
     const int mid_tiles = ceil_div(mid_max, TT);
-    // The persistent middle kernel takes every SM: CTAs that find an SM
-    // busy with the (short) sink-set kernel start when it is done, and the
-    // atomic queue balances the work.
-    const int P = sms;
+    // The persistent middle kernel takes every SM (less ALSPEC_MID_SM_RESERVE):
+    // CTAs that find an SM busy with the (short) sink-set kernel start when
+    // it is done, and the atomic queue balances the work.
+    const int P = std::max(1, sms - ALSPEC_MID_SM_RESERVE);
     std::vector<double> sizes;  // chunk sizes as fractions of a head's middle
     if (mid_tiles > 0) {
         if (d.split_tokens > 0) {

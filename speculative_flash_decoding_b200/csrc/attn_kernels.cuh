@@ -274,8 +274,7 @@ struct Cfg {
     static constexpr int kDepositBytes = NCW * kSlotFloats * 4;
     static constexpr int kSpwMax = SPEC ? 3 : (MMA ? ALSPEC_MID_SPW : 4);
     static constexpr int kSpwBudget =
-        (kSmemLimit - 1024 - kDepositBytes - 4096 - (SPEC ? G * (D + 2) * 4 : 0)) /
-        (NTW * kStageBytes);
+        (kSmemLimit - 1024 - kDepositBytes - 4096) / (NTW * kStageBytes);
     static constexpr int SPW = kSpwBudget < 1 ? 1 : (kSpwBudget > kSpwMax ? kSpwMax : kSpwBudget);
     static constexpr int STAGES = NTW * SPW;
     // Dynamic shared memory layout (offsets from a 1024-byte aligned base).
@@ -284,10 +283,7 @@ struct Cfg {
     static constexpr int kOffBar = kOffMeta + STAGES * 16;
     static constexpr int kNumBars = 2 * STAGES + 2;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-    // Sink-set kernel: this CTA's merged partial, read by its cluster peers.
-    static constexpr int kOffCPart = kOffMisc + 16;
-    static constexpr int kCPartBytes = SPEC ? G * (D + 2) * 4 : 0;
-    static constexpr int kSmemBytes = kOffCPart + kCPartBytes + 1024;  // + alignment slack
+    static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
     static_assert(kRowBytes % 128 == 0, "row must be a multiple of 128 bytes");
     static_assert(G == 1 || G == 2 || G == 4 || G == 8, "group size");
     static_assert(!MMA || (sizeof(T) == 2 && G <= 8), "tensor-core engine: bf16, g <= 8");
@@ -698,36 +694,75 @@ struct EngineOf<C, T, D, G, true> {
     using type = MmaEngine<C, D, G>;
 };
 
-// Sink-set kernel, several CTAs per head: the CTAs of a cluster hold their
-// partials in shared memory; after a cluster barrier CTA r merges outputs
-// [r * G * D / n1, (r + 1) * G * D / n1) from every CTA's partial (fixed
-// rank order) and writes them; a second barrier keeps every CTA's shared
+// Sink-set kernel, several CTAs per head (one cluster): every consumer warp
+// of every CTA leaves its state (m, l, o for its GW heads) in its deposit
+// slot.  After a cluster barrier CTA r merges outputs
+// [r * G * D / n1, (r + 1) * G * D / n1) from all n1 x NTW states of the
+// head (fixed order: rank, then token slot; all loads of an output issued
+// together) and writes them; a second barrier keeps every CTA's shared
 // memory alive until its peers have read it.  Every thread of every CTA
 // reaches both barriers (all waits before them are bounded).
-template <int D, int G, int NCW>
-__device__ __forceinline__ void cluster_merge(const Params& p, float* cpart, int warp, int lane) {
+template <int D, int G, class C>
+__device__ __forceinline__ void cluster_merge(const Params& p, float* deposit, int warp, int lane) {
+    constexpr int kMaxRanks = 8;
     cluster_sync();
     const int n = p.n1;
     const int rank = (int)cluster_ctarank();
     const int bh0 = (int)blockIdx.x / n;
     const int b = bh0 / p.Hkv;
     const int kvh = bh0 % p.Hkv;
-    if (warp < NCW) {
+    if (warp < C::NCW) {
         const int per = (G * D + n - 1) / n;
-        const uint32_t local = smem_addr(cpart);
+        const uint32_t local = smem_addr(deposit);
         for (int idx = rank * per + warp * 32 + lane; idx < min(G * D, (rank + 1) * per);
-             idx += NCW * 32) {
+             idx += C::NCW * 32) {
             const int hh = idx / D;
             const int e = idx % D;
-            const uint32_t off = (uint32_t)(hh * (D + 2)) * 4u;
-            float M = -INFINITY;
-            for (int j = 0; j < n; ++j) M = fmaxf(M, ld_dsmem(dsmem_addr(local + off, j)));
-            float L = 0.f, O = 0.f;
-            for (int j = 0; j < n; ++j) {
-                const uint32_t base = dsmem_addr(local + off, j);
-                const float f = merge_weight(ld_dsmem(base), M);
-                L = fmaf(f, ld_dsmem(base + 4u), L);
-                O = fmaf(f, ld_dsmem(base + 8u + 4u * e), O);
+            // State of head hh in token slot w: slot (hh / GW) * NTW + w,
+            // head hh % GW inside it.
+            const uint32_t head_off =
+                (uint32_t)(((hh / C::GW) * C::NTW) * C::kSlotFloats + (hh % C::GW) * (D + 2)) * 4u;
+            // Ranks in groups of R whose states fit in registers; all loads of
+            // a group are issued together, groups merge online.
+            constexpr int R = C::NTW <= 4 ? kMaxRanks : kMaxRanks / 2;
+            float M = -INFINITY, L = 0.f, O = 0.f;
+            for (int j0 = 0; j0 < n; j0 += R) {
+                float m[R][C::NTW], l[R][C::NTW], o[R][C::NTW];
+#pragma unroll
+                for (int j = 0; j < R; ++j) {
+#pragma unroll
+                    for (int w = 0; w < C::NTW; ++w) {
+                        if (j0 + j < n) {
+                            const uint32_t a =
+                                dsmem_addr(local + head_off + (uint32_t)(w * C::kSlotFloats) * 4u,
+                                           (uint32_t)(j0 + j));
+                            m[j][w] = ld_dsmem(a);
+                            l[j][w] = ld_dsmem(a + 4u);
+                            o[j][w] = ld_dsmem(a + 8u + 4u * e);
+                        } else {
+                            m[j][w] = -INFINITY;
+                            l[j][w] = 0.f;
+                            o[j][w] = 0.f;
+                        }
+                    }
+                }
+                float Mg = M;
+#pragma unroll
+                for (int j = 0; j < R; ++j)
+#pragma unroll
+                    for (int w = 0; w < C::NTW; ++w) Mg = fmaxf(Mg, m[j][w]);
+                const float f0 = merge_weight(M, Mg);
+                L *= f0;
+                O *= f0;
+#pragma unroll
+                for (int j = 0; j < R; ++j)
+#pragma unroll
+                    for (int w = 0; w < C::NTW; ++w) {
+                        const float f = merge_weight(m[j][w], Mg);
+                        L = fmaf(f, l[j][w], L);
+                        O = fmaf(f, o[j][w], O);
+                    }
+                M = Mg;
             }
             const size_t bh = (size_t)b * p.Hq + kvh * G + hh;
             if (e == 0) {
@@ -843,7 +878,7 @@ __device__ __forceinline__ void produce(const Params& p, unsigned char* smem, in
 // share of it).
 template <typename T, int D, int G, bool SPEC, bool MMA>
 __device__ __forceinline__ void consume(const Params& p, unsigned char* smem, float* deposit,
-                                        float* cpart, int4* meta, uint64_t* full_bar,
+                                        int4* meta, uint64_t* full_bar,
                                         uint64_t* empty_bar, uint64_t* dep_bar, uint64_t* free_bar,
                                         volatile int* abort) {
     using C = Cfg<T, D, G, SPEC, MMA>;
@@ -895,6 +930,12 @@ __device__ __forceinline__ void consume(const Params& p, unsigned char* smem, fl
 
         // ---- end of this item: combine the warps' states into one partial.
         st.deposit(deposit + (hw * C::NTW + tw) * C::kSlotFloats, lane);
+        if (SPEC && p.n1 > 1) {
+            // Sink set split over a cluster: the warps' states stay in the
+            // deposit slots and the cluster merge reads them directly.
+            __syncwarp();
+            continue;
+        }
         if (!sync_on(dep_bar, ph_dep)) break;
         {
             const int ctid = warp * 32 + lane;
@@ -919,23 +960,14 @@ __device__ __forceinline__ void consume(const Params& p, unsigned char* smem, fl
                 }
                 const size_t bh = (size_t)b * p.Hq + kvh * G + hh;
                 if (SPEC) {
-                    if (per == 1) {
-                        // A single sink-set item per head is the whole sink
-                        // set: publish O_spec directly.
-                        if (e == 0) {
-                            p.spec_ml[bh * 2] = M;
-                            p.spec_ml[bh * 2 + 1] = L;
-                        }
-                        p.spec_o[bh * D + e] = O;
-                        p.out_spec[bh * D + e] = __fdiv_rn(O, L);
-                    } else {
-                        // Keep this CTA's partial for the cluster merge.
-                        if (e == 0) {
-                            cpart[hh * (D + 2)] = M;
-                            cpart[hh * (D + 2) + 1] = L;
-                        }
-                        cpart[hh * (D + 2) + 2 + e] = O;
+                    // A single sink-set CTA per head holds the whole sink
+                    // set: publish O_spec directly.
+                    if (e == 0) {
+                        p.spec_ml[bh * 2] = M;
+                        p.spec_ml[bh * 2 + 1] = L;
                     }
+                    p.spec_o[bh * D + e] = O;
+                    p.out_spec[bh * D + e] = __fdiv_rn(O, L);
                     continue;
                 }
                 const size_t row = bh * per + chunk;
@@ -969,7 +1001,6 @@ __global__ void __launch_bounds__(Cfg<T, D, G, SPEC, MMA>::kThreads, 1)
     uint64_t* free_bar = dep_bar + 1;           // consumer warps: writes done
     Shared* sh = reinterpret_cast<Shared*>(smem + C::kOffMisc);
     volatile int* abort = &sh->abort;
-    float* cpart = reinterpret_cast<float*>(smem + C::kOffCPart);
     // Sink-set kernel with several CTAs per head: those CTAs are one cluster.
     const bool clustered = SPEC && p.n1 > 1;
 
@@ -987,10 +1018,11 @@ __global__ void __launch_bounds__(Cfg<T, D, G, SPEC, MMA>::kThreads, 1)
         fence_barrier_init();
     }
     if (clustered) {
-        // An empty partial (m = -inf, l = 0, o = 0): a CTA whose slice of a
-        // short sink set has no tiles contributes nothing to the merge.
-        for (int i = threadIdx.x; i < G * (D + 2); i += C::kThreads)
-            cpart[i] = i % (D + 2) == 0 ? -INFINITY : 0.f;
+        // Empty states (m = -inf, l = 0, o = 0) in every warp's deposit slot:
+        // a CTA whose slice of a short sink set has no tiles (or a warp with
+        // only padding tiles) contributes nothing to the merge.
+        for (int i = threadIdx.x; i < C::NCW * C::kSlotFloats; i += C::kThreads)
+            deposit[i] = (i % C::kSlotFloats) % (D + 2) == 0 ? -INFINITY : 0.f;
     }
     // The merge kernel that follows this (middle) kernel may be resident
     // already: it only prepares until this grid has completed.
@@ -1003,10 +1035,10 @@ __global__ void __launch_bounds__(Cfg<T, D, G, SPEC, MMA>::kThreads, 1)
         if (!clustered) return;
         __syncwarp();  // the warp waits for its producer lane, then joins the cluster merge
     } else {
-        consume<T, D, G, SPEC, MMA>(p, smem, deposit, cpart, meta, full_bar, empty_bar, dep_bar,
+        consume<T, D, G, SPEC, MMA>(p, smem, deposit, meta, full_bar, empty_bar, dep_bar,
                                     free_bar, abort);
     }
-    if (clustered) cluster_merge<D, G, C::NCW>(p, cpart, warp, lane);
+    if (clustered) cluster_merge<D, G, C>(p, deposit, warp, lane);
 }
 
 // ------------------------------------------------------- merge + verify
