@@ -595,18 +595,22 @@ struct MmaEngine {
         const uint32_t kb = smem_addr(ks);
         const uint32_t vb = smem_addr(vs);
 
-        // S^T = Q K^T: 4 n-tiles of 8 tokens.
+        // S^T = Q K^T: 4 n-tiles of 8 tokens.  Even and odd k-steps go to
+        // separate accumulators (half-length MMA dependency chains).
         float s[TT / 8][4];
 #pragma unroll
         for (int j = 0; j < TT / 8; ++j) {
+            float s2[4] = {0.f, 0.f, 0.f, 0.f};
             s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
 #pragma unroll
             for (int kp = 0; kp < KS / 2; ++kp) {
                 uint32_t b0, b1, b2, b3;
                 ldsm_x4(addr(kb, 8 * j + (lane & 7), 4 * kp + (lane >> 3)), b0, b1, b2, b3);
                 mma_bf16_16816(s[j], qa[2 * kp][0], 0u, qa[2 * kp][1], 0u, b0, b1);
-                mma_bf16_16816(s[j], qa[2 * kp + 1][0], 0u, qa[2 * kp + 1][1], 0u, b2, b3);
+                mma_bf16_16816(s2, qa[2 * kp + 1][0], 0u, qa[2 * kp + 1][1], 0u, b2, b3);
             }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) s[j][i] += s2[i];
         }
 
         // Online softmax on row g (lanes 4g..4g+3 hold its 32 scores).
