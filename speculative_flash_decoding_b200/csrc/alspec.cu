@@ -165,6 +165,7 @@ void make_plan(const alspec_desc& d, int S, int W, int sms, Plan* pl) {
     pl->n1 = std::max(1, std::min({kMaxSpecItems, room1, ceil_div(tiles_max, 4)}));
     const int tiles_per_item = ceil_div(tiles_max, pl->n1);
     pl->c1 = tiles_per_item * TT;
+    pl->n1 = ceil_div(tiles_max, tiles_per_item);  // no CTA without tiles at L_max
     pl->grid1 = heads * pl->n1;
 
     const int ns = std::min(S, L);
