@@ -158,11 +158,11 @@ void make_plan(const alspec_desc& d, int S, int W, int sms, Plan* pl) {
     const int heads = d.batch * d.n_kv_heads;
     const int L = d.max_seq_len;
     const int tiles_max = ceil_div(std::min(S, L), TT) + ceil_div(std::min(W, L), TT);
-    // CTAs per head for the sink set (one thread-block cluster): about 4
+    // CTAs per head for the sink set (one thread-block cluster): about 7
     // tiles each (one per consumer warp), at most 8 (the portable cluster
     // size), and all heads together within half of the SMs.
     const int room1 = std::max(1, sms / 2 / std::max(1, heads));
-    pl->n1 = std::max(1, std::min({kMaxSpecItems, room1, ceil_div(tiles_max, 4)}));
+    pl->n1 = std::max(1, std::min({kMaxSpecItems, room1, ceil_div(tiles_max, 7)}));
     const int tiles_per_item = ceil_div(tiles_max, pl->n1);
     pl->c1 = tiles_per_item * TT;
     pl->n1 = ceil_div(tiles_max, tiles_per_item);  // no CTA without tiles at L_max

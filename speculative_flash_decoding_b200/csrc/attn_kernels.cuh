@@ -265,7 +265,9 @@ struct Cfg {
     // the former, so those configurations run 7 consumer warps.
     static constexpr int kLanePairs = (kRowBytes / 128) * Elem<T>::kPairs;
     static constexpr bool kHeavy = !MMA && GW * kLanePairs >= 32;
-    static constexpr int NTW = MMA ? 4 : (kHeavy ? 7 : 8) / NHW;
+    // Tensor-core engine: 4 consumer warps stream the middle; the sink-set
+    // kernel (latency-bound, a few tiles per CTA) uses 7, one tile each.
+    static constexpr int NTW = MMA ? (SPEC ? 7 : 4) : (kHeavy ? 7 : 8) / NHW;
     static constexpr int NCW = NTW * NHW;
     static constexpr int kThreads = (NCW + 1) * 32;
     static constexpr int kTileBytes = TT * kRowBytes;  // K or V part of a stage
@@ -274,7 +276,8 @@ struct Cfg {
     static constexpr int kDepositBytes = NCW * kSlotFloats * 4;
     static constexpr int kSpwMax = SPEC ? 3 : (MMA ? ALSPEC_MID_SPW : 4);
     static constexpr int kSpwBudget =
-        (kSmemLimit - 1024 - kDepositBytes - 4096) / (NTW * kStageBytes);
+        (kSmemLimit - 1024 - kDepositBytes - 4096 - (SPEC ? G * (D + 2) * 4 : 0)) /
+        (NTW * kStageBytes);
     static constexpr int SPW = kSpwBudget < 1 ? 1 : (kSpwBudget > kSpwMax ? kSpwMax : kSpwBudget);
     static constexpr int STAGES = NTW * SPW;
     // Dynamic shared memory layout (offsets from a 1024-byte aligned base).
@@ -283,7 +286,10 @@ struct Cfg {
     static constexpr int kOffBar = kOffMeta + STAGES * 16;
     static constexpr int kNumBars = 2 * STAGES + 2;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-    static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
+    // Sink-set kernel: this CTA's merged partial, read by its cluster peers.
+    static constexpr int kOffCPart = kOffMisc + 16;
+    static constexpr int kCPartBytes = SPEC ? G * (D + 2) * 4 : 0;
+    static constexpr int kSmemBytes = kOffCPart + kCPartBytes + 1024;  // + alignment slack
     static_assert(kRowBytes % 128 == 0, "row must be a multiple of 128 bytes");
     static_assert(G == 1 || G == 2 || G == 4 || G == 8, "group size");
     static_assert(!MMA || (sizeof(T) == 2 && G <= 8), "tensor-core engine: bf16, g <= 8");
@@ -698,16 +704,15 @@ struct EngineOf<C, T, D, G, true> {
     using type = MmaEngine<C, D, G>;
 };
 
-// Sink-set kernel, several CTAs per head (one cluster): every consumer warp
-// of every CTA leaves its state (m, l, o for its GW heads) in its deposit
-// slot.  After a cluster barrier CTA r merges outputs
-// [r * G * D / n1, (r + 1) * G * D / n1) from all n1 x NTW states of the
-// head (fixed order: rank, then token slot; all loads of an output issued
-// together) and writes them; a second barrier keeps every CTA's shared
-// memory alive until its peers have read it.  Every thread of every CTA
-// reaches both barriers (all waits before them are bounded).
+// Sink-set kernel, several CTAs per head (one cluster): each CTA holds its
+// merged partial (m, l, o for the G heads) in shared memory.  After a
+// cluster barrier CTA r merges outputs [r * G * D / n1, (r + 1) * G * D / n1)
+// from the n1 partials (rank order, all remote loads issued together) and
+// writes them; a second barrier keeps every CTA's shared memory alive until
+// its peers have read it.  Every thread of every CTA reaches both barriers
+// (all waits before them are bounded).
 template <int D, int G, class C>
-__device__ __forceinline__ void cluster_merge(const Params& p, float* deposit, int warp, int lane) {
+__device__ __forceinline__ void cluster_merge(const Params& p, float* cpart, int warp, int lane) {
     constexpr int kMaxRanks = 8;
     cluster_sync();
     const int n = p.n1;
@@ -715,69 +720,48 @@ __device__ __forceinline__ void cluster_merge(const Params& p, float* deposit, i
     const int bh0 = (int)blockIdx.x / n;
     const int b = bh0 / p.Hkv;
     const int kvh = bh0 % p.Hkv;
-    if (warp < C::NCW) {
-        const int per = (G * D + n - 1) / n;
-        const uint32_t local = smem_addr(deposit);
-        for (int idx = rank * per + warp * 32 + lane; idx < min(G * D, (rank + 1) * per);
-             idx += C::NCW * 32) {
-            const int hh = idx / D;
-            const int e = idx % D;
-            // State of head hh in token slot w: slot (hh / GW) * NTW + w,
-            // head hh % GW inside it.
-            const uint32_t head_off =
-                (uint32_t)(((hh / C::GW) * C::NTW) * C::kSlotFloats + (hh % C::GW) * (D + 2)) * 4u;
-            // Ranks in groups of R whose states fit in registers; all loads of
-            // a group are issued together, groups merge online.
-            constexpr int R = C::NTW <= 4 ? kMaxRanks : kMaxRanks / 2;
-            float M = -INFINITY, L = 0.f, O = 0.f;
-            for (int j0 = 0; j0 < n; j0 += R) {
-                float m[R][C::NTW], l[R][C::NTW], o[R][C::NTW];
+    const int per = (G * D + n - 1) / n;
+    const uint32_t local = smem_addr(cpart);
+    for (int idx = rank * per + (int)threadIdx.x; idx < min(G * D, (rank + 1) * per);
+         idx += C::kThreads) {
+        const int hh = idx / D;
+        const int e = idx % D;
+        const uint32_t off = (uint32_t)(hh * (D + 2)) * 4u;
+        float m[kMaxRanks], l[kMaxRanks], o[kMaxRanks];
 #pragma unroll
-                for (int j = 0; j < R; ++j) {
-#pragma unroll
-                    for (int w = 0; w < C::NTW; ++w) {
-                        if (j0 + j < n) {
-                            const uint32_t a =
-                                dsmem_addr(local + head_off + (uint32_t)(w * C::kSlotFloats) * 4u,
-                                           (uint32_t)(j0 + j));
-                            m[j][w] = ld_dsmem(a);
-                            l[j][w] = ld_dsmem(a + 4u);
-                            o[j][w] = ld_dsmem(a + 8u + 4u * e);
-                        } else {
-                            m[j][w] = -INFINITY;
-                            l[j][w] = 0.f;
-                            o[j][w] = 0.f;
-                        }
-                    }
-                }
-                float Mg = M;
-#pragma unroll
-                for (int j = 0; j < R; ++j)
-#pragma unroll
-                    for (int w = 0; w < C::NTW; ++w) Mg = fmaxf(Mg, m[j][w]);
-                const float f0 = merge_weight(M, Mg);
-                L *= f0;
-                O *= f0;
-#pragma unroll
-                for (int j = 0; j < R; ++j)
-#pragma unroll
-                    for (int w = 0; w < C::NTW; ++w) {
-                        const float f = merge_weight(m[j][w], Mg);
-                        L = fmaf(f, l[j][w], L);
-                        O = fmaf(f, o[j][w], O);
-                    }
-                M = Mg;
+        for (int j = 0; j < kMaxRanks; ++j) {
+            if (j < n) {
+                const uint32_t a = dsmem_addr(local + off, (uint32_t)j);
+                m[j] = ld_dsmem(a);
+                l[j] = ld_dsmem(a + 4u);
+                o[j] = ld_dsmem(a + 8u + 4u * e);
+            } else {
+                m[j] = -INFINITY;
+                l[j] = 0.f;
+                o[j] = 0.f;
             }
-            const size_t bh = (size_t)b * p.Hq + kvh * G + hh;
-            if (e == 0) {
-                p.spec_ml[bh * 2] = M;
-                p.spec_ml[bh * 2 + 1] = L;
-            }
-            p.spec_o[bh * D + e] = O;
-            p.out_spec[bh * D + e] = __fdiv_rn(O, L);
         }
+        float M = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < kMaxRanks; ++j) M = fmaxf(M, m[j]);
+        float L = 0.f, O = 0.f;
+#pragma unroll
+        for (int j = 0; j < kMaxRanks; ++j) {
+            const float f = merge_weight(m[j], M);
+            L = fmaf(f, l[j], L);
+            O = fmaf(f, o[j], O);
+        }
+        const size_t bh = (size_t)b * p.Hq + kvh * G + hh;
+        if (e == 0) {
+            p.spec_ml[bh * 2] = M;
+            p.spec_ml[bh * 2 + 1] = L;
+        }
+        p.spec_o[bh * D + e] = O;
+        p.out_spec[bh * D + e] = __fdiv_rn(O, L);
     }
     cluster_sync();
+    (void)warp;
+    (void)lane;
 }
 
 // Producer lane: pull items, fill the stage ring, send end markers.
@@ -1005,6 +989,7 @@ __global__ void __launch_bounds__(Cfg<T, D, G, SPEC, MMA>::kThreads, 1)
     uint64_t* free_bar = dep_bar + 1;           // consumer warps: writes done
     Shared* sh = reinterpret_cast<Shared*>(smem + C::kOffMisc);
     volatile int* abort = &sh->abort;
+    float* cpart = reinterpret_cast<float*>(smem + C::kOffCPart);
     // Sink-set kernel with several CTAs per head: those CTAs are one cluster.
     const bool clustered = SPEC && p.n1 > 1;
 
@@ -1042,7 +1027,28 @@ __global__ void __launch_bounds__(Cfg<T, D, G, SPEC, MMA>::kThreads, 1)
         consume<T, D, G, SPEC, MMA>(p, smem, deposit, meta, full_bar, empty_bar, dep_bar,
                                     free_bar, abort);
     }
-    if (clustered) cluster_merge<D, G, C>(p, deposit, warp, lane);
+    if (clustered) {
+        // Every thread of the CTA is here (no early exits in this mode):
+        // merge the warps' states into this CTA's partial, then the cluster.
+        __syncthreads();
+        for (int idx = threadIdx.x; idx < G * (D + 2); idx += C::kThreads) {
+            const int hh = idx / (D + 2);
+            const int e = idx % (D + 2);
+            const float* base =
+                deposit + (hh / C::GW) * C::NTW * C::kSlotFloats + (hh % C::GW) * (D + 2);
+            float M = -INFINITY;
+#pragma unroll
+            for (int w = 0; w < C::NTW; ++w) M = fmaxf(M, base[w * C::kSlotFloats]);
+            float acc = 0.f;
+#pragma unroll
+            for (int w = 0; w < C::NTW; ++w) {
+                const float* ws = base + w * C::kSlotFloats;
+                acc = fmaf(merge_weight(ws[0], M), ws[e < 2 ? 1 : e], acc);
+            }
+            cpart[idx] = e == 0 ? M : acc;  // (m, l, o[0..D)) of head hh
+        }
+        cluster_merge<D, G, C>(p, cpart, warp, lane);
+    }
 }
 
 // ------------------------------------------------------- merge + verify
