@@ -276,20 +276,28 @@ struct Cfg {
     static constexpr int kDepositBytes = NCW * kSlotFloats * 4;
     static constexpr int kSpwMax = SPEC ? 3 : (MMA ? ALSPEC_MID_SPW : 4);
     static constexpr int kSpwBudget =
-        (kSmemLimit - 1024 - kDepositBytes - 4096 - (SPEC ? G * (D + 2) * 4 : 0)) /
+        (kSmemLimit - 1024 - kDepositBytes - 4096 - 512 - (SPEC ? G * (D + 2) * 4 : 0)) /
         (NTW * kStageBytes);
     static constexpr int SPW = kSpwBudget < 1 ? 1 : (kSpwBudget > kSpwMax ? kSpwMax : kSpwBudget);
     static constexpr int STAGES = NTW * SPW;
-    // Dynamic shared memory layout (offsets from a 1024-byte aligned base).
+    // Dynamic shared memory layout (offsets from a 1024-byte aligned base;
+    // every region starts on a 128-byte boundary: the stage metadata are
+    // int4, the barriers 8-byte words).
+    static constexpr int align128(int x) { return (x + 127) / 128 * 128; }
     static constexpr int kOffDeposit = STAGES * kStageBytes;
-    static constexpr int kOffMeta = kOffDeposit + kDepositBytes;
-    static constexpr int kOffBar = kOffMeta + STAGES * 16;
+    static constexpr int kOffMeta = align128(kOffDeposit + kDepositBytes);
+    static constexpr int kOffBar = align128(kOffMeta + STAGES * 16);
     static constexpr int kNumBars = 2 * STAGES + 2;
-    static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+    static constexpr int kOffMisc = align128(kOffBar + kNumBars * 8);
     // Sink-set kernel: this CTA's merged partial, read by its cluster peers.
-    static constexpr int kOffCPart = kOffMisc + 16;
+    static constexpr int kOffCPart = align128(kOffMisc + 16);
     static constexpr int kCPartBytes = SPEC ? G * (D + 2) * 4 : 0;
     static constexpr int kSmemBytes = kOffCPart + kCPartBytes + 1024;  // + alignment slack
+    static_assert(kOffDeposit % 1024 == 0 && kStageBytes % 1024 == 0 && kTileBytes % 1024 == 0,
+                  "TMA destinations with 128-byte swizzle need 1024-byte alignment");
+    static_assert(kOffMeta % 16 == 0 && kOffBar % 8 == 0 && kOffMisc % 16 == 0 &&
+                      kOffCPart % 16 == 0 && (kSlotFloats * 4) % 8 == 0,
+                  "shared-memory region alignment");
     static_assert(kRowBytes % 128 == 0, "row must be a multiple of 128 bytes");
     static_assert(G == 1 || G == 2 || G == 4 || G == 8, "group size");
     static_assert(!MMA || (sizeof(T) == 2 && G <= 8), "tensor-core engine: bf16, g <= 8");
