@@ -158,6 +158,30 @@ alspec_status alspec_decode(const alspec_desc* desc,
                             void* stream, void* spec_event, void* const* prof_events);
 
 /*
+ * alspec_decode with publication time stamps measured by the kernels
+ * themselves (no events), for timing inside CUDA graphs, where an event
+ * record node does not mark when the work before it ended.
+ *   trace_ns  device, 2 x uint64, 8-byte aligned, zeroed by the caller
+ *             before the call.  The kernels raise (atomic max):
+ *               [0] to the global timer (ns) after the last write of O_spec,
+ *               [1] to the global timer after the last write of O_exact,
+ *                   rel_l2 and commit.
+ *             The library never reads or clears it; NULL is an
+ *             ALSPEC_ERR_INVALID_ARG.
+ * Other arguments as for alspec_decode (no spec event, no profiling events).
+ * The stamps come from the same clock for all calls on a device, so
+ * trace[0] of one call minus trace[1] of the call before it is the latency
+ * of O_spec from the end of the previous step.
+ */
+alspec_status alspec_decode_traced(const alspec_desc* desc,
+                                   const void* q, const void* k_cache, const void* v_cache,
+                                   const int32_t* seq_lens, int n_sink, int window,
+                                   float lambda, float* out_spec, float* out_exact,
+                                   float* rel_l2, uint8_t* commit,
+                                   void* workspace, size_t workspace_bytes,
+                                   void* stream, unsigned long long* trace_ns);
+
+/*
  * Work plan the library would use (host only, no CUDA call except the SM
  * count query).  info[] receives, in order:
  *   0 tokens per sink-set work item      1 sink-set items per (b, kv head)

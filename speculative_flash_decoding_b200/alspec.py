@@ -70,6 +70,8 @@ SIGNATURES = {
     "alspec_last_cuda_error": (_i, []),
     "alspec_decode_noalloc": (_i, [_descp, _vp, _vp, _vp, _vp, _i, _i, _f, _vp, _vp, _vp, _vp,
                                    _vp]),
+    "alspec_decode_traced": (_i, [_descp, _vp, _vp, _vp, _vp, _i, _i, _f, _vp, _vp, _vp, _vp,
+                                  _vp, _sz, _vp, _vp]),
 }
 
 ALSPEC_NOALLOC_SCRATCH_BYTES = 8 << 20
@@ -121,6 +123,18 @@ def alspec_decode(desc: alspec_desc, q: int, k_cache: int, v_cache: int, seq_len
     return int(_lib.alspec_decode(ctypes.byref(desc), q, k_cache, v_cache, seq_lens, n_sink,
                                   window, lam, out_spec, out_exact, rel_l2, commit, workspace,
                                   workspace_bytes, stream, spec_event or None, prof))
+
+
+def alspec_decode_traced(desc: alspec_desc, q: int, k_cache: int, v_cache: int, seq_lens: int,
+                         n_sink: int, window: int, lam: float, out_spec: int, out_exact: int,
+                         rel_l2: int, commit: int, workspace: int, workspace_bytes: int,
+                         stream: int, trace_ns: int) -> int:
+    """trace_ns: device address of 2 zeroed uint64 words; the kernels leave
+    the global-timer ns of O_spec's and O_exact's publication there."""
+    return int(_lib.alspec_decode_traced(ctypes.byref(desc), q, k_cache, v_cache, seq_lens,
+                                         n_sink, window, lam, out_spec, out_exact, rel_l2,
+                                         commit, workspace, workspace_bytes, stream,
+                                         trace_ns or None))
 
 
 def alspec_decode_noalloc(desc: alspec_desc, q: int, k_cache: int, v_cache: int, seq_lens: int,
@@ -247,11 +261,24 @@ class Decoder:
                     commit=t.empty(d.batch, dtype=t.uint8, **kw))
 
     def decode(self, q, k, v, seq_lens, lam, out=None, stream=None, spec_event=None,
-               prof_events=None):
-        """prof_events: None or ALSPEC_PROF_EVENTS torch.cuda.Event(enable_timing=True)."""
+               prof_events=None, trace=None):
+        """prof_events: None or ALSPEC_PROF_EVENTS torch.cuda.Event(enable_timing=True).
+        trace: None or a zeroed int64 device tensor of 2 elements (see
+        alspec_decode_traced); exclusive with the events."""
         t = self.torch
         out = out if out is not None else self.alloc_outputs()
         s = stream if stream is not None else t.cuda.current_stream(self.device)
+        if trace is not None:
+            if spec_event is not None or prof_events is not None:
+                raise ValueError("trace excludes spec_event and prof_events")
+            st = alspec_decode_traced(self.desc, q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                      seq_lens.data_ptr(), self.n_sink, self.window, float(lam),
+                                      out["out_spec"].data_ptr(), out["out_exact"].data_ptr(),
+                                      out["rel_l2"].data_ptr(), out["commit"].data_ptr(),
+                                      self.workspace.data_ptr(), self.workspace_bytes,
+                                      s.cuda_stream, trace.data_ptr())
+            _check(st, "alspec_decode_traced")
+            return out
         ev = spec_event.cuda_event if spec_event is not None else 0
         prof = None
         if prof_events is not None:

@@ -22,7 +22,7 @@ namespace alspec {
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr int kMaxSpecItems = 8;  // sink-set CTAs per (sequence, KV head): a portable cluster
+constexpr int kMaxSpecItems = kMaxSpecCtas;  // sink-set CTAs per (sequence, KV head)
 
 #ifndef ALSPEC_MID_SM_RESERVE
 #define ALSPEC_MID_SM_RESERVE 0
@@ -158,11 +158,11 @@ void make_plan(const alspec_desc& d, int S, int W, int sms, Plan* pl) {
     const int heads = d.batch * d.n_kv_heads;
     const int L = d.max_seq_len;
     const int tiles_max = ceil_div(std::min(S, L), TT) + ceil_div(std::min(W, L), TT);
-    // CTAs per head for the sink set (one thread-block cluster): about 7
-    // tiles each (one per consumer warp), at most 8 (the portable cluster
-    // size), and all heads together within half of the SMs.
+    // CTAs per head for the sink set (one thread-block cluster): about
+    // ALSPEC_SPEC_TILES tiles each, at most 8 (the portable cluster size),
+    // and all heads together within half of the SMs.
     const int room1 = std::max(1, sms / 2 / std::max(1, heads));
-    pl->n1 = std::max(1, std::min({kMaxSpecItems, room1, ceil_div(tiles_max, 7)}));
+    pl->n1 = std::max(1, std::min({kMaxSpecItems, room1, ceil_div(tiles_max, ALSPEC_SPEC_TILES)}));
     const int tiles_per_item = ceil_div(tiles_max, pl->n1);
     pl->c1 = tiles_per_item * TT;
     pl->n1 = ceil_div(tiles_max, tiles_per_item);  // no CTA without tiles at L_max
@@ -412,13 +412,20 @@ alspec_status alspec_query_chunks(const alspec_desc* desc, int n_sink, int windo
     return ALSPEC_OK;
 }
 
-alspec_status alspec_decode(const alspec_desc* desc, const void* q, const void* k_cache,
-                            const void* v_cache, const int32_t* seq_lens, int n_sink, int window,
-                            float lambda, float* out_spec, float* out_exact, float* rel_l2,
-                            uint8_t* commit, void* workspace, size_t workspace_bytes,
-                            void* stream, void* spec_event, void* const* prof_events) {
+}  // extern "C"
+
+namespace alspec {
+namespace {
+
+alspec_status decode_impl(const alspec_desc* desc, const void* q, const void* k_cache,
+                          const void* v_cache, const int32_t* seq_lens, int n_sink, int window,
+                          float lambda, float* out_spec, float* out_exact, float* rel_l2,
+                          uint8_t* commit, void* workspace, size_t workspace_bytes, void* stream,
+                          void* spec_event, void* const* prof_events,
+                          unsigned long long* trace_ns) {
     alspec_status st = check_desc(desc, n_sink, window);
     if (st != ALSPEC_OK) return st;
+    if (reinterpret_cast<uintptr_t>(trace_ns) & 7u) return ALSPEC_ERR_INVALID_ARG;
     if (!q || !k_cache || !v_cache || !seq_lens || !out_spec || !out_exact || !rel_l2 || !commit)
         return ALSPEC_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
@@ -467,6 +474,7 @@ alspec_status alspec_decode(const alspec_desc* desc, const void* q, const void* 
     p.dn = reinterpret_cast<float*>(ws + pl.off_dn);
     p.out_spec = out_spec;
     p.out_exact = out_exact;
+    p.trace = trace_ns;
     p.rel_l2 = rel_l2;
     p.commit = commit;
     p.timeout_ns = (unsigned long long)(desc->timeout_ms > 0 ? desc->timeout_ms : 2000) * 1000000ull;
@@ -514,6 +522,33 @@ alspec_status alspec_decode(const alspec_desc* desc, const void* q, const void* 
         return st;
     if (!prof(4, s)) return ALSPEC_ERR_CUDA;
     return ALSPEC_OK;
+}
+
+}  // namespace
+}  // namespace alspec
+
+extern "C" {
+
+alspec_status alspec_decode(const alspec_desc* desc, const void* q, const void* k_cache,
+                            const void* v_cache, const int32_t* seq_lens, int n_sink, int window,
+                            float lambda, float* out_spec, float* out_exact, float* rel_l2,
+                            uint8_t* commit, void* workspace, size_t workspace_bytes,
+                            void* stream, void* spec_event, void* const* prof_events) {
+    return decode_impl(desc, q, k_cache, v_cache, seq_lens, n_sink, window, lambda, out_spec,
+                       out_exact, rel_l2, commit, workspace, workspace_bytes, stream, spec_event,
+                       prof_events, nullptr);
+}
+
+alspec_status alspec_decode_traced(const alspec_desc* desc, const void* q, const void* k_cache,
+                                   const void* v_cache, const int32_t* seq_lens, int n_sink,
+                                   int window, float lambda, float* out_spec, float* out_exact,
+                                   float* rel_l2, uint8_t* commit, void* workspace,
+                                   size_t workspace_bytes, void* stream,
+                                   unsigned long long* trace_ns) {
+    if (!trace_ns) return ALSPEC_ERR_INVALID_ARG;
+    return decode_impl(desc, q, k_cache, v_cache, seq_lens, n_sink, window, lambda, out_spec,
+                       out_exact, rel_l2, commit, workspace, workspace_bytes, stream, nullptr,
+                       nullptr, trace_ns);
 }
 
 alspec_status alspec_get_device_error(void* workspace, size_t workspace_bytes, void* stream,

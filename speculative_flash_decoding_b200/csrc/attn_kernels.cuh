@@ -56,6 +56,17 @@
 namespace alspec {
 
 constexpr int kSmemLimit = 227 * 1024;
+// Sink-set CTAs per (sequence, KV head) at most: one portable cluster.
+constexpr int kMaxSpecCtas = 8;
+
+// Sink-set tokens per CTA, in tensor-core tiles of 32 (the planner's target),
+// and the consumer warps of the tensor-core sink-set kernel.
+#ifndef ALSPEC_SPEC_TILES
+#define ALSPEC_SPEC_TILES 7
+#endif
+#ifndef ALSPEC_SPEC_WARPS
+#define ALSPEC_SPEC_WARPS 7
+#endif
 
 // Stages per token slot of the tensor-core middle kernel: 3 stages of 16 KB
 // per consumer warp keep up to 192 KB in flight per SM -- well above the HBM
@@ -119,7 +130,18 @@ struct Params {
     float* rel_l2;
     uint8_t* commit;
     unsigned long long timeout_ns;
+    unsigned long long* trace;  // optional: [0] O_spec, [1] O_exact published (ns)
 };
+
+// Optional publication time stamps: after this thread's writes (and those
+// ordered before them), raise trace[which] to the global timer.  The last
+// writer of a result leaves its time there.
+__device__ __forceinline__ void trace_publish(const Params& p, int which) {
+    if (p.trace) {
+        __threadfence();
+        atomicMax(p.trace + which, (unsigned long long)global_ns());
+    }
+}
 
 __host__ __device__ __forceinline__ int cdiv(int a, int b) { return (a + b - 1) / b; }
 
@@ -267,7 +289,7 @@ struct Cfg {
     static constexpr bool kHeavy = !MMA && GW * kLanePairs >= 32;
     // Tensor-core engine: 4 consumer warps stream the middle; the sink-set
     // kernel (latency-bound, a few tiles per CTA) uses 7, one tile each.
-    static constexpr int NTW = MMA ? (SPEC ? 7 : 4) : (kHeavy ? 7 : 8) / NHW;
+    static constexpr int NTW = MMA ? (SPEC ? ALSPEC_SPEC_WARPS : 4) : (kHeavy ? 7 : 8) / NHW;
     static constexpr int NCW = NTW * NHW;
     static constexpr int kThreads = (NCW + 1) * 32;
     static constexpr int kTileBytes = TT * kRowBytes;  // K or V part of a stage
@@ -275,9 +297,12 @@ struct Cfg {
     static constexpr int kSlotFloats = GW * (D + 2);
     static constexpr int kDepositBytes = NCW * kSlotFloats * 4;
     static constexpr int kSpwMax = SPEC ? 3 : (MMA ? ALSPEC_MID_SPW : 4);
+    // Sink-set kernel: the cluster leader gathers one partial (m, l, o for
+    // the G heads) per CTA of the cluster.
+    static constexpr int kGatherFloats = G * (D + 2);
+    static constexpr int kGatherBytes = SPEC ? kMaxSpecCtas * kGatherFloats * 4 : 0;
     static constexpr int kSpwBudget =
-        (kSmemLimit - 1024 - kDepositBytes - 4096 - 512 - (SPEC ? G * (D + 2) * 4 : 0)) /
-        (NTW * kStageBytes);
+        (kSmemLimit - 1024 - kDepositBytes - 4096 - 512 - kGatherBytes) / (NTW * kStageBytes);
     static constexpr int SPW = kSpwBudget < 1 ? 1 : (kSpwBudget > kSpwMax ? kSpwMax : kSpwBudget);
     static constexpr int STAGES = NTW * SPW;
     // Dynamic shared memory layout (offsets from a 1024-byte aligned base;
@@ -287,16 +312,14 @@ struct Cfg {
     static constexpr int kOffDeposit = STAGES * kStageBytes;
     static constexpr int kOffMeta = align128(kOffDeposit + kDepositBytes);
     static constexpr int kOffBar = align128(kOffMeta + STAGES * 16);
-    static constexpr int kNumBars = 2 * STAGES + 2;
+    static constexpr int kNumBars = 2 * STAGES + 3;
     static constexpr int kOffMisc = align128(kOffBar + kNumBars * 8);
-    // Sink-set kernel: this CTA's merged partial, read by its cluster peers.
-    static constexpr int kOffCPart = align128(kOffMisc + 16);
-    static constexpr int kCPartBytes = SPEC ? G * (D + 2) * 4 : 0;
-    static constexpr int kSmemBytes = kOffCPart + kCPartBytes + 1024;  // + alignment slack
+    static constexpr int kOffGather = align128(kOffMisc + 16);
+    static constexpr int kSmemBytes = kOffGather + kGatherBytes + 1024;  // + alignment slack
     static_assert(kOffDeposit % 1024 == 0 && kStageBytes % 1024 == 0 && kTileBytes % 1024 == 0,
                   "TMA destinations with 128-byte swizzle need 1024-byte alignment");
     static_assert(kOffMeta % 16 == 0 && kOffBar % 8 == 0 && kOffMisc % 16 == 0 &&
-                      kOffCPart % 16 == 0 && (kSlotFloats * 4) % 8 == 0,
+                      kOffGather % 16 == 0 && (kSlotFloats * 4) % 8 == 0,
                   "shared-memory region alignment");
     static_assert(kRowBytes % 128 == 0, "row must be a multiple of 128 bytes");
     static_assert(G == 1 || G == 2 || G == 4 || G == 8, "group size");
@@ -712,52 +735,73 @@ struct EngineOf<C, T, D, G, true> {
     using type = MmaEngine<C, D, G>;
 };
 
-// Sink-set kernel, several CTAs per head (one cluster): each CTA holds its
-// merged partial (m, l, o for the G heads) in shared memory.  After a
-// cluster barrier CTA r merges outputs [r * G * D / n1, (r + 1) * G * D / n1)
-// from the n1 partials (rank order, all remote loads issued together) and
-// writes them; a second barrier keeps every CTA's shared memory alive until
-// its peers have read it.  Every thread of every CTA reaches both barriers
-// (all waits before them are bounded).
+// Sink-set kernel, several CTAs per head (one cluster): every CTA merges its
+// warps' states into one partial (m, l, o for the G heads) and stores it into
+// slot `rank` of the cluster leader's (rank 0) gather area, then arrives on
+// the leader's gather barrier with release semantics; the leader waits for
+// all n1 arrivals (bounded), merges the slots in rank order and publishes
+// O_spec.  No CTA reads another's shared memory, so the others exit at once.
+// Every thread of every CTA gets here (all waits before are bounded).
 template <int D, int G, class C>
-__device__ __forceinline__ void cluster_merge(const Params& p, float* cpart, int warp, int lane) {
-    constexpr int kMaxRanks = 8;
-    cluster_sync();
+__device__ __forceinline__ void cluster_gather(const Params& p, const float* deposit,
+                                               float* gather, uint64_t* gather_bar) {
+    constexpr int kF = C::kGatherFloats;
     const int n = p.n1;
-    const int rank = (int)cluster_ctarank();
+    const uint32_t rank = cluster_ctarank();
+    // The leader's gather barrier is initialised (every CTA arrived on the
+    // cluster barrier after its set-up).
+    cluster_wait();
+    const uint32_t slot = dsmem_addr(smem_addr(gather + rank * kF), 0);
+    for (int idx = threadIdx.x; idx < kF; idx += C::kThreads) {
+        const int hh = idx / (D + 2);
+        const int e = idx % (D + 2);
+        const float* base =
+            deposit + (hh / C::GW) * C::NTW * C::kSlotFloats + (hh % C::GW) * (D + 2);
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < C::NTW; ++w) M = fmaxf(M, base[w * C::kSlotFloats]);
+        float acc = 0.f;
+#pragma unroll
+        for (int w = 0; w < C::NTW; ++w) {
+            const float* ws = base + w * C::kSlotFloats;
+            acc = fmaf(merge_weight(ws[0], M), ws[e < 2 ? 1 : e], acc);
+        }
+        st_dsmem(slot + 4u * idx, e == 0 ? M : acc);  // (m, l, o[0..D)) of head hh
+    }
+    fence_acq_rel_cluster();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        mbar_arrive_cluster(dsmem_addr(smem_addr(gather_bar), 0));
+        fence_acq_rel_cluster();
+    }
+    if (rank != 0) return;
+
+    // Leader: every thread waits (bounded) for the n1 partials.
+    bool ok = true;
+    {
+        const uint64_t t0 = global_ns();
+        for (uint32_t it = 0; !mbar_try_wait_cluster(gather_bar, 0); ++it) {
+            if ((it & 31) == 31 && global_ns() - t0 > p.timeout_ns) {
+                ok = false;
+                break;
+            }
+        }
+    }
+    if (!ok) atomicOr(p.ctr + kCtrError, kErrTimeout);
     const int bh0 = (int)blockIdx.x / n;
     const int b = bh0 / p.Hkv;
     const int kvh = bh0 % p.Hkv;
-    const int per = (G * D + n - 1) / n;
-    const uint32_t local = smem_addr(cpart);
-    for (int idx = rank * per + (int)threadIdx.x; idx < min(G * D, (rank + 1) * per);
-         idx += C::kThreads) {
+    for (int idx = threadIdx.x; idx < G * D; idx += C::kThreads) {
         const int hh = idx / D;
         const int e = idx % D;
-        const uint32_t off = (uint32_t)(hh * (D + 2)) * 4u;
-        float m[kMaxRanks], l[kMaxRanks], o[kMaxRanks];
-#pragma unroll
-        for (int j = 0; j < kMaxRanks; ++j) {
-            if (j < n) {
-                const uint32_t a = dsmem_addr(local + off, (uint32_t)j);
-                m[j] = ld_dsmem(a);
-                l[j] = ld_dsmem(a + 4u);
-                o[j] = ld_dsmem(a + 8u + 4u * e);
-            } else {
-                m[j] = -INFINITY;
-                l[j] = 0.f;
-                o[j] = 0.f;
-            }
-        }
+        const float* g = gather + hh * (D + 2);
         float M = -INFINITY;
-#pragma unroll
-        for (int j = 0; j < kMaxRanks; ++j) M = fmaxf(M, m[j]);
+        for (int j = 0; j < n; ++j) M = fmaxf(M, g[j * kF]);
         float L = 0.f, O = 0.f;
-#pragma unroll
-        for (int j = 0; j < kMaxRanks; ++j) {
-            const float f = merge_weight(m[j], M);
-            L = fmaf(f, l[j], L);
-            O = fmaf(f, o[j], O);
+        for (int j = 0; j < n; ++j) {
+            const float f = merge_weight(g[j * kF], M);
+            L = fmaf(f, g[j * kF + 1], L);
+            O = fmaf(f, g[j * kF + 2 + e], O);
         }
         const size_t bh = (size_t)b * p.Hq + kvh * G + hh;
         if (e == 0) {
@@ -767,104 +811,119 @@ __device__ __forceinline__ void cluster_merge(const Params& p, float* cpart, int
         p.spec_o[bh * D + e] = O;
         p.out_spec[bh * D + e] = __fdiv_rn(O, L);
     }
-    cluster_sync();
-    (void)warp;
-    (void)lane;
+    if (p.trace) {
+        __syncthreads();
+        if (threadIdx.x == 0) trace_publish(p, 0);
+    }
 }
 
-// Producer lane: pull items, fill the stage ring, send end markers.
+// Fill stage s with tile t of item `item` (meta word, barrier arrival with
+// the expected bytes, the K and V copies).  Any lane may fill any stage.
+template <typename T, int D, int G, bool SPEC, bool MMA>
+__device__ __forceinline__ void fill_stage(const Params& p, unsigned char* smem, int4* meta,
+                                           uint64_t* full_bar, int s, int item, const Item& it,
+                                           int t, int ntiles) {
+    using C = Cfg<T, D, G, SPEC, MMA>;
+    constexpr int TT = C::TT;
+    const int head_row = (it.b * p.Hkv + it.kvh) * p.Lmax;
+    int start = 0, nvalid = 0;
+    if (t < it.ntiles) tile_rows<SPEC, TT>(it, t, start, nvalid);
+    meta[s] = make_int4(item, t, nvalid, t >= ntiles - C::NTW ? kLastTileFlag : 0);
+    if (nvalid == 0) {
+        mbar_arrive(full_bar + s);
+        return;
+    }
+    char* ks = reinterpret_cast<char*>(smem) + s * C::kStageBytes;
+    char* vs = ks + C::kTileBytes;
+    if (MMA) {
+        // Whole boxes; rows past the tensor end arrive as zeros.
+        mbar_arrive_expect_tx(full_bar + s, (uint32_t)C::kStageBytes);
+#pragma unroll
+        for (int h = 0; h < D / 64; ++h) {
+            tma_load_2d(ks + h * TT * 128, &p.tmap_k, 64 * h, head_row + start, full_bar + s);
+            tma_load_2d(vs + h * TT * 128, &p.tmap_v, 64 * h, head_row + start, full_bar + s);
+        }
+    } else {
+        const uint32_t bytes = (uint32_t)nvalid * C::kRowBytes;
+        mbar_arrive_expect_tx(full_bar + s, 2u * bytes);
+        const size_t off = ((size_t)head_row + start) * C::kRowBytes;
+        bulk_load(ks, reinterpret_cast<const char*>(p.k) + off, bytes, full_bar + s);
+        bulk_load(vs, reinterpret_cast<const char*>(p.v) + off, bytes, full_bar + s);
+    }
+}
+
+// The producer warp: fill the stage ring with the tiles of the items this CTA
+// pulls, then send end markers.  The first item (`item0`, taken before the
+// CTA's init barrier) fills the untouched stages one tile per lane, so the
+// first copies leave within a few hundred cycles; lane 0 alone continues
+// with the rest, waiting for each stage to be released.
 template <typename T, int D, int G, bool SPEC, bool MMA>
 __device__ __forceinline__ void produce(const Params& p, unsigned char* smem, int4* meta,
                                         uint64_t* full_bar, uint64_t* empty_bar,
-                                        volatile int* abort) {
+                                        volatile int* abort, int lane, int item0,
+                                        const Item& it0) {
     using C = Cfg<T, D, G, SPEC, MMA>;
-    constexpr int TT = C::TT;
     const int n_items = p.B * p.Hkv * (SPEC ? p.n1 : p.n2);
-    {
-        if (MMA) {
-            prefetch_tmap(&p.tmap_k);
-            prefetch_tmap(&p.tmap_v);
-        }
-        uint32_t gt = 0;
-        bool ok = true;
-        for (int iter = 0; ok; ++iter) {
-            int item;
-            if (SPEC) {
-                item = iter == 0 ? (int)blockIdx.x : n_items;
-            } else {
-                item = (int)atomicAdd(p.ctr + kCtrQueue, 1u);
+    auto rounded = [](const Item& it) { return (it.ntiles + C::NTW - 1) / C::NTW * C::NTW; };
+    const bool have0 = item0 < n_items && it0.ntiles > 0;
+    const int fresh = have0 ? min(rounded(it0), C::STAGES) : 0;
+    for (int t = lane; t < fresh; t += 32)
+        fill_stage<T, D, G, SPEC, MMA>(p, smem, meta, full_bar, t, item0, it0, t, rounded(it0));
+    if (lane != 0) return;
+
+    uint32_t gt = (uint32_t)fresh;
+    bool ok = true;
+    // Sequential part: wait for stage gt % STAGES, fill it.
+    auto run = [&](int item, const Item& it, int t_begin) {
+        const int ntiles = rounded(it);
+        for (int t = t_begin; t < ntiles; ++t, ++gt) {
+            const int s = gt % C::STAGES;
+            if (!wait_one(empty_bar + s, ((gt / C::STAGES) & 1) ^ 1, abort, p)) {
+                ok = false;
+                return;
             }
+            fill_stage<T, D, G, SPEC, MMA>(p, smem, meta, full_bar, s, item, it, t, ntiles);
+        }
+    };
+    if (have0) run(item0, it0, fresh);
+    if (!SPEC && item0 < n_items) {
+        while (ok) {
+            const int item = (int)atomicAdd(p.ctr + kCtrQueue, 1u);
             if (item >= n_items || *abort) break;
-            const Item it = decode_item<SPEC, TT>(p, item, true);
-            if (it.ntiles == 0) continue;
-            const int head_row = (it.b * p.Hkv + it.kvh) * p.Lmax;
-            const size_t head_byte = (size_t)head_row * C::kRowBytes;
-            const int ntiles = (it.ntiles + C::NTW - 1) / C::NTW * C::NTW;
-            for (int t = 0; t < ntiles; ++t, ++gt) {
-                const int s = gt % C::STAGES;
-                if (!wait_one(empty_bar + s, ((gt / C::STAGES) & 1) ^ 1, abort, p)) {
-                    ok = false;
-                    break;
-                }
-                int start = 0, nvalid = 0;
-                if (t < it.ntiles) tile_rows<SPEC, TT>(it, t, start, nvalid);
-                meta[s] = make_int4(item, t, nvalid, t >= ntiles - C::NTW ? kLastTileFlag : 0);
-                if (nvalid == 0) {
-                    mbar_arrive(full_bar + s);
-                    continue;
-                }
-                char* ks = reinterpret_cast<char*>(smem) + s * C::kStageBytes;
-                char* vs = ks + C::kTileBytes;
-                if (MMA) {
-                    // Whole boxes; rows past the tensor end arrive as zeros.
-                    mbar_arrive_expect_tx(full_bar + s, (uint32_t)C::kStageBytes);
-#pragma unroll
-                    for (int h = 0; h < D / 64; ++h) {
-                        tma_load_2d(ks + h * TT * 128, &p.tmap_k, 64 * h, head_row + start,
-                                    full_bar + s);
-                        tma_load_2d(vs + h * TT * 128, &p.tmap_v, 64 * h, head_row + start,
-                                    full_bar + s);
-                    }
-                } else {
-                    const uint32_t bytes = (uint32_t)nvalid * C::kRowBytes;
-                    mbar_arrive_expect_tx(full_bar + s, 2u * bytes);
-                    const size_t off = head_byte + (size_t)start * C::kRowBytes;
-                    bulk_load(ks, reinterpret_cast<const char*>(p.k) + off, bytes, full_bar + s);
-                    bulk_load(vs, reinterpret_cast<const char*>(p.v) + off, bytes, full_bar + s);
-                }
+            const Item it = decode_item<SPEC, C::TT>(p, item, true);
+            if (it.ntiles > 0) run(item, it, 0);
+        }
+    }
+    if (ok) {
+        // One end marker per token slot, so every consumer warp sees one.
+        for (int i = 0; i < C::NTW; ++i, ++gt) {
+            const int s = gt % C::STAGES;
+            if (!wait_one(empty_bar + s, ((gt / C::STAGES) & 1) ^ 1, abort, p)) {
+                ok = false;
+                break;
+            }
+            meta[s] = make_int4(-1, 0, 0, 0);
+            mbar_arrive(full_bar + s);
+        }
+    }
+    if (!ok) {
+        // Drain: wait (bounded) for the copies of the most recent fill of
+        // every stage, so that none lands after this CTA exits.
+        const uint32_t lo = gt > (uint32_t)C::STAGES ? gt - C::STAGES : 0;
+        for (uint32_t g2 = lo; g2 < gt; ++g2) {
+            const int s = g2 % C::STAGES;
+            const uint64_t t0 = global_ns();
+            while (!mbar_try_wait(full_bar + s, (g2 / C::STAGES) & 1)) {
+                if (global_ns() - t0 > p.timeout_ns) break;
             }
         }
-        if (ok) {
-            // One end marker per token slot, so every consumer warp sees one.
-            for (int i = 0; i < C::NTW; ++i, ++gt) {
-                const int s = gt % C::STAGES;
-                if (!wait_one(empty_bar + s, ((gt / C::STAGES) & 1) ^ 1, abort, p)) {
-                    ok = false;
-                    break;
-                }
-                meta[s] = make_int4(-1, 0, 0, 0);
-                mbar_arrive(full_bar + s);
-            }
-        }
-        if (!ok) {
-            // Drain: wait (bounded) for the copies of the most recent fill of
-            // every stage, so that none lands after this CTA exits.
-            const uint32_t lo = gt > (uint32_t)C::STAGES ? gt - C::STAGES : 0;
-            for (uint32_t g2 = lo; g2 < gt; ++g2) {
-                const int s = g2 % C::STAGES;
-                const uint64_t t0 = global_ns();
-                while (!mbar_try_wait(full_bar + s, (g2 / C::STAGES) & 1)) {
-                    if (global_ns() - t0 > p.timeout_ns) break;
-                }
-            }
-        }
-        if (!SPEC) {
-            // The CTA that stops last resets the queue for the next call.
-            const unsigned t = atomicAdd(p.ctr + kCtrDone, 1u);
-            if (t == gridDim.x - 1) {
-                atomicExch(p.ctr + kCtrQueue, 0u);
-                atomicExch(p.ctr + kCtrDone, 0u);
-            }
+    }
+    if (!SPEC) {
+        // The CTA that stops last resets the queue for the next call.
+        const unsigned t = atomicAdd(p.ctr + kCtrDone, 1u);
+        if (t == gridDim.x - 1) {
+            atomicExch(p.ctr + kCtrQueue, 0u);
+            atomicExch(p.ctr + kCtrDone, 0u);
         }
     }
 }
@@ -896,6 +955,15 @@ __device__ __forceinline__ void consume(const Params& p, unsigned char* smem, fl
     };
     uint32_t gt = tw;
     int b = 0, kvh = 0, chunk = 0;
+    if (SPEC && p.n1 > 1) {
+        // Empty state (m = -inf, l = 0, o = 0) in this warp's deposit slot:
+        // a CTA whose slice of a short sink set has no tiles contributes
+        // nothing to the cluster merge.
+        float* slot = deposit + (hw * C::NTW + tw) * C::kSlotFloats;
+        for (int h = 0; h < C::GW; ++h)
+            for (int e = lane; e < D + 2; e += 32) slot[h * (D + 2) + e] = e == 0 ? -INFINITY : 0.f;
+        __syncwarp();
+    }
     if (SPEC) {
         // The item is known up front: fetch q while the first tiles load.
         const int bh = (int)blockIdx.x / p.n1;
@@ -995,9 +1063,10 @@ __global__ void __launch_bounds__(Cfg<T, D, G, SPEC, MMA>::kThreads, 1)
     uint64_t* empty_bar = full_bar + C::STAGES;
     uint64_t* dep_bar = empty_bar + C::STAGES;  // consumer warps: phase sync
     uint64_t* free_bar = dep_bar + 1;           // consumer warps: writes done
+    uint64_t* gather_bar = free_bar + 1;        // sink-set cluster leader: partials in
     Shared* sh = reinterpret_cast<Shared*>(smem + C::kOffMisc);
     volatile int* abort = &sh->abort;
-    float* cpart = reinterpret_cast<float*>(smem + C::kOffCPart);
+    float* gather = reinterpret_cast<float*>(smem + C::kOffGather);
     // Sink-set kernel with several CTAs per head: those CTAs are one cluster.
     const bool clustered = SPEC && p.n1 > 1;
 
@@ -1011,51 +1080,54 @@ __global__ void __launch_bounds__(Cfg<T, D, G, SPEC, MMA>::kThreads, 1)
         }
         mbar_init(dep_bar, C::NCW);
         mbar_init(free_bar, C::NCW);
+        mbar_init(gather_bar, clustered ? p.n1 : 1);
         sh->abort = 0;
         fence_barrier_init();
     }
-    if (clustered) {
-        // Empty states (m = -inf, l = 0, o = 0) in every warp's deposit slot:
-        // a CTA whose slice of a short sink set has no tiles (or a warp with
-        // only padding tiles) contributes nothing to the merge.
-        for (int i = threadIdx.x; i < C::NCW * C::kSlotFloats; i += C::kThreads)
-            deposit[i] = (i % C::kSlotFloats) % (D + 2) == 0 ? -INFINITY : 0.f;
+    // The producer warp fetches the tensor maps and takes its first item now,
+    // so that those loads, the queue ticket and the sequence-length load
+    // overlap the barrier set-up.
+    const int n_items = p.B * p.Hkv * (SPEC ? p.n1 : p.n2);
+    int item0 = n_items;
+    Item it0{};
+    if (warp == C::NCW) {
+        if (MMA && lane == 0) {
+            prefetch_tmap(&p.tmap_k);
+            prefetch_tmap(&p.tmap_v);
+        }
+        if (SPEC) {
+            item0 = (int)blockIdx.x;
+        } else {
+            unsigned v = 0;
+            if (lane == 0) v = atomicAdd(p.ctr + kCtrQueue, 1u);
+            item0 = (int)__shfl_sync(0xffffffffu, v, 0);
+        }
+        if (item0 < n_items) it0 = decode_item<SPEC, C::TT>(p, item0, lane == 0);
     }
     // The merge kernel that follows this (middle) kernel may be resident
     // already: it only prepares until this grid has completed.
     if (!SPEC) pdl_launch_dependents();
     __syncthreads();
+    if (clustered) cluster_arrive_relaxed();  // this CTA's barriers are set up
 
     if (warp == C::NCW) {
         // ---------------------------------------------------- producer
-        if (lane == 0) produce<T, D, G, SPEC, MMA>(p, smem, meta, full_bar, empty_bar, abort);
+        produce<T, D, G, SPEC, MMA>(p, smem, meta, full_bar, empty_bar, abort, lane, item0, it0);
         if (!clustered) return;
         __syncwarp();  // the warp waits for its producer lane, then joins the cluster merge
     } else {
         consume<T, D, G, SPEC, MMA>(p, smem, deposit, meta, full_bar, empty_bar, dep_bar,
                                     free_bar, abort);
     }
+    if (SPEC && !clustered && warp < C::NCW && p.trace) {
+        // One CTA per head: its consumer warps wrote O_spec.
+        __syncwarp();
+        if (lane == 0) trace_publish(p, 0);
+    }
     if (clustered) {
-        // Every thread of the CTA is here (no early exits in this mode):
-        // merge the warps' states into this CTA's partial, then the cluster.
+        // Every thread of the CTA is here (no early exits in this mode).
         __syncthreads();
-        for (int idx = threadIdx.x; idx < G * (D + 2); idx += C::kThreads) {
-            const int hh = idx / (D + 2);
-            const int e = idx % (D + 2);
-            const float* base =
-                deposit + (hh / C::GW) * C::NTW * C::kSlotFloats + (hh % C::GW) * (D + 2);
-            float M = -INFINITY;
-#pragma unroll
-            for (int w = 0; w < C::NTW; ++w) M = fmaxf(M, base[w * C::kSlotFloats]);
-            float acc = 0.f;
-#pragma unroll
-            for (int w = 0; w < C::NTW; ++w) {
-                const float* ws = base + w * C::kSlotFloats;
-                acc = fmaf(merge_weight(ws[0], M), ws[e < 2 ? 1 : e], acc);
-            }
-            cpart[idx] = e == 0 ? M : acc;  // (m, l, o[0..D)) of head hh
-        }
-        cluster_merge<D, G, C>(p, cpart, warp, lane);
+        cluster_gather<D, G, C>(p, deposit, gather, gather_bar);
     }
 }
 
@@ -1216,6 +1288,7 @@ __global__ void __launch_bounds__(D * kMergeParts) merge_kernel(const __grid_con
                 p.commit[b] = r <= (double)p.lambda ? 1 : 0;
             }
         }
+        if (lane == 0) trace_publish(p, 1);
     }
 }
 

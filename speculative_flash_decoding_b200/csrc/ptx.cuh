@@ -119,7 +119,7 @@ __device__ __forceinline__ void pdl_wait_prerequisite() {
 
 // Thread-block clusters: rank of this CTA, a full cluster barrier (every
 // thread of every CTA of the cluster; release/acquire orders shared-memory
-// writes before remote reads), and loads from another CTA's shared memory.
+// writes before remote reads), and accesses to another CTA's shared memory.
 __device__ __forceinline__ uint32_t cluster_ctarank() {
     uint32_t r;
     asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
@@ -143,6 +143,47 @@ __device__ __forceinline__ float ld_dsmem(uint32_t addr) {
     float v;
     asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
     return v;
+}
+
+// Split form of the cluster barrier: a relaxed arrive (orders nothing) and
+// a wait with acquire semantics.  Every thread of every CTA of the cluster
+// arrives once and waits once.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void cluster_wait() {
+    asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+}
+
+// Store to another CTA's shared memory (an address from dsmem_addr).
+__device__ __forceinline__ void st_dsmem(uint32_t addr, float v) {
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+
+__device__ __forceinline__ void fence_acq_rel_cluster() {
+    asm volatile("fence.acq_rel.cluster;" ::: "memory");
+}
+
+// Arrive, with release semantics at cluster scope, on an mbarrier of another
+// CTA of the cluster (an address from dsmem_addr).
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(addr)
+                 : "memory");
+}
+
+// One probe of a local mbarrier with acquire semantics at cluster scope: on
+// success the writes released by the arrivals of other CTAs are visible.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
 }
 
 __device__ __forceinline__ uint64_t global_ns() {

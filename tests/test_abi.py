@@ -136,3 +136,14 @@ def test_null_handles():
     assert sfd.alspec_workspace_init(0, 16, 0) == ab.ALSPEC_ERR_INVALID_ARG
     st, err = sfd.alspec_get_device_error(0, 1024, 0)
     assert st == ab.ALSPEC_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("trace,code", [(0, ab.ALSPEC_ERR_INVALID_ARG),
+                                        ((1 << 20) + 4, ab.ALSPEC_ERR_INVALID_ARG)])
+def test_traced_decode_rejects_bad_trace_buffer(trace, code):
+    """A missing or misaligned time-stamp buffer is refused before any launch."""
+    d = desc(max_seq_len=4096)
+    fake = 1 << 20
+    st = sfd.alspec_decode_traced(d, fake, fake, fake, fake, 4, 64, 0.1, fake, fake, fake, fake,
+                                  fake, sfd.alspec_workspace_size(d, 4, 64), 0, trace)
+    assert st == code

@@ -88,6 +88,30 @@ def test_edge_lengths(cuda_device, dtype, d, g, engine):
                 assert out["rel_l2"][b].item() == 0.0 and out["commit"][b].item() == 1
 
 
+@pytest.mark.parametrize("d,engine", [(128, "tensor_cores"), (64, "tensor_cores"),
+                                      (128, "cuda_cores")])
+def test_short_sequences_in_a_clustered_sink_set(cuda_device, d, engine):
+    """A 4096-row cache splits each head's sink set over several CTAs (one
+    cluster); short sequences leave some of those CTAs without tiles."""
+    import speculative_flash_decoding_b200 as sfd
+    lens = [1, 3, 40, 1000, 1028, 1029, 2100, 4096]
+    wl = workloads.Workload("short-in-cluster", B=len(lens), Hq=8, Hkv=2, d=d, L=4096, S=4,
+                            W=1024, lam=0.3, dtype="bf16", seed=4242 + d)
+    desc = sfd.make_desc(wl.B, wl.Hq, wl.Hkv, wl.d, wl.L, wl.dtype, engine=engine)
+    st, plan = sfd.alspec_query_plan(desc, wl.S, wl.W)
+    assert st == 0 and plan["n1"] > 1
+    data = workloads.make_layer(wl, device=cuda_device)
+    data["lens"] = lens
+    data["seq_lens"] = torch.tensor(lens, dtype=torch.int32, device=cuda_device)
+    dec, out = gpu_decode(wl, data, cuda_device, engine=engine)
+    assert_parity(out, oracle_decode(wl, data), wl.lam, what=f"short in cluster d{d} {engine}")
+    for b, L in enumerate(lens):
+        if L <= wl.S + wl.W:
+            assert torch.equal(out["out_spec"][b], out["out_exact"][b])
+            assert out["rel_l2"][b].item() == 0.0 and out["commit"][b].item() == 1
+    assert dec.device_error() == (0, 0)
+
+
 def test_deterministic_and_reusable_workspace(cuda_device):
     wl = _small(1)
     data = workloads.make_layer(wl, device=cuda_device)
@@ -136,6 +160,43 @@ def test_spec_event_marks_o_spec_complete(cuda_device):
     assert torch.equal(spec_at_event, out["out_spec"].cpu())
     ref = oracle_decode(wl, data)
     assert_parity({k: v.cpu() for k, v in out.items()}, ref, wl.lam, what="spec event")
+
+
+def test_traced_decode_stamps_and_outputs(cuda_device):
+    """The traced entry point computes the same bits and leaves two time
+    stamps: O_spec published before O_exact, in eager calls and in a graph."""
+    import speculative_flash_decoding_b200 as sfd
+    wl = _small(2)
+    layers = [workloads.make_layer(wl, layer=i, device=cuda_device) for i in range(2)]
+    dec = sfd.Decoder(wl.B, wl.Hq, wl.Hkv, wl.d, wl.L, wl.dtype, wl.S, wl.W, device=cuda_device)
+    trace = torch.zeros(2, 2, dtype=torch.int64, device=cuda_device)
+    for i, data in enumerate(layers):
+        plain = {k: v.clone() for k, v in dec.decode(data["q"], data["k"], data["v"],
+                                                      data["seq_lens"], wl.lam).items()}
+        traced = dec.decode(data["q"], data["k"], data["v"], data["seq_lens"], wl.lam,
+                            trace=trace[i])
+        torch.cuda.synchronize()
+        for k in plain:
+            assert torch.equal(plain[k], traced[k]), k
+    t = trace.cpu().numpy()
+    assert (t > 0).all() and (t[:, 0] < t[:, 1]).all() and t[0, 1] < t[1, 0], t
+    stream = torch.cuda.Stream(cuda_device)
+    outs = [dec.alloc_outputs() for _ in layers]
+    with torch.cuda.stream(stream):
+        assert sfd.alspec_graph_begin(stream.cuda_stream) == 0
+        for i, (data, o) in enumerate(zip(layers, outs)):
+            dec.decode(data["q"], data["k"], data["v"], data["seq_lens"], wl.lam, out=o,
+                       stream=stream, trace=trace[i])
+        st, graph = sfd.alspec_graph_end(stream.cuda_stream)
+        assert st == 0 and graph
+        trace.zero_()
+        assert sfd.alspec_graph_launch(graph, stream.cuda_stream) == 0
+        stream.synchronize()
+        assert sfd.alspec_graph_destroy(graph) == 0
+    t = trace.cpu().numpy()
+    assert (t > 0).all() and (t[:, 0] < t[:, 1]).all() and t[0, 1] < t[1, 0], t
+    # O_spec of layer 1 comes well before the end of its exact path.
+    assert (t[1, 0] - t[0, 1]) < (t[1, 1] - t[0, 1])
 
 
 def test_graph_replay_matches_direct_calls(cuda_device):
