@@ -62,10 +62,10 @@ constexpr int kMaxSpecCtas = 8;
 // Sink-set tokens per CTA, in tensor-core tiles of 32 (the planner's target),
 // and the consumer warps of the tensor-core sink-set kernel.
 #ifndef ALSPEC_SPEC_TILES
-#define ALSPEC_SPEC_TILES 7
+#define ALSPEC_SPEC_TILES 5
 #endif
 #ifndef ALSPEC_SPEC_WARPS
-#define ALSPEC_SPEC_WARPS 7
+#define ALSPEC_SPEC_WARPS 5
 #endif
 
 // Stages per token slot of the tensor-core middle kernel: 3 stages of 16 KB
@@ -288,7 +288,7 @@ struct Cfg {
     static constexpr int kLanePairs = (kRowBytes / 128) * Elem<T>::kPairs;
     static constexpr bool kHeavy = !MMA && GW * kLanePairs >= 32;
     // Tensor-core engine: 4 consumer warps stream the middle; the sink-set
-    // kernel (latency-bound, a few tiles per CTA) uses 7, one tile each.
+    // kernel (latency-bound, a few tiles per CTA) uses one warp per tile.
     static constexpr int NTW = MMA ? (SPEC ? ALSPEC_SPEC_WARPS : 4) : (kHeavy ? 7 : 8) / NHW;
     static constexpr int NCW = NTW * NHW;
     static constexpr int kThreads = (NCW + 1) * 32;
@@ -297,12 +297,14 @@ struct Cfg {
     static constexpr int kSlotFloats = GW * (D + 2);
     static constexpr int kDepositBytes = NCW * kSlotFloats * 4;
     static constexpr int kSpwMax = SPEC ? 3 : (MMA ? ALSPEC_MID_SPW : 4);
-    // Sink-set kernel: the cluster leader gathers one partial (m, l, o for
-    // the G heads) per CTA of the cluster.
+    // Sink-set kernel: every CTA of a cluster gathers one partial (m, l, o
+    // for the G heads) per CTA of the cluster, in slots padded to 16 bytes.
     static constexpr int kGatherFloats = G * (D + 2);
-    static constexpr int kGatherBytes = SPEC ? kMaxSpecCtas * kGatherFloats * 4 : 0;
+    static constexpr int kGatherStride = (kGatherFloats + 3) / 4 * 4;
+    static constexpr int kGatherBytes = SPEC ? kMaxSpecCtas * kGatherStride * 4 : 0;
+
     static constexpr int kSpwBudget =
-        (kSmemLimit - 1024 - kDepositBytes - 4096 - 512 - kGatherBytes) / (NTW * kStageBytes);
+        (kSmemLimit - 1024 - kDepositBytes - 4096 - 768 - kGatherBytes) / (NTW * kStageBytes);
     static constexpr int SPW = kSpwBudget < 1 ? 1 : (kSpwBudget > kSpwMax ? kSpwMax : kSpwBudget);
     static constexpr int STAGES = NTW * SPW;
     // Dynamic shared memory layout (offsets from a 1024-byte aligned base;
@@ -736,47 +738,58 @@ struct EngineOf<C, T, D, G, true> {
 };
 
 // Sink-set kernel, several CTAs per head (one cluster): every CTA merges its
-// warps' states into one partial (m, l, o for the G heads) and stores it into
-// slot `rank` of the cluster leader's (rank 0) gather area, then arrives on
-// the leader's gather barrier with release semantics; the leader waits for
-// all n1 arrivals (bounded), merges the slots in rank order and publishes
-// O_spec.  No CTA reads another's shared memory, so the others exit at once.
-// Every thread of every CTA gets here (all waits before are bounded).
+// warps' states into one partial (m, l, o for the G heads) and sends it with
+// asynchronous 16-byte stores into slot `rank` of the gather area of every
+// CTA of the cluster; the bytes complete on each CTA's gather barrier, which
+// expects all n1 slots.  Each CTA then waits (bounded), merges the slots in
+// rank order for its slice [rank * per, (rank + 1) * per) of the G * D
+// outputs and publishes that slice of O_spec.  A last cluster barrier, which
+// each CTA reaches only after all bytes sent to it have landed, keeps every
+// CTA resident until its stores are done.  Every thread of every CTA gets
+// here (all waits before are bounded) and has waited once on the cluster
+// barrier since the set-up, so every gather barrier is initialised.
 template <int D, int G, class C>
 __device__ __forceinline__ void cluster_gather(const Params& p, const float* deposit,
                                                float* gather, uint64_t* gather_bar) {
     constexpr int kF = C::kGatherFloats;
+    constexpr int kStride = C::kGatherStride;
+    constexpr int NTW = C::NTW;
     const int n = p.n1;
     const uint32_t rank = cluster_ctarank();
-    // The leader's gather barrier is initialised (every CTA arrived on the
-    // cluster barrier after its set-up).
-    cluster_wait();
-    const uint32_t slot = dsmem_addr(smem_addr(gather + rank * kF), 0);
-    for (int idx = threadIdx.x; idx < kF; idx += C::kThreads) {
-        const int hh = idx / (D + 2);
-        const int e = idx % (D + 2);
-        const float* base =
-            deposit + (hh / C::GW) * C::NTW * C::kSlotFloats + (hh % C::GW) * (D + 2);
-        float M = -INFINITY;
+    const uint32_t dst = smem_addr(gather + rank * kStride);
+    const uint32_t bar = smem_addr(gather_bar);
+    for (int v = threadIdx.x; v < kStride / 4; v += C::kThreads) {
+        float x[4];
 #pragma unroll
-        for (int w = 0; w < C::NTW; ++w) M = fmaxf(M, base[w * C::kSlotFloats]);
-        float acc = 0.f;
+        for (int k = 0; k < 4; ++k) {
+            const int idx = 4 * v + k;
+            float val = 0.f;
+            if (idx < kF) {
+                const int hh = idx / (D + 2);
+                const int e = idx % (D + 2);
+                const float* base =
+                    deposit + (hh / C::GW) * NTW * C::kSlotFloats + (hh % C::GW) * (D + 2);
+                float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < C::NTW; ++w) {
-            const float* ws = base + w * C::kSlotFloats;
-            acc = fmaf(merge_weight(ws[0], M), ws[e < 2 ? 1 : e], acc);
+                for (int w = 0; w < NTW; ++w) M = fmaxf(M, base[w * C::kSlotFloats]);
+                if (e == 0) {
+                    val = M;
+                } else {
+#pragma unroll
+                    for (int w = 0; w < NTW; ++w) {
+                        const float* ws = base + w * C::kSlotFloats;
+                        val = fmaf(merge_weight(ws[0], M), ws[e < 2 ? 1 : e], val);
+                    }
+                }
+            }
+            x[k] = val;  // (m, l, o[0..D)) of head hh
         }
-        st_dsmem(slot + 4u * idx, e == 0 ? M : acc);  // (m, l, o[0..D)) of head hh
+        for (int j = 0; j < n; ++j)
+            st_async_v4(dsmem_addr(dst, (uint32_t)j) + 16u * (uint32_t)v, x,
+                        dsmem_addr(bar, (uint32_t)j));
     }
-    fence_acq_rel_cluster();
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        mbar_arrive_cluster(dsmem_addr(smem_addr(gather_bar), 0));
-        fence_acq_rel_cluster();
-    }
-    if (rank != 0) return;
 
-    // Leader: every thread waits (bounded) for the n1 partials.
+    // Wait (bounded) for the n1 slots sent to this CTA.
     bool ok = true;
     {
         const uint64_t t0 = global_ns();
@@ -791,17 +804,27 @@ __device__ __forceinline__ void cluster_gather(const Params& p, const float* dep
     const int bh0 = (int)blockIdx.x / n;
     const int b = bh0 / p.Hkv;
     const int kvh = bh0 % p.Hkv;
-    for (int idx = threadIdx.x; idx < G * D; idx += C::kThreads) {
+    const int per = (G * D + n - 1) / n;
+    const int hi = min(G * D, ((int)rank + 1) * per);
+    for (int idx = (int)rank * per + (int)threadIdx.x; idx < hi; idx += C::kThreads) {
         const int hh = idx / D;
         const int e = idx % D;
         const float* g = gather + hh * (D + 2);
+        float m[kMaxSpecCtas];
         float M = -INFINITY;
-        for (int j = 0; j < n; ++j) M = fmaxf(M, g[j * kF]);
+#pragma unroll
+        for (int j = 0; j < kMaxSpecCtas; ++j) {
+            m[j] = j < n ? g[j * kStride] : -INFINITY;
+            M = fmaxf(M, m[j]);
+        }
         float L = 0.f, O = 0.f;
-        for (int j = 0; j < n; ++j) {
-            const float f = merge_weight(g[j * kF], M);
-            L = fmaf(f, g[j * kF + 1], L);
-            O = fmaf(f, g[j * kF + 2 + e], O);
+#pragma unroll
+        for (int j = 0; j < kMaxSpecCtas; ++j) {
+            if (j < n) {
+                const float f = merge_weight(m[j], M);
+                L = fmaf(f, g[j * kStride + 1], L);
+                O = fmaf(f, g[j * kStride + 2 + e], O);
+            }
         }
         const size_t bh = (size_t)b * p.Hq + kvh * G + hh;
         if (e == 0) {
@@ -811,10 +834,11 @@ __device__ __forceinline__ void cluster_gather(const Params& p, const float* dep
         p.spec_o[bh * D + e] = O;
         p.out_spec[bh * D + e] = __fdiv_rn(O, L);
     }
-    if (p.trace) {
-        __syncthreads();
-        if (threadIdx.x == 0) trace_publish(p, 0);
-    }
+    __syncthreads();
+    if (threadIdx.x == 0) trace_publish(p, 0);
+    __syncwarp();
+    cluster_arrive_relaxed();
+    cluster_wait();
 }
 
 // Fill stage s with tile t of item `item` (meta word, barrier arrival with
@@ -963,6 +987,9 @@ __device__ __forceinline__ void consume(const Params& p, unsigned char* smem, fl
         for (int h = 0; h < C::GW; ++h)
             for (int e = lane; e < D + 2; e += 32) slot[h * (D + 2) + e] = e == 0 ? -INFINITY : 0.f;
         __syncwarp();
+        // Every CTA of the cluster has set up its barriers once this passes
+        // (long before the first tile lands).
+        cluster_wait_any();
     }
     if (SPEC) {
         // The item is known up front: fetch q while the first tiles load.
@@ -1080,7 +1107,9 @@ __global__ void __launch_bounds__(Cfg<T, D, G, SPEC, MMA>::kThreads, 1)
         }
         mbar_init(dep_bar, C::NCW);
         mbar_init(free_bar, C::NCW);
-        mbar_init(gather_bar, clustered ? p.n1 : 1);
+        mbar_init(gather_bar, 1);
+        // Every CTA of a cluster receives every CTA's slot as transaction bytes.
+        if (clustered) mbar_arrive_expect_tx(gather_bar, (uint32_t)(p.n1 * C::kGatherStride * 4));
         sh->abort = 0;
         fence_barrier_init();
     }
@@ -1114,6 +1143,7 @@ __global__ void __launch_bounds__(Cfg<T, D, G, SPEC, MMA>::kThreads, 1)
         // ---------------------------------------------------- producer
         produce<T, D, G, SPEC, MMA>(p, smem, meta, full_bar, empty_bar, abort, lane, item0, it0);
         if (!clustered) return;
+        cluster_wait_any();  // the cluster's barriers are set up
         __syncwarp();  // the warp waits for its producer lane, then joins the cluster merge
     } else {
         consume<T, D, G, SPEC, MMA>(p, smem, deposit, meta, full_bar, empty_bar, dep_bar,

@@ -156,6 +156,23 @@ __device__ __forceinline__ void cluster_wait() {
     asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
 }
 
+// Wait on the cluster barrier; threads of a warp may call it at different
+// points (no .aligned).
+__device__ __forceinline__ void cluster_wait_any() {
+    asm volatile("barrier.cluster.wait;" ::: "memory");
+}
+
+// Asynchronous 16-byte store into another CTA's shared memory (addresses
+// from dsmem_addr, 16-byte aligned); its bytes count as completed
+// transaction bytes on the mbarrier `bar` of that CTA.
+__device__ __forceinline__ void st_async_v4(uint32_t addr, const float (&x)[4], uint32_t bar) {
+    asm volatile(
+        "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, "
+        "[%5];" ::"r"(addr),
+        "f"(x[0]), "f"(x[1]), "f"(x[2]), "f"(x[3]), "r"(bar)
+        : "memory");
+}
+
 // Store to another CTA's shared memory (an address from dsmem_addr).
 __device__ __forceinline__ void st_dsmem(uint32_t addr, float v) {
     asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
