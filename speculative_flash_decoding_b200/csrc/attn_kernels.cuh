@@ -1164,7 +1164,7 @@ __global__ void __launch_bounds__(Cfg<T, D, G, SPEC, MMA>::kThreads, 1)
 // ------------------------------------------------------- merge + verify
 
 constexpr int kMergeParts = 4;  // thread groups sharing a head's chunks
-constexpr int kMergeBatch = 8;  // chunk loads each thread keeps in flight
+constexpr int kMergeBatch = 32;  // chunk loads each thread keeps in flight
 
 // One CTA per (query head, sequence), D x 4 threads: thread (part, e) owns
 // output element e and the chunks list[part], list[part + 4], ...  O_exact
@@ -1187,7 +1187,7 @@ __global__ void __launch_bounds__(D * kMergeParts) merge_kernel(const __grid_con
     const int lane = tid & 31;
     const size_t bh = (size_t)b * p.Hq + h;
     __shared__ int list[kMaxChunks];      // non-empty chunks, in order
-    __shared__ float2 cml[kMaxChunks];    // their (m, l), then (weight, weighted l)
+    __shared__ float wts[kMaxChunks];     // their merge weights
     __shared__ float red[2][NW];
     __shared__ float accs[kMergeParts][D];
     __shared__ int nlist;
@@ -1208,18 +1208,26 @@ __global__ void __launch_bounds__(D * kMergeParts) merge_kernel(const __grid_con
         }
         nlist = count;
     }
+    __syncthreads();
+    const int n = nlist;
     // Everything above only read inputs; the partials are written by the
     // kernels this one follows, which may still be running.
     pdl_wait_prerequisite();
+    // One round of independent loads: the sink-set partial, this thread's
+    // chunk (m, l) (one chunk per thread: n <= kMaxChunks <= NT) and this
+    // thread's column of its first kMergeBatch chunks (every kMergeParts-th).
+    static_assert(kMaxChunks <= NT, "one chunk (m, l) per thread");
     const float2 sml = __ldcg(reinterpret_cast<const float2*>(p.spec_ml) + bh);
     const float os = __ldcg(p.spec_o + bh * D + e);
-    __syncthreads();
-    const int n = nlist;
-    float M = sml.x;
-    for (int i = tid; i < n; i += NT) {
-        cml[i] = __ldcg(&mml[list[i]]);
-        M = fmaxf(M, cml[i].x);
+    const float2 cm = tid < n ? __ldcg(&mml[list[tid]]) : make_float2(-INFINITY, 0.f);
+    const float* mo = p.mid_o + bh * p.n2 * D + e;
+    float v[kMergeBatch];
+#pragma unroll
+    for (int u = 0; u < kMergeBatch; ++u) {
+        const int i = part + u * kMergeParts;
+        v[u] = i < n ? __ldcg(mo + list[i] * D) : 0.f;
     }
+    float M = fmaxf(sml.x, cm.x);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     if (lane == 0) red[0][warp] = M;
@@ -1228,30 +1236,33 @@ __global__ void __launch_bounds__(D * kMergeParts) merge_kernel(const __grid_con
     for (int w = 0; w < NW; ++w) M = fmaxf(M, red[0][w]);
     // Weights, and the normaliser: sum of weight * l in a fixed order.
     float lsum = 0.f;
-    for (int i = tid; i < n; i += NT) {
-        const float w = merge_weight(cml[i].x, M);
-        cml[i].x = w;
-        lsum = fmaf(w, cml[i].y, lsum);
+    if (tid < n) {
+        const float w = merge_weight(cm.x, M);
+        wts[tid] = w;
+        lsum = w * cm.y;
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
     if (lane == 0) red[1][warp] = lsum;
     __syncthreads();
 
-    // Weighted value rows: batches of independent loads.
-    const float* mo = p.mid_o + bh * p.n2 * D + e;
+    // Weighted value rows, in chunk order per thread.
     float acc = 0.f;
-    for (int i0 = part; i0 < n; i0 += kMergeParts * kMergeBatch) {
-        float v[kMergeBatch];
+#pragma unroll
+    for (int u = 0; u < kMergeBatch; ++u) {
+        const int i = part + u * kMergeParts;
+        if (i < n) acc = fmaf(wts[i], v[u], acc);
+    }
+    for (int i0 = part + kMergeParts * kMergeBatch; i0 < n; i0 += kMergeParts * kMergeBatch) {
 #pragma unroll
         for (int u = 0; u < kMergeBatch; ++u) {
             const int i = i0 + u * kMergeParts;
-            v[u] = i < n ? __ldcg(mo + (size_t)list[i] * D) : 0.f;
+            v[u] = i < n ? __ldcg(mo + list[i] * D) : 0.f;
         }
 #pragma unroll
         for (int u = 0; u < kMergeBatch; ++u) {
             const int i = i0 + u * kMergeParts;
-            if (i < n) acc = fmaf(cml[i].x, v[u], acc);
+            if (i < n) acc = fmaf(wts[i], v[u], acc);
         }
     }
     accs[part][e] = acc;
@@ -1285,14 +1296,12 @@ __global__ void __launch_bounds__(D * kMergeParts) merge_kernel(const __grid_con
         }
         if (lane == 0) {
             *reinterpret_cast<float2*>(p.dn + bh * 2) = make_float2(dd, nn);
-            __threadfence();
+            // Release: this head's (dd, nn) before the ticket; acquire: the
+            // last head's CTA sees every head's.
             unsigned* word = p.ctr + ctr_seq(p.B, p.Hkv, b);
-            const unsigned t = atomicAdd(word, 1u);
+            const unsigned t = atom_add_acq_rel_gpu(word, 1u);
             last = t == (unsigned)(p.Hq - 1);
-            if (last) {
-                atomicExch(word, 0u);
-                __threadfence();
-            }
+            if (last) atomicExch(word, 0u);
         }
         if (__shfl_sync(0xffffffffu, lane == 0 ? last : 0, 0)) {
             double D2 = 0.0, N2 = 0.0;
