@@ -226,7 +226,7 @@ void make_plan(const alspec_desc& d, int S, int W, int sms, Plan* pl) {
     pl->off_spec_o = take(B * Hq * D * sizeof(float));
     pl->off_mid_ml = take(B * Hq * n2 * 2 * sizeof(float));
     pl->off_mid_o = take(B * Hq * n2 * D * sizeof(float));
-    pl->off_dn = take(B * Hq * 2 * sizeof(float));
+    pl->off_dn = take(B * Hq * merge_splits(D) * 2 * sizeof(float));
     pl->total = off;
 }
 
@@ -517,7 +517,8 @@ alspec_status decode_impl(const alspec_desc* desc, const void* q, const void* k_
     // Programmatic launch right behind the middle kernel (when there is one
     // and no profiling event sits between them).
     const bool pdl = pl.n2 > 0 && !prof_events;
-    if ((st = launch(mk, dim3(desc->n_q_heads, desc->batch), dim3(desc->head_dim * kMergeParts),
+    if ((st = launch(mk, dim3(desc->n_q_heads * merge_splits(desc->head_dim), desc->batch),
+                     dim3(kMergeThreads),
                      0, s, p, pdl ? kLaunchProgrammatic : 0, 0)) != ALSPEC_OK)
         return st;
     if (!prof(4, s)) return ALSPEC_ERR_CUDA;

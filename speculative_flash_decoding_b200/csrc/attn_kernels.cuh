@@ -859,20 +859,22 @@ __device__ __forceinline__ void fill_stage(const Params& p, unsigned char* smem,
     }
     char* ks = reinterpret_cast<char*>(smem) + s * C::kStageBytes;
     char* vs = ks + C::kTileBytes;
+    // The cache rows are read once: evict them from L2 first.
+    const uint64_t pol = l2_evict_first_policy();
     if (MMA) {
         // Whole boxes; rows past the tensor end arrive as zeros.
         mbar_arrive_expect_tx(full_bar + s, (uint32_t)C::kStageBytes);
 #pragma unroll
         for (int h = 0; h < D / 64; ++h) {
-            tma_load_2d(ks + h * TT * 128, &p.tmap_k, 64 * h, head_row + start, full_bar + s);
-            tma_load_2d(vs + h * TT * 128, &p.tmap_v, 64 * h, head_row + start, full_bar + s);
+            tma_load_2d(ks + h * TT * 128, &p.tmap_k, 64 * h, head_row + start, full_bar + s, pol);
+            tma_load_2d(vs + h * TT * 128, &p.tmap_v, 64 * h, head_row + start, full_bar + s, pol);
         }
     } else {
         const uint32_t bytes = (uint32_t)nvalid * C::kRowBytes;
         mbar_arrive_expect_tx(full_bar + s, 2u * bytes);
         const size_t off = ((size_t)head_row + start) * C::kRowBytes;
-        bulk_load(ks, reinterpret_cast<const char*>(p.k) + off, bytes, full_bar + s);
-        bulk_load(vs, reinterpret_cast<const char*>(p.v) + off, bytes, full_bar + s);
+        bulk_load(ks, reinterpret_cast<const char*>(p.k) + off, bytes, full_bar + s, pol);
+        bulk_load(vs, reinterpret_cast<const char*>(p.v) + off, bytes, full_bar + s, pol);
     }
 }
 
@@ -1163,33 +1165,42 @@ __global__ void __launch_bounds__(Cfg<T, D, G, SPEC, MMA>::kThreads, 1)
 
 // ------------------------------------------------------- merge + verify
 
-constexpr int kMergeParts = 4;  // thread groups sharing a head's chunks
+constexpr int kMergeCols = 32;   // output columns per CTA (one per lane)
+constexpr int kMergeParts = 8;   // warps per CTA, each over every 8th chunk
 constexpr int kMergeBatch = 32;  // chunk loads each thread keeps in flight
+constexpr int kMergeThreads = kMergeCols * kMergeParts;
 
-// One CTA per (query head, sequence), D x 4 threads: thread (part, e) owns
-// output element e and the chunks list[part], list[part + 4], ...  O_exact
-// merges the sink-set partial with the sequence's non-empty middle partials;
-// O_spec is rebuilt from the same sink-set partial with the same division,
-// so the two are bit-identical when the middle is empty.  Each head's
-// squared distance and squared norm are reduced in a fixed order; the CTA
-// finishing the last head of a sequence sums them over heads (fixed order,
-// fp64) and writes rel_l2 and the commit flag.
+// Number of (squared distance, squared norm) slots per query head.
+__host__ __device__ constexpr int merge_splits(int d) { return d / kMergeCols; }
+
+// One CTA per (32 output columns of a query head, sequence): lane e of warp
+// `part` owns column split * 32 + e over the chunks list[part],
+// list[part + 8], ...  O_exact merges the sink-set partial with the
+// sequence's non-empty middle partials; O_spec is rebuilt from the same
+// sink-set partial with the same division, so the two are bit-identical when
+// the middle is empty.  Each CTA's squared distance and squared norm over
+// its columns are reduced in a fixed order; the CTA finishing last among a
+// sequence's sums them (fixed order, fp64) and writes rel_l2 and the flag.
+// Splitting a head over D / 32 CTAs spreads the partials' loads over more
+// SMs: one SM pulling a head's 89 x 128 partial columns took ~2 us.
 template <int D, int TT>
-__global__ void __launch_bounds__(D * kMergeParts) merge_kernel(const __grid_constant__ Params p) {
-    constexpr int NT = D * kMergeParts;
-    constexpr int NW = NT / 32;
-    const int h = blockIdx.x;
+__global__ void __launch_bounds__(kMergeThreads) merge_kernel(const __grid_constant__ Params p) {
+    constexpr int NT = kMergeThreads;
+    constexpr int NW = kMergeParts;
+    constexpr int NS = merge_splits(D);
+    const int h = (int)blockIdx.x / NS;
+    const int split = (int)blockIdx.x % NS;
     const int b = blockIdx.y;
     const int tid = threadIdx.x;
-    const int e = tid % D;
-    const int part = tid / D;
-    const int warp = tid >> 5;
     const int lane = tid & 31;
+    const int part = tid >> 5;
+    const int warp = part;
+    const int e = split * kMergeCols + lane;
     const size_t bh = (size_t)b * p.Hq + h;
     __shared__ int list[kMaxChunks];      // non-empty chunks, in order
     __shared__ float wts[kMaxChunks];     // their merge weights
     __shared__ float red[2][NW];
-    __shared__ float accs[kMergeParts][D];
+    __shared__ float accs[kMergeParts][kMergeCols];
     __shared__ int nlist;
     __shared__ int last;
 
@@ -1215,8 +1226,9 @@ __global__ void __launch_bounds__(D * kMergeParts) merge_kernel(const __grid_con
     pdl_wait_prerequisite();
     // One round of independent loads: the sink-set partial, this thread's
     // chunk (m, l) (one chunk per thread: n <= kMaxChunks <= NT) and this
-    // thread's column of its first kMergeBatch chunks (every kMergeParts-th).
+    // lane's column of its warp's first kMergeBatch chunks.
     static_assert(kMaxChunks <= NT, "one chunk (m, l) per thread");
+    static_assert(D % kMergeCols == 0, "head size");
     const float2 sml = __ldcg(reinterpret_cast<const float2*>(p.spec_ml) + bh);
     const float os = __ldcg(p.spec_o + bh * D + e);
     const float2 cm = tid < n ? __ldcg(&mml[list[tid]]) : make_float2(-INFINITY, 0.f);
@@ -1265,51 +1277,43 @@ __global__ void __launch_bounds__(D * kMergeParts) merge_kernel(const __grid_con
             if (i < n) acc = fmaf(wts[i], v[u], acc);
         }
     }
-    accs[part][e] = acc;
+    accs[part][lane] = acc;
     __syncthreads();
-    if (part == 0) {
+    if (warp == 0) {
         const float f0 = merge_weight(sml.x, M);
         float a = f0 * os;
         float l = f0 * sml.y;
 #pragma unroll
-        for (int q = 0; q < kMergeParts; ++q) a += accs[q][e];
+        for (int q = 0; q < kMergeParts; ++q) a += accs[q][lane];
 #pragma unroll
         for (int w = 0; w < NW; ++w) l += red[1][w];
         const float o_spec = __fdiv_rn(os, sml.y);
         const float o_exact = __fdiv_rn(a, l);
         p.out_exact[bh * D + e] = o_exact;
         const float diff = o_exact - o_spec;
-        accs[0][e] = diff * diff;  // each thread only rewrites its own column
-        accs[1][e] = o_exact * o_exact;
-    }
-    __syncthreads();
-    if (warp == 0) {
-        float dd = 0.f, nn = 0.f;
-        for (int i = lane; i < D; i += 32) {
-            dd += accs[0][i];
-            nn += accs[1][i];
-        }
+        float dd = diff * diff;
+        float nn = o_exact * o_exact;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
             dd += __shfl_xor_sync(0xffffffffu, dd, o);
             nn += __shfl_xor_sync(0xffffffffu, nn, o);
         }
         if (lane == 0) {
-            *reinterpret_cast<float2*>(p.dn + bh * 2) = make_float2(dd, nn);
-            // Release: this head's (dd, nn) before the ticket; acquire: the
-            // last head's CTA sees every head's.
+            *reinterpret_cast<float2*>(p.dn + (bh * NS + split) * 2) = make_float2(dd, nn);
+            // Release: this CTA's (dd, nn) before the ticket; acquire: the
+            // sequence's last CTA sees every CTA's.
             unsigned* word = p.ctr + ctr_seq(p.B, p.Hkv, b);
             const unsigned t = atom_add_acq_rel_gpu(word, 1u);
-            last = t == (unsigned)(p.Hq - 1);
+            last = t == (unsigned)(p.Hq * NS - 1);
             if (last) atomicExch(word, 0u);
         }
         if (__shfl_sync(0xffffffffu, lane == 0 ? last : 0, 0)) {
             double D2 = 0.0, N2 = 0.0;
-            for (int hh = lane; hh < p.Hq; hh += 32) {
-                const float2 v =
-                    __ldcg(reinterpret_cast<const float2*>(p.dn) + (size_t)b * p.Hq + hh);
-                D2 += (double)v.x;
-                N2 += (double)v.y;
+            const float2* dn = reinterpret_cast<const float2*>(p.dn) + (size_t)b * p.Hq * NS;
+            for (int i = lane; i < p.Hq * NS; i += 32) {
+                const float2 x = __ldcg(dn + i);
+                D2 += (double)x.x;
+                N2 += (double)x.y;
             }
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) {

@@ -51,27 +51,36 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return done != 0;
 }
 
+// L2 cache policy for data read exactly once: its lines are the first to
+// be evicted, so that what is reused (partials, queries) stays in L2.
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
 // 1-D bulk copy of `bytes` (a multiple of 16, both addresses 16-byte
-// aligned) from global to this CTA's shared memory; completion arrives as
-// transaction bytes on `bar`.
+// aligned) from global to this CTA's shared memory, with L2 policy `pol`;
+// completion arrives as transaction bytes on `bar`.
 __device__ __forceinline__ void bulk_load(void* dst_smem, const void* src_gmem, uint32_t bytes,
-                                          uint64_t* bar) {
+                                          uint64_t* bar, uint64_t pol) {
     asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
-            "r"(smem_addr(dst_smem)),
-        "l"(src_gmem), "r"(bytes), "r"(smem_addr(bar))
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1], %2, [%3], %4;" ::"r"(smem_addr(dst_smem)),
+        "l"(src_gmem), "r"(bytes), "r"(smem_addr(bar)), "l"(pol)
         : "memory");
 }
 
 // 2-D tiled TMA load of one box at element coordinates (x, y) of the tensor
-// map; x * element size must be a multiple of 16 bytes.  Rows outside the
-// tensor are filled with zeros; the full box counts as transaction bytes.
+// map, with L2 policy `pol`; x * element size must be a multiple of 16
+// bytes.  Rows outside the tensor are filled with zeros; the full box counts
+// as transaction bytes.
 __device__ __forceinline__ void tma_load_2d(void* dst_smem, const void* tmap, int x, int y,
-                                            uint64_t* bar) {
+                                            uint64_t* bar, uint64_t pol) {
     asm volatile(
         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_addr(dst_smem)),
-        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(smem_addr(bar))
+        ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_addr(dst_smem)),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(smem_addr(bar)), "l"(pol)
         : "memory");
 }
 
