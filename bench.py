@@ -60,6 +60,50 @@ def dist_env():
 
 # ------------------------------------------------------------------ helpers
 
+class Ranks:
+    """One process per GPU (launched by torchrun): rank and world size from
+    the environment, a process group (NCCL on the GPUs, gloo in the CPU
+    tests) for the barrier and the max-over-ranks reduction of times.  The
+    ranks are independent replicas: no collective touches the data path."""
+
+    def __init__(self, backend, device):
+        import torch
+        self.torch = torch
+        self.rank, self.world, self.local = dist_env()
+        self.device = device
+        self.pg = None
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            kw = {"device_id": device} if backend == "nccl" else {}
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
+            self.pg = dist
+
+    def barrier(self):
+        if self.device.type == "cuda":
+            self.torch.cuda.synchronize(self.device)
+        if self.pg:
+            self.pg.barrier()
+
+    def max(self, x):
+        """The largest x over all ranks (every rank gets it)."""
+        if not self.pg:
+            return float(x)
+        t = self.torch.tensor([float(x)], dtype=self.torch.float64, device=self.device)
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            self.pg.destroy_process_group()
+            self.pg = None
+
+
+def job_throughput(bytes_per_rank, world, ms_per_step):
+    """Whole-job GB/s: every rank's bytes over the slowest rank's step time."""
+    return bytes_per_rank * world / (ms_per_step * 1e-3) / 1e9
+
+
 def measured_peak():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -232,13 +276,7 @@ def run_alspec(args, wl):
     rank, world, local = dist_env()
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
-    pg = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=device)
-        pg = dist
+    ranks = Ranks("nccl", device)
 
     n_layers = args.layers or wl.n_layers
     layers = [workloads.make_layer(wl, layer=i, device=device) for i in range(n_layers)]
@@ -313,10 +351,7 @@ def run_alspec(args, wl):
 
     lat = [capture_latency(traces[j]) for j in range(prof_steps)]
 
-    def barrier():
-        torch.cuda.synchronize(device)
-        if pg:
-            pg.barrier()
+    barrier = ranks.barrier
 
     for _ in range(args.warmup):
         sfd.alspec_graph_launch(warm_graph, stream.cuda_stream)
@@ -328,26 +363,37 @@ def run_alspec(args, wl):
         uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
     except Exception:
         uuid = None
+    # Steps whose cache fits a few times in L2 are preceded by an untimed
+    # write of twice the L2 size, then a read of another such buffer (so the
+    # step does not pay for writing the flush's dirty lines back); each step
+    # is then timed on its own.
+    l2_bytes = int(getattr(torch.cuda.get_device_properties(device), "L2_cache_size", 0) or
+                   (126 << 20))
+    flush = kv_bytes < 4 * l2_bytes
+    scrub = torch.empty(2 * l2_bytes, dtype=torch.uint8, device=device) if flush else None
+    clean = torch.ones(l2_bytes // 2, dtype=torch.int32, device=device) if flush else None
+    sink = torch.empty((), dtype=torch.int64, device=device) if flush else None
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
-    step_marks = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    step_begin = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    step_end = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     with ClockSampler(uuid) as clocks:
         barrier()
         t_start.record(stream)
         for i in range(args.steps):
-            step_marks[i].record(stream)
+            if flush:
+                with torch.cuda.stream(stream):
+                    scrub.zero_()
+                    torch.sum(clean, dim=0, out=sink)
+            step_begin[i].record(stream)
             st = sfd.alspec_graph_launch(graphs[i], stream.cuda_stream)
             assert st == 0
-        step_marks[args.steps].record(stream)
+            step_end[i].record(stream)
         t_end.record(stream)
         barrier()
-    ms_total = t_start.elapsed_time(t_end)
-    ms_per_step = ms_total / args.steps
-    if pg:
-        t = torch.tensor([ms_per_step], device=device)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms_per_step = float(t.item())
-    per_step = [step_marks[i].elapsed_time(step_marks[i + 1]) for i in range(args.steps)]
+    per_step = [step_begin[i].elapsed_time(step_end[i]) for i in range(args.steps)]
+    ms_total = sum(per_step) if flush else t_start.elapsed_time(t_end)
+    ms_per_step = ranks.max(ms_total / args.steps)
 
     # Profiled pass: same step with per-layer events captured in the graphs.
     barrier()
@@ -408,21 +454,16 @@ def run_alspec(args, wl):
                 stream.synchronize()
             e1.record(stream)
         barrier()
-        e2e_ms = e0.elapsed_time(e1) / args.steps
-        if pg:
-            t = torch.tensor([e2e_ms], device=device)
-            pg.all_reduce(t, op=pg.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = ranks.max(e0.elapsed_time(e1) / args.steps)
         h2d = q_host.numel() * q_host.element_size() + lens_host.numel() * lens_host.element_size()
         d2h = rel_host.numel() * rel_host.element_size() + com_host.numel() * com_host.element_size()
-        e2e = {"value": kv_bytes * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+        e2e = {"value": job_throughput(kv_bytes, world, e2e_ms), "unit": "GB/s",
                "us_per_step": e2e_ms * 1e3, "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h)}
 
     for g in [warm_graph] + graphs + prof_graphs + lat:
         sfd.alspec_graph_destroy(g)
-    if pg:
-        pg.destroy_process_group()
+    ranks.close()
     if rank != 0:
         return
 
@@ -433,7 +474,7 @@ def run_alspec(args, wl):
     mid_avg_ms = sum(mid_ms) / len(mid_ms)
     achieved = mid_bytes / (mid_avg_ms * 1e-3) / 1e9
     traffic = stored_traffic()
-    value = kv_bytes * world / (ms_per_step * 1e-3) / 1e9
+    value = job_throughput(kv_bytes, world, ms_per_step)
 
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
@@ -461,7 +502,11 @@ def run_alspec(args, wl):
         "config": {"workload": wl.name, "layers": n_layers, "batch": wl.B, "q_heads": wl.Hq,
                    "kv_heads": wl.Hkv, "head_dim": wl.d, "context": wl.L, "sink": wl.S,
                    "window": wl.W, "lambda": wl.lam, "kv_bytes_per_step": kv_bytes,
-                   "l2": "inputs larger than L2: 537 MB of KV per layer, 17.2 GB per step; no flush",
+                   "l2": ("L2 flushed before every timed step (untimed write of %d MB, then "
+                          "a read of %d MB of other data); %.1f MB of KV per step"
+                          % (2 * l2_bytes >> 20, 2 * l2_bytes >> 20, kv_bytes / 1e6))
+                   if flush else ("inputs larger than L2: %.1f MB of KV per step against "
+                                  "%d MB of L2; no flush" % (kv_bytes / 1e6, l2_bytes >> 20)),
                    "parallelism": "replicas" if world > 1 else "single",
                    "timing": "CUDA graph per step, CUDA events on the launch stream; "
                              "per-kernel times from a second pass of graphs with per-layer "

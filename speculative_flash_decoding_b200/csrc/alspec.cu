@@ -24,6 +24,10 @@ namespace {
 constexpr int kMaxDevices = 64;
 constexpr int kMaxSpecItems = kMaxSpecCtas;  // sink-set CTAs per (sequence, KV head)
 
+// Smallest middle chunk of the guided self-scheduled split, in tiles.
+#ifndef ALSPEC_GSS_MIN_TILES
+#define ALSPEC_GSS_MIN_TILES 16
+#endif
 #ifndef ALSPEC_MID_SM_RESERVE
 #define ALSPEC_MID_SM_RESERVE 0
 #endif
@@ -182,7 +186,7 @@ void make_plan(const alspec_desc& d, int S, int W, int sms, Plan* pl) {
             const int n = std::min(kMaxChunks, ceil_div(mid_tiles, ct));
             for (int c = 0; c < n; ++c) sizes.push_back((double)ct / mid_tiles);
         } else {
-            const double smin = std::min(1.0, 16.0 / mid_tiles);
+            const double smin = std::min(1.0, (double)ALSPEC_GSS_MIN_TILES / mid_tiles);
             double r = 1.0;
             while (r > 1e-9 && (int)sizes.size() < kMaxChunks) {
                 double s = std::max((double)heads * r / (1.5 * P), smin);
