@@ -50,6 +50,8 @@ def parse_args():
     ap.add_argument("--split-tokens", type=int, default=0,
                     help="exact-path item size for the longest sequence (0 = library's choice)")
     ap.add_argument("--engine", default="auto", choices=["auto", "cuda_cores", "tensor_cores"])
+    ap.add_argument("--lambda-sweep", action="store_true",
+                    help="hit rate against the threshold on the commit-mixing workload family")
     return ap.parse_args()
 
 
@@ -544,11 +546,57 @@ def run_alspec(args, wl):
     print(json.dumps(line), flush=True)
 
 
+LAMBDA_GRID = (0.0, 1e-4, 2e-4, 5e-4, 1e-3, 2e-3, 5e-3, 1e-2, 2e-2, 5e-2, 0.1, 0.2, 0.5, 1.0)
+
+
+def run_lambda_sweep(args):
+    """Hit rate (share of tokens whose speculative attention output would be
+    committed) against the threshold lambda, on the commit-mixing family:
+    per layer one decode of a batch of 8 sequences of 24K-32K tokens with
+    strong sinks and occasional needles.  The flag is rel_l2 <= lambda, so
+    one decode per layer gives the whole curve; the decode at the middle
+    threshold checks the device's flags against that rule."""
+    import numpy as np
+    import torch
+    import workloads
+    import speculative_flash_decoding_b200 as sfd
+    rank, world, local = dist_env()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    wl = workloads.COMMIT_VARIANT
+    n_layers = args.layers or 8
+    dec = sfd.Decoder(wl.B, wl.Hq, wl.Hkv, wl.d, wl.L, wl.dtype, wl.S, wl.W, device=device)
+    rel = []
+    for layer in range(n_layers):
+        data = workloads.make_layer(wl, layer=layer, device=device)
+        out = dec.decode(data["q"], data["k"], data["v"], data["seq_lens"], wl.lam)
+        r = out["rel_l2"].cpu().numpy().astype(np.float64)
+        flags = out["commit"].cpu().numpy()
+        assert (flags == (r <= wl.lam)).all()
+        rel.append(r)
+        del data
+    r = np.concatenate(rel)
+    hit = [float((r <= lam).mean()) for lam in LAMBDA_GRID]
+    if rank != 0:
+        return
+    line = {"metric": "hit rate vs lambda (commit-mixing family)", "unit": "fraction of tokens",
+            "lambdas": list(LAMBDA_GRID), "hit_rate": hit, "tokens": int(r.size),
+            "rel_l2_quantiles": {q: float(np.quantile(r, q)) for q in (0.1, 0.25, 0.5, 0.75, 0.9)},
+            "data": "synthetic",
+            "config": {"workload": wl.name, "layers": n_layers, "batch": wl.B, "q_heads": wl.Hq,
+                       "kv_heads": wl.Hkv, "head_dim": wl.d, "lengths": list(wl.ragged),
+                       "sink": wl.S, "window": wl.W, "sink_bump": wl.sink_bump,
+                       "needle_bump": wl.needle_bump, "needles": list(wl.needles)}}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse_args()
     import workloads
     wl = workloads.CONFIGS[args.config]
-    if args.impl == "reference":
+    if args.lambda_sweep:
+        run_lambda_sweep(args)
+    elif args.impl == "reference":
         run_reference(args, wl)
     else:
         run_alspec(args, wl)

@@ -58,6 +58,31 @@ def test_commit_variant_gives_both_flags(cuda_device):
     assert 0 < ref["commit"].sum() < wl.B, "variant should mix commit and discard"
 
 
+LAMBDAS = (0.0, 1e-4, 3e-4, 1e-3, 3e-3, 1e-2, 3e-2, 0.1, 0.3, 1.0)
+
+
+def test_lambda_sweep_flags_match_oracle(cuda_device):
+    """Hit-rate curve on the commit-mixing family: at every threshold the
+    flags equal the oracle's (outside the +-1e-3 band around lambda) and
+    rel_l2 does not depend on lambda."""
+    from parity import FLAG_BAND
+    wl = workloads.COMMIT_VARIANT.replace(L=8192, ragged=(6000, 8192))
+    hits = np.zeros(len(LAMBDAS))
+    for layer in range(3):
+        data = workloads.make_layer(wl, layer=layer, device=cuda_device)
+        r_ref = oracle_decode(wl, data)["rel_l2"]
+        dec, first = gpu_decode(wl, data, cuda_device)
+        for j, lam in enumerate(LAMBDAS):
+            out = dec.decode(data["q"], data["k"], data["v"], data["seq_lens"], lam)
+            torch.cuda.synchronize()
+            assert torch.equal(out["rel_l2"].cpu(), first["rel_l2"])
+            flags = out["commit"].cpu().numpy()
+            clear = np.abs(r_ref - lam) > FLAG_BAND
+            assert (flags[clear] == (r_ref[clear] <= lam)).all(), (lam, flags, r_ref)
+            hits[j] += flags.mean() / 3
+    assert (np.diff(hits) >= 0).all() and hits[0] == 0.0 and hits[-1] > 0.5, hits
+
+
 EDGE = []
 for dtype, d, engine in (("f32", 64, "cuda_cores"), ("bf16", 64, "cuda_cores"),
                          ("bf16", 128, "cuda_cores"), ("f32", 128, "cuda_cores"),
