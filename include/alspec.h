@@ -182,6 +182,52 @@ alspec_status alspec_decode_traced(const alspec_desc* desc,
                                    void* stream, unsigned long long* trace_ns);
 
 /*
+ * Output projection of attention outputs -- the linear map that follows
+ * self-attention in a decoder layer (the post-attention op the pages run
+ * speculatively, "Approach"):
+ *     y[b, j] = sum_i x[b, i] * w[j, i]
+ * on CUDA cores (decode batches are small: the op streams w once).
+ *   x     device fp32 [batch][k], 16-byte aligned
+ *   w     device bf16 [n][k] (row j = output feature j), 16-byte aligned
+ *   y     device fp32 [batch][n]
+ *   skip  device uint8 [batch] or NULL: rows b with skip[b] != 0 are not
+ *         written (pass the commit flags to redo only discarded tokens)
+ *   batch 1..8; k a positive multiple of 8; n >= 1.
+ * Asynchronous on `stream`; ALSPEC_ERR_INVALID_ARG for a bad argument.
+ */
+alspec_status alspec_oproj(const float* x, const void* w, float* y, const uint8_t* skip,
+                           int batch, int k, int n, void* stream);
+
+/*
+ * alspec_decode followed by the output projection of the attention output,
+ * run speculatively (the single-GPU form of the pages' speculative
+ * post-attention ops with commit or discard, "Approach"):
+ *   y[b] = o_proj(commit[b] ? O_spec[b] : O_exact[b]),  o_proj as in
+ *   alspec_oproj with w_o bf16 [hidden][n_q_heads * head_dim].
+ * The projection of O_spec runs on the high-priority stream right after the
+ * sink-set kernel, beside the exact path; after the merge, the projection of
+ * O_exact overwrites the rows of discarded tokens.  Inside a stream capture
+ * that recomputation is a conditional node of the graph which the merge
+ * kernel enables only when it discards a token; outside a capture it is
+ * launched and skips committed rows.  With every token committed, y is
+ * final when the flags are, instead of one projection later.
+ *   y        device fp32 [batch][hidden]; batch <= 8
+ *   trace_ns NULL, or device 3 x uint64 zeroed by the caller: [0] and [1] as
+ *            in alspec_decode_traced, [2] raised to the global timer after
+ *            each projection's last write (y is final at max([1], [2])).
+ * out_spec and out_exact must be 16-byte aligned.  Other arguments as for
+ * alspec_decode.
+ */
+alspec_status alspec_decode_oproj(const alspec_desc* desc,
+                                  const void* q, const void* k_cache, const void* v_cache,
+                                  const int32_t* seq_lens, int n_sink, int window,
+                                  float lambda, const void* w_o, int hidden,
+                                  float* out_spec, float* out_exact, float* rel_l2,
+                                  uint8_t* commit, float* y,
+                                  void* workspace, size_t workspace_bytes,
+                                  void* stream, unsigned long long* trace_ns);
+
+/*
  * Work plan the library would use (host only, no CUDA call except the SM
  * count query).  info[] receives, in order:
  *   0 tokens per sink-set work item      1 sink-set items per (b, kv head)

@@ -29,9 +29,12 @@ _SIGS = {
     "alspec_oracle_commit": ("d", "d"),
     "alspec_oracle_decode": ("i", "i", "i", "i", "i", "i", "p", "p", "p", "p", "i",
                              "i", "d", "p", "p", "p", "p", "i"),
+    "alspec_oracle_oproj": ("i", "i", "i", "p", "p", "i", "p"),
+    "alspec_oracle_oproj_gated": ("i", "i", "i", "p", "p", "p", "p", "i", "p"),
 }
 _RES = {"alspec_oracle_head": "i", "alspec_oracle_rel_l2": "d",
-        "alspec_oracle_commit": "i", "alspec_oracle_decode": "i"}
+        "alspec_oracle_commit": "i", "alspec_oracle_decode": "i",
+        "alspec_oracle_oproj": "i", "alspec_oracle_oproj_gated": "i"}
 _CT = {"i": ctypes.c_int, "p": ctypes.c_void_p, "l": ctypes.c_long, "d": ctypes.c_double}
 
 _libs = {}
@@ -134,3 +137,35 @@ def decode(q, k, v, seq_lens, n_sink, window, lam, n_threads=0, lib=None):
         raise ValueError(f"alspec_oracle_decode failed with status {-used}")
     return dict(out_spec=out_spec, out_exact=out_exact, rel_l2=rel, commit=flag,
                 threads=used)
+
+
+def oproj(x, w, lib=None):
+    """y[b, j] = sum_i x[b, i] * w[j, i] in fp64 (the projection after attention).
+
+    x: [B, K] (any float array, widened to fp64); w: [N, K] float32, float64
+    or bfloat16 bits (uint16)."""
+    x = np.ascontiguousarray(np.asarray(x, np.float64).reshape(-1, np.shape(w)[-1]))
+    w = np.ascontiguousarray(w)
+    B, K = x.shape
+    N = w.shape[0]
+    y = np.zeros((B, N), np.float64)
+    rc = _load(lib).alspec_oracle_oproj(B, K, N, _ptr(x), _ptr(w), _dtype_code(w), _ptr(y))
+    if rc != 0:
+        raise ValueError(f"oracle oproj rejected its arguments ({rc})")
+    return y
+
+
+def oproj_gated(o_spec, o_exact, commit, w, lib=None):
+    """y[b] = oproj(commit[b] ? o_spec[b] : o_exact[b]) (commit or discard)."""
+    w = np.ascontiguousarray(w)
+    K = w.shape[1]
+    os_ = np.ascontiguousarray(np.asarray(o_spec, np.float64).reshape(-1, K))
+    oe = np.ascontiguousarray(np.asarray(o_exact, np.float64).reshape(-1, K))
+    c = np.ascontiguousarray(np.asarray(commit, np.uint8).reshape(-1))
+    B, N = os_.shape[0], w.shape[0]
+    y = np.zeros((B, N), np.float64)
+    rc = _load(lib).alspec_oracle_oproj_gated(B, K, N, _ptr(os_), _ptr(oe), _ptr(c), _ptr(w),
+                                              _dtype_code(w), _ptr(y))
+    if rc != 0:
+        raise ValueError(f"oracle oproj_gated rejected its arguments ({rc})")
+    return y

@@ -31,6 +31,9 @@
  * and the weighted sum of value rows.  There is no tiling, no online
  * rescaling and no reordering beyond that definition.
  *
+ * It also holds the output projection that follows attention (a plain
+ * matrix-vector product per token) and its commit-gated form.
+ *
  * Parity status of every function here: pinned by tests/test_oracle.py
  * (hand-derived cases in tests/golden, closed forms, invariants, a planted
  * needle, and a numpy textbook cross-check).
@@ -259,4 +262,53 @@ int alspec_oracle_decode(int B, int Hq, int Hkv, int d, int Lmax, int dtype,
         commit[b] = (uint8_t)alspec_oracle_commit(rel_l2[b], lambda);
     }
     return used;
+}
+
+/*
+ * Output projection that follows self-attention in a decoder layer: the
+ * post-attention op that attention-level speculation runs on the
+ * approximate output while the exact one is computed (atlas.scime.ai
+ * summary, "Approach").  The plain definition, in double:
+ *   y[b][j] = sum over i = 0 .. K-1, ascending, of x[b][i] * w[j][i]
+ *   x : [B, K] doubles;  w : [N, K] of element type w_dtype (row j is output
+ *   feature j);  y : [B, N] doubles.
+ * Returns OR_OK or OR_BAD_ARG.
+ */
+int alspec_oracle_oproj(int B, int K, int N, const double* x, const void* w, int w_dtype,
+                        double* y) {
+    if (B <= 0 || K <= 0 || N <= 0 || !x || !w || !y || !elem_size(w_dtype)) {
+        return OR_BAD_ARG;
+    }
+    for (int b = 0; b < B; ++b) {
+        for (int j = 0; j < N; ++j) {
+            double acc = 0.0;
+            for (int i = 0; i < K; ++i) {
+                acc += x[(size_t)b * K + i] * load_elem(w, w_dtype, (size_t)j * K + i);
+            }
+            y[(size_t)b * N + j] = acc;
+        }
+    }
+    return OR_OK;
+}
+
+/*
+ * The projection with commit or discard ("Approach": the speculative
+ * post-attention result is kept when the check commits, otherwise the op is
+ * redone on the exact attention output):
+ *   y[b] = o_proj(commit[b] ? o_spec[b] : o_exact[b])
+ * o_spec, o_exact : [B, K] doubles; commit : [B] bytes (non-zero = commit).
+ */
+int alspec_oracle_oproj_gated(int B, int K, int N, const double* o_spec, const double* o_exact,
+                              const uint8_t* commit, const void* w, int w_dtype, double* y) {
+    if (B <= 0 || !o_spec || !o_exact || !commit) {
+        return OR_BAD_ARG;
+    }
+    for (int b = 0; b < B; ++b) {
+        const double* x = commit[b] ? o_spec + (size_t)b * K : o_exact + (size_t)b * K;
+        int rc = alspec_oracle_oproj(1, K, N, x, w, w_dtype, y + (size_t)b * N);
+        if (rc != OR_OK) {
+            return rc;
+        }
+    }
+    return OR_OK;
 }

@@ -17,6 +17,7 @@
 
 #include "alspec.h"
 #include "attn_kernels.cuh"
+#include "oproj_kernels.cuh"
 
 namespace alspec {
 namespace {
@@ -63,6 +64,7 @@ struct DeviceState {
     cudaStream_t hi = nullptr;
     cudaEvent_t fork = nullptr;
     cudaEvent_t join = nullptr;
+    cudaEvent_t join2 = nullptr;  // after the speculative output projection
     int sm_count = 0;
     int prio_hi = 0;
     std::set<const void*> attr_done;
@@ -82,7 +84,8 @@ alspec_status get_device_state(DeviceState** out) {
             !ok(cudaDeviceGetStreamPriorityRange(&lo, &hi)) ||
             !ok(cudaStreamCreateWithPriority(&d.hi, cudaStreamNonBlocking, hi)) ||
             !ok(cudaEventCreateWithFlags(&d.fork, cudaEventDisableTiming)) ||
-            !ok(cudaEventCreateWithFlags(&d.join, cudaEventDisableTiming))) {
+            !ok(cudaEventCreateWithFlags(&d.join, cudaEventDisableTiming)) ||
+            !ok(cudaEventCreateWithFlags(&d.join2, cudaEventDisableTiming))) {
             return ALSPEC_ERR_CUDA;
         }
         d.prio_hi = hi;
@@ -421,12 +424,41 @@ alspec_status alspec_query_chunks(const alspec_desc* desc, int n_sink, int windo
 namespace alspec {
 namespace {
 
+// The output projection that follows attention, run speculatively on O_spec
+// and redone on O_exact for discarded tokens (alspec_decode_oproj).
+struct OprojReq {
+    const void* w;  // bf16 [hidden][Hq * d]
+    int hidden;
+    float* y;       // fp32 [B][hidden]
+};
+
+bool oproj_args_ok(const float* x, const void* w, const float* y, int batch, int k, int n) {
+    return x && w && y && batch >= 1 && batch <= kOprojMaxB && k >= 8 && k % 8 == 0 && n >= 1 &&
+           aligned16(x) && aligned16(w) && (reinterpret_cast<uintptr_t>(y) & 3u) == 0;
+}
+
+OprojParams oproj_params(const float* x, const void* w, float* y, const uint8_t* skip, int batch,
+                         int k, int n, unsigned long long* trace) {
+    OprojParams o{};
+    o.x = x;
+    o.w = static_cast<const uint4*>(w);
+    o.y = y;
+    o.skip = skip;
+    o.B = batch;
+    o.K = k;
+    o.N = n;
+    o.trace = trace;
+    return o;
+}
+
+dim3 oproj_grid(int n) { return dim3((unsigned)ceil_div(n, kOprojWarps * kOprojRows)); }
+
 alspec_status decode_impl(const alspec_desc* desc, const void* q, const void* k_cache,
                           const void* v_cache, const int32_t* seq_lens, int n_sink, int window,
                           float lambda, float* out_spec, float* out_exact, float* rel_l2,
                           uint8_t* commit, void* workspace, size_t workspace_bytes, void* stream,
                           void* spec_event, void* const* prof_events,
-                          unsigned long long* trace_ns) {
+                          unsigned long long* trace_ns, const OprojReq* op = nullptr) {
     alspec_status st = check_desc(desc, n_sink, window);
     if (st != ALSPEC_OK) return st;
     if (reinterpret_cast<uintptr_t>(trace_ns) & 7u) return ALSPEC_ERR_INVALID_ARG;
@@ -500,6 +532,15 @@ alspec_status decode_impl(const alspec_desc* desc, const void* q, const void* k_
         return ALSPEC_ERR_CUDA;
     if (!prof(1, ds->hi)) return ALSPEC_ERR_CUDA;
     if (!ok(cudaEventRecord(ds->join, ds->hi))) return ALSPEC_ERR_CUDA;
+    const int kdim = desc->n_q_heads * desc->head_dim;
+    if (op) {
+        // Speculative output projection of O_spec, beside the exact path.
+        const OprojParams o = oproj_params(out_spec, op->w, op->y, nullptr, desc->batch, kdim,
+                                           op->hidden, trace_ns ? trace_ns + 2 : nullptr);
+        oproj_kernel<<<oproj_grid(op->hidden), kOprojWarps * 32, 0, ds->hi>>>(o);
+        if (!ok(cudaGetLastError()) || !ok(cudaEventRecord(ds->join2, ds->hi)))
+            return ALSPEC_ERR_CUDA;
+    }
 #ifdef ALSPEC_SPEC_SERIAL
     if (!ok(cudaStreamWaitEvent(s, ds->join, 0))) return ALSPEC_ERR_CUDA;
 #endif
@@ -518,6 +559,24 @@ alspec_status decode_impl(const alspec_desc* desc, const void* q, const void* k_
         mk = pl.tt == 32 ? merge_kernel<128, 32> : merge_kernel<128, 16>;
     else
         mk = pl.tt == 32 ? merge_kernel<64, 32> : merge_kernel<64, 16>;
+    // Inside a stream capture the recomputation of discarded tokens' output
+    // projection is a conditional node: the merge kernel sets its condition
+    // when it discards a token.
+    bool capturing = false;
+    cudaGraphConditionalHandle cond = 0;
+    if (op) {
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        cudaGraph_t cg = nullptr;
+        if (!ok(cudaStreamGetCaptureInfo(s, &cs, nullptr, &cg, nullptr, nullptr)))
+            return ALSPEC_ERR_CUDA;
+        capturing = cs == cudaStreamCaptureStatusActive;
+        if (capturing) {
+            if (!ok(cudaGraphConditionalHandleCreate(&cond, cg, 0, cudaGraphCondAssignDefault)))
+                return ALSPEC_ERR_CUDA;
+            p.cond = static_cast<unsigned long long>(cond);
+            p.cond_on = 1;
+        }
+    }
     // Programmatic launch right behind the middle kernel (when there is one
     // and no profiling event sits between them).
     const bool pdl = pl.n2 > 0 && !prof_events;
@@ -525,6 +584,44 @@ alspec_status decode_impl(const alspec_desc* desc, const void* q, const void* k_
                      dim3(kMergeThreads),
                      0, s, p, pdl ? kLaunchProgrammatic : 0, 0)) != ALSPEC_OK)
         return st;
+    if (op) {
+        // Redo the projection on O_exact for the discarded tokens, after the
+        // speculative one (both write y).
+        if (!ok(cudaStreamWaitEvent(s, ds->join2, 0))) return ALSPEC_ERR_CUDA;
+        OprojParams r = oproj_params(out_exact, op->w, op->y, commit, desc->batch, kdim,
+                                     op->hidden, trace_ns ? trace_ns + 2 : nullptr);
+        if (capturing) {
+            cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+            cudaGraph_t g = nullptr;
+            const cudaGraphNode_t* deps = nullptr;
+            size_t ndeps = 0;
+            if (!ok(cudaStreamGetCaptureInfo(s, &cs, nullptr, &g, &deps, &ndeps)))
+                return ALSPEC_ERR_CUDA;
+            cudaGraphNodeParams cp{};
+            cp.type = cudaGraphNodeTypeConditional;
+            cp.conditional.handle = cond;
+            cp.conditional.type = cudaGraphCondTypeIf;
+            cp.conditional.size = 1;
+            cudaGraphNode_t cn = nullptr;
+            if (!ok(cudaGraphAddNode(&cn, g, deps, ndeps, &cp))) return ALSPEC_ERR_CUDA;
+            cudaGraphNodeParams kp{};
+            kp.type = cudaGraphNodeTypeKernel;
+            kp.kernel.func = reinterpret_cast<void*>(oproj_kernel);
+            kp.kernel.gridDim = oproj_grid(op->hidden);
+            kp.kernel.blockDim = dim3(kOprojWarps * 32);
+            kp.kernel.sharedMemBytes = 0;
+            void* args[] = {&r};
+            kp.kernel.kernelParams = args;
+            cudaGraphNode_t kn = nullptr;
+            if (!ok(cudaGraphAddNode(&kn, cp.conditional.phGraph_out[0], nullptr, 0, &kp)) ||
+                !ok(cudaStreamUpdateCaptureDependencies(s, &cn, 1,
+                                                        cudaStreamSetCaptureDependencies)))
+                return ALSPEC_ERR_CUDA;
+        } else {
+            oproj_kernel<<<oproj_grid(op->hidden), kOprojWarps * 32, 0, s>>>(r);
+            if (!ok(cudaGetLastError())) return ALSPEC_ERR_CUDA;
+        }
+    }
     if (!prof(4, s)) return ALSPEC_ERR_CUDA;
     return ALSPEC_OK;
 }
@@ -554,6 +651,32 @@ alspec_status alspec_decode_traced(const alspec_desc* desc, const void* q, const
     return decode_impl(desc, q, k_cache, v_cache, seq_lens, n_sink, window, lambda, out_spec,
                        out_exact, rel_l2, commit, workspace, workspace_bytes, stream, nullptr,
                        nullptr, trace_ns);
+}
+
+alspec_status alspec_oproj(const float* x, const void* w, float* y, const uint8_t* skip, int batch,
+                           int k, int n, void* stream) {
+    if (!oproj_args_ok(x, w, y, batch, k, n)) return ALSPEC_ERR_INVALID_ARG;
+    const OprojParams o = oproj_params(x, w, y, skip, batch, k, n, nullptr);
+    oproj_kernel<<<oproj_grid(n), kOprojWarps * 32, 0, static_cast<cudaStream_t>(stream)>>>(o);
+    return ok(cudaGetLastError()) ? ALSPEC_OK : ALSPEC_ERR_CUDA;
+}
+
+alspec_status alspec_decode_oproj(const alspec_desc* desc, const void* q, const void* k_cache,
+                                  const void* v_cache, const int32_t* seq_lens, int n_sink,
+                                  int window, float lambda, const void* w_o, int hidden,
+                                  float* out_spec, float* out_exact, float* rel_l2,
+                                  uint8_t* commit, float* y, void* workspace,
+                                  size_t workspace_bytes, void* stream,
+                                  unsigned long long* trace_ns) {
+    if (!desc) return ALSPEC_ERR_INVALID_ARG;
+    const int kdim = desc->n_q_heads * desc->head_dim;
+    if (!oproj_args_ok(out_spec, w_o, y, desc->batch, kdim, hidden) || !out_exact ||
+        !aligned16(out_exact))
+        return ALSPEC_ERR_INVALID_ARG;
+    const OprojReq op{w_o, hidden, y};
+    return decode_impl(desc, q, k_cache, v_cache, seq_lens, n_sink, window, lambda, out_spec,
+                       out_exact, rel_l2, commit, workspace, workspace_bytes, stream, nullptr,
+                       nullptr, trace_ns, &op);
 }
 
 alspec_status alspec_get_device_error(void* workspace, size_t workspace_bytes, void* stream,
@@ -623,6 +746,7 @@ alspec_status alspec_shutdown(void) {
         if (cudaStreamSynchronize(s.hi) != cudaSuccess) st = ALSPEC_ERR_CUDA;
         cudaEventDestroy(s.fork);
         cudaEventDestroy(s.join);
+        if (s.join2) cudaEventDestroy(s.join2);
         cudaStreamDestroy(s.hi);
         s = DeviceState{};
     }

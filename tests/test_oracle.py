@@ -325,3 +325,61 @@ def test_bad_arguments_raise():
         oracle.decode(q, k, k, np.array([4], np.int32), 0, 0, 0.1)      # empty sink set
     with pytest.raises(ValueError):
         oracle.head(np.zeros(4), np.zeros((3, 4)), np.zeros((3, 4)), -1, 2)
+
+
+# ------------------------------------------------------- output projection
+
+OPROJ_GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden",
+                            "oproj_cases.json")
+
+
+def _oproj_cases():
+    with open(OPROJ_GOLDEN) as f:
+        return {c["name"]: c for c in json.load(f)["cases"]}
+
+
+def test_oproj_hand_cases():
+    c = _oproj_cases()
+    a = c["non_square_two_tokens"]
+    y = oracle.oproj(np.array(a["x"]), np.array(a["w"], np.float32))
+    assert np.array_equal(y, np.array(a["y"]))
+    g = c["gated_one_commit_one_discard"]
+    y = oracle.oproj_gated(g["o_spec"], g["o_exact"], g["commit"], np.array(g["w"], np.float64))
+    assert np.array_equal(y, np.array(g["y"]))
+    h = c["bf16_weights"]
+    y = oracle.oproj(np.array(h["x"]), np.array(h["w_bf16_bits"], np.uint16))
+    assert np.array_equal(y, np.array(h["y"]))
+
+
+def test_oproj_one_hot_rows_pick_entries():
+    """w row j = unit vector e_pi(j): y[b, j] = x[b, pi(j)] exactly."""
+    rng = np.random.default_rng(11)
+    K, N = 24, 17
+    perm = rng.integers(0, K, N)
+    w = np.zeros((N, K), np.float32)
+    w[np.arange(N), perm] = 1.0
+    x = rng.standard_normal((3, K))
+    assert np.array_equal(oracle.oproj(x, w), x[:, perm])
+
+
+def test_oproj_all_ones_gives_row_sums():
+    """Closed form: w = 1 everywhere gives every output the sum of its row."""
+    rng = np.random.default_rng(12)
+    x = rng.standard_normal((2, 64))
+    y = oracle.oproj(x, np.ones((5, 64), np.float32))
+    for b in range(2):
+        assert np.allclose(y[b], math.fsum(x[b]), rtol=0, atol=1e-12)
+
+
+def test_oproj_is_linear_and_gating_selects_rows():
+    rng = np.random.default_rng(13)
+    K, N = 32, 9
+    w = rng.standard_normal((N, K)).astype(np.float32)
+    x1, x2 = rng.standard_normal((2, K)), rng.standard_normal((2, K))
+    lhs = oracle.oproj(2.0 * x1 - 0.5 * x2, w)
+    rhs = 2.0 * oracle.oproj(x1, w) - 0.5 * oracle.oproj(x2, w)
+    assert np.allclose(lhs, rhs, rtol=0, atol=1e-12)
+    commit = np.array([1, 0], np.uint8)
+    y = oracle.oproj_gated(x1, x2, commit, w)
+    assert np.array_equal(y[0], oracle.oproj(x1[:1], w)[0])
+    assert np.array_equal(y[1], oracle.oproj(x2[1:], w)[0])

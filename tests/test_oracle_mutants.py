@@ -17,7 +17,7 @@ import pytest
 import oracle
 from oracle import build as oracle_build
 
-from test_oracle import GOLDEN, _num, sink_index, textbook
+from test_oracle import GOLDEN, OPROJ_GOLDEN, _num, sink_index, textbook
 
 MUTANTS = {
     "no_softmax_scale": ("const double scale = 1.0 / sqrt((double)d);",
@@ -32,6 +32,11 @@ MUTANTS = {
     "norm_of_spec": ("den += o_exact[i] * o_exact[i];", "den += o_spec[i] * o_spec[i];"),
     "no_normalisation": ("double p = scores[j] / z;", "double p = scores[j];"),
     "no_max_subtraction": ("scores[j] = exp(scores[j] - m);", "scores[j] = exp(scores[j]);"),
+    "oproj_transposed_weight": ("load_elem(w, w_dtype, (size_t)j * K + i)",
+                                "load_elem(w, w_dtype, (size_t)i * N + j)"),
+    "oproj_drops_last_term": ("for (int i = 0; i < K; ++i) {", "for (int i = 0; i < K - 1; ++i) {"),
+    "oproj_gate_inverted": ("const double* x = commit[b] ? o_spec + (size_t)b * K : o_exact + (size_t)b * K;",
+                            "const double* x = commit[b] ? o_exact + (size_t)b * K : o_spec + (size_t)b * K;"),
 }
 
 
@@ -86,6 +91,18 @@ def _pins_pass(lib):
         k2 = k + 900.0 * math.sqrt(d) * q / (q @ q)
         o_s2, o_e2 = oracle.head(q, k2, v, S, W, lib=lib)
         if not (np.allclose(o_e2, o_e, atol=1e-9) and np.allclose(o_s2, o_s, atol=1e-9)):
+            return False
+        # Output projection: hand cases (non-square, gated, bf16 weights).
+        with open(OPROJ_GOLDEN) as f:
+            pc = {c["name"]: c for c in json.load(f)["cases"]}
+        a = pc["non_square_two_tokens"]
+        if not np.array_equal(oracle.oproj(np.array(a["x"]), np.array(a["w"], np.float32),
+                                           lib=lib), np.array(a["y"])):
+            return False
+        g = pc["gated_one_commit_one_discard"]
+        if not np.array_equal(oracle.oproj_gated(g["o_spec"], g["o_exact"], g["commit"],
+                                                 np.array(g["w"], np.float64), lib=lib),
+                              np.array(g["y"])):
             return False
     except (ValueError, FloatingPointError):
         return False
