@@ -50,6 +50,8 @@ def parse_args():
     ap.add_argument("--split-tokens", type=int, default=0,
                     help="exact-path item size for the longest sequence (0 = library's choice)")
     ap.add_argument("--engine", default="auto", choices=["auto", "cuda_cores", "tensor_cores"])
+    ap.add_argument("--oproj", action="store_true",
+                    help="speculative output projection against the serial one (32 x 128K)")
     ap.add_argument("--lambda-sweep", action="store_true",
                     help="hit rate against the threshold on the commit-mixing workload family")
     return ap.parse_args()
@@ -590,12 +592,127 @@ def run_lambda_sweep(args):
     print(json.dumps(line), flush=True)
 
 
+def run_oproj_bench(args):
+    """Latency the speculative output projection hides.  Per layer of the
+    32 x 128K step, the projection after attention (Llama-3.1-8B o_proj:
+    4096 x 4096 bf16 weights, synthetic) is either run after the merge on
+    O_exact (serial) or run on O_spec beside the exact path and redone on
+    O_exact only for discarded tokens (speculative: gated by a kernel that
+    reads the flags, or by a conditional graph node).  The steps are CUDA
+    graphs of 32 layers, each layer after the previous one's projection;
+    timed with events, warm-up first.  Two data
+    sets: the workload as specified (every token discarded) and the same
+    shape with strong sinks and no needles (tokens commit)."""
+    import torch
+    import workloads
+    import speculative_flash_decoding_b200 as sfd
+    rank, world, local = dist_env()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    base = workloads.CONFIGS[2]
+    n_layers = args.layers or base.n_layers
+    hidden = 4096
+    g = torch.Generator(device="cpu").manual_seed(4242)
+    weights = [(torch.randn(hidden, base.Hq * base.d, generator=g) / 64.0).to(torch.bfloat16)
+               .to(device) for _ in range(n_layers)]
+    results = {}
+    # The projection alone: 32 back-to-back calls (one per layer's weights),
+    # 32 MB of weights each, larger than L2 together.
+    x = torch.randn(base.B, base.Hq * base.d, device=device)
+    y = torch.empty(base.B, hidden, device=device)
+    st = torch.cuda.Stream(device)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    with torch.cuda.stream(st):
+        for rep in range(4):
+            if rep == 3:
+                ev[0].record(st)
+            for w in weights:
+                assert sfd.alspec_oproj(x.data_ptr(), w.data_ptr(), y.data_ptr(), 0, base.B,
+                                        base.Hq * base.d, hidden, st.cuda_stream) == 0
+        ev[1].record(st)
+    st.synchronize()
+    us = ev[0].elapsed_time(ev[1]) * 1e3 / n_layers
+    w_bytes = hidden * base.Hq * base.d * 2
+    peak, peak_kind = measured_peak()
+    results["oproj_alone"] = {"us_per_call": us, "weight_bytes": w_bytes,
+                              "gbs": w_bytes / (us * 1e-6) / 1e9,
+                              "frac_of_hbm_peak": w_bytes / (us * 1e-6) / 1e9 / peak,
+                              "peak_kind": peak_kind}
+    for tag, wl in (("as_specified", base),
+                    ("strong_sinks_no_needles", base.replace(sink_bump=24.0, needles=("none",)))):
+        layers = [workloads.make_layer(wl, layer=i, device=device) for i in range(n_layers)]
+        dec = sfd.Decoder(wl.B, wl.Hq, wl.Hkv, wl.d, wl.L, wl.dtype, wl.S, wl.W, device=device)
+        outs = []
+        for _ in range(n_layers):
+            o = dec.alloc_outputs()
+            o["y"] = torch.empty(wl.B, hidden, device=device)
+            outs.append(o)
+        stream = torch.cuda.Stream(device)
+        kdim = wl.Hq * wl.d
+        with torch.cuda.stream(stream):
+            for d, o in zip(layers, outs):   # creates the library's stream and events
+                dec.decode(d["q"], d["k"], d["v"], d["seq_lens"], wl.lam, out=o, stream=stream)
+        stream.synchronize()
+
+        def capture(speculative):
+            with torch.cuda.stream(stream):
+                assert sfd.alspec_graph_begin(stream.cuda_stream) == 0
+                for d, o, w in zip(layers, outs, weights):
+                    if speculative:
+                        dec.decode_oproj(d["q"], d["k"], d["v"], d["seq_lens"], wl.lam, w,
+                                         out=o, stream=stream, gate=speculative)
+                    else:
+                        dec.decode(d["q"], d["k"], d["v"], d["seq_lens"], wl.lam, out=o,
+                                   stream=stream)
+                        assert sfd.alspec_oproj(o["out_exact"].data_ptr(), w.data_ptr(),
+                                                o["y"].data_ptr(), 0, wl.B, kdim, hidden,
+                                                stream.cuda_stream) == 0
+                st, gr = sfd.alspec_graph_end(stream.cuda_stream)
+                assert st == 0
+            return gr
+
+        res = {}
+        for name, spec in (("serial", False), ("speculative", "kernel"),
+                           ("speculative_graph_conditional", "graph_conditional")):
+            gr = capture(spec)
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+            with torch.cuda.stream(stream):
+                for _ in range(max(3, args.warmup)):
+                    assert sfd.alspec_graph_launch(gr, stream.cuda_stream) == 0
+                ev[0].record(stream)
+                for _ in range(args.steps):
+                    assert sfd.alspec_graph_launch(gr, stream.cuda_stream) == 0
+                ev[1].record(stream)
+            stream.synchronize()
+            ms = ev[0].elapsed_time(ev[1]) / args.steps
+            res[name] = {"us_per_step": ms * 1e3, "us_per_layer": ms * 1e3 / n_layers}
+            hit = float(torch.stack([o["commit"].float().mean() for o in outs]).mean().item())
+            assert sfd.alspec_graph_destroy(gr) == 0
+        res["hit_rate"] = hit
+        res["hidden_us_per_layer"] = (res["serial"]["us_per_layer"] -
+                                      res["speculative"]["us_per_layer"])
+        results[tag] = res
+        del layers, outs
+        torch.cuda.empty_cache()
+    if rank != 0:
+        return
+    line = {"metric": "per-layer latency to the output projection's result, serial vs "
+                      "speculative", "unit": "us", "higher_is_better": False,
+            "steps": args.steps, "data": "synthetic",
+            "config": {"workload": base.name, "layers": n_layers, "hidden": hidden,
+                       "weights": "bf16 [4096, 4096] per layer, N(0, 1/64^2)"},
+            "results": results}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse_args()
     import workloads
     wl = workloads.CONFIGS[args.config]
     if args.lambda_sweep:
         run_lambda_sweep(args)
+    elif args.oproj:
+        run_oproj_bench(args)
     elif args.impl == "reference":
         run_reference(args, wl)
     else:

@@ -19,9 +19,9 @@
  * Conventions for every entry point:
  *   - Pointers named "device" are CUDA device pointers; "host" pointers are
  *     ordinary host memory.  The caller owns every buffer.  The library never
- *     allocates device memory in alspec_decode; it owns only one
- *     high-priority stream and two events per device, created on first use
- *     and released by alspec_shutdown().
+ *     allocates device memory in alspec_decode; it owns only a
+ *     high-priority stream, a lowest-priority stream and three events per
+ *     device, created on first use and released by alspec_shutdown().
  *   - Streams and events are passed as `void*` holding a cudaStream_t /
  *     cudaEvent_t (NULL stream = the legacy default stream).
  *   - Calls are asynchronous on the given stream unless stated otherwise;
@@ -61,6 +61,12 @@ typedef enum {
     ALSPEC_ENGINE_CUDA_CORES = 1,    /* packed fp32 FMAs; any dtype               */
     ALSPEC_ENGINE_TENSOR_CORES = 2   /* bf16 m16n8k16 MMAs; bf16 only             */
 } alspec_engine;
+
+/* Gating of the recomputation in alspec_decode_oproj. */
+typedef enum {
+    ALSPEC_GATE_KERNEL = 0,             /* a kernel that reads the flags           */
+    ALSPEC_GATE_GRAPH_CONDITIONAL = 1   /* a CUDA-graph IF node (inside a capture) */
+} alspec_gate;
 
 /* Number of events alspec_decode's prof_events array holds. */
 #define ALSPEC_PROF_EVENTS 5
@@ -186,17 +192,20 @@ alspec_status alspec_decode_traced(const alspec_desc* desc,
  * self-attention in a decoder layer (the post-attention op the pages run
  * speculatively, "Approach"):
  *     y[b, j] = sum_i x[b, i] * w[j, i]
- * on CUDA cores (decode batches are small: the op streams w once).
+ * on CUDA cores (decode batches are small: the op streams w once, with bulk
+ * copies, one CTA per SM).
  *   x     device fp32 [batch][k], 16-byte aligned
  *   w     device bf16 [n][k] (row j = output feature j), 16-byte aligned
  *   y     device fp32 [batch][n]
  *   skip  device uint8 [batch] or NULL: rows b with skip[b] != 0 are not
  *         written (pass the commit flags to redo only discarded tokens)
+ *   err   device uint32 or NULL: ALSPEC_DEVERR_TIMEOUT is ORed in when one of
+ *         the kernel's bounded waits (2 s) expires (y is then incomplete)
  *   batch 1..8; k a positive multiple of 8; n >= 1.
  * Asynchronous on `stream`; ALSPEC_ERR_INVALID_ARG for a bad argument.
  */
 alspec_status alspec_oproj(const float* x, const void* w, float* y, const uint8_t* skip,
-                           int batch, int k, int n, void* stream);
+                           int batch, int k, int n, uint32_t* err, void* stream);
 
 /*
  * alspec_decode followed by the output projection of the attention output,
@@ -204,14 +213,22 @@ alspec_status alspec_oproj(const float* x, const void* w, float* y, const uint8_
  * post-attention ops with commit or discard, "Approach"):
  *   y[b] = o_proj(commit[b] ? O_spec[b] : O_exact[b]),  o_proj as in
  *   alspec_oproj with w_o bf16 [hidden][n_q_heads * head_dim].
- * The projection of O_spec runs on the high-priority stream right after the
- * sink-set kernel, beside the exact path; after the merge, the projection of
- * O_exact overwrites the rows of discarded tokens.  Inside a stream capture
- * that recomputation is a conditional node of the graph which the merge
- * kernel enables only when it discards a token; outside a capture it is
- * launched and skips committed rows.  With every token committed, y is
- * final when the flags are, instead of one projection later.
+ * The projection of O_spec runs right after the sink-set kernel, beside the
+ * exact path, on the library's lowest-priority stream (a form without shared
+ * memory, which shares SMs with the middle kernel).  After the merge, the
+ * projection of O_exact (the bulk-copy form of alspec_oproj) overwrites the
+ * rows of discarded tokens.  With every token committed, y is final when the
+ * flags are, instead of one projection later.  Wait timeouts go to the
+ * workspace's device error word.
  *   y        device fp32 [batch][hidden]; batch <= 8
+ *   gate     how the recomputation is gated (alspec_gate):
+ *            ALSPEC_GATE_KERNEL: it is always launched and reads the flags
+ *            (it exits at once when every token committed);
+ *            ALSPEC_GATE_GRAPH_CONDITIONAL: inside a stream capture it is an
+ *            IF conditional node of the graph, which the merge kernel enables
+ *            when it discards a token (outside a capture as GATE_KERNEL).
+ *            Evaluating the conditional node was measured at ~7 us per layer
+ *            on B200, more than the kernel launch it saves.
  *   trace_ns NULL, or device 3 x uint64 zeroed by the caller: [0] and [1] as
  *            in alspec_decode_traced, [2] raised to the global timer after
  *            each projection's last write (y is final at max([1], [2])).
@@ -223,7 +240,7 @@ alspec_status alspec_decode_oproj(const alspec_desc* desc,
                                   const int32_t* seq_lens, int n_sink, int window,
                                   float lambda, const void* w_o, int hidden,
                                   float* out_spec, float* out_exact, float* rel_l2,
-                                  uint8_t* commit, float* y,
+                                  uint8_t* commit, float* y, int gate,
                                   void* workspace, size_t workspace_bytes,
                                   void* stream, unsigned long long* trace_ns);
 

@@ -72,9 +72,9 @@ SIGNATURES = {
                                    _vp]),
     "alspec_decode_traced": (_i, [_descp, _vp, _vp, _vp, _vp, _i, _i, _f, _vp, _vp, _vp, _vp,
                                   _vp, _sz, _vp, _vp]),
-    "alspec_oproj": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _vp]),
+    "alspec_oproj": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp]),
     "alspec_decode_oproj": (_i, [_descp, _vp, _vp, _vp, _vp, _i, _i, _f, _vp, _i, _vp, _vp,
-                                 _vp, _vp, _vp, _vp, _sz, _vp, _vp]),
+                                 _vp, _vp, _vp, _i, _vp, _sz, _vp, _vp]),
 }
 
 ALSPEC_NOALLOC_SCRATCH_BYTES = 8 << 20
@@ -141,21 +141,26 @@ def alspec_decode_traced(desc: alspec_desc, q: int, k_cache: int, v_cache: int, 
 
 
 def alspec_oproj(x: int, w: int, y: int, skip: int, batch: int, k: int, n: int,
-                 stream: int) -> int:
-    """y[b, j] = sum_i x[b, i] * w[j, i]; rows with skip[b] != 0 untouched."""
-    return int(_lib.alspec_oproj(x, w, y, skip or None, batch, k, n, stream))
+                 stream: int, err: int = 0) -> int:
+    """y[b, j] = sum_i x[b, i] * w[j, i]; rows with skip[b] != 0 untouched;
+    err: device address of a uint32 error word, or 0."""
+    return int(_lib.alspec_oproj(x, w, y, skip or None, batch, k, n, err or None, stream))
+
+
+ALSPEC_GATE_KERNEL, ALSPEC_GATE_GRAPH_CONDITIONAL = 0, 1
+GATES = {"kernel": ALSPEC_GATE_KERNEL, "graph_conditional": ALSPEC_GATE_GRAPH_CONDITIONAL}
 
 
 def alspec_decode_oproj(desc: alspec_desc, q: int, k_cache: int, v_cache: int, seq_lens: int,
                         n_sink: int, window: int, lam: float, w_o: int, hidden: int,
                         out_spec: int, out_exact: int, rel_l2: int, commit: int, y: int,
-                        workspace: int, workspace_bytes: int, stream: int,
+                        gate: int, workspace: int, workspace_bytes: int, stream: int,
                         trace_ns: int = 0) -> int:
     """Decode plus the speculative output projection y = o_proj(O_spec or O_exact)."""
     return int(_lib.alspec_decode_oproj(ctypes.byref(desc), q, k_cache, v_cache, seq_lens,
                                         n_sink, window, lam, w_o, hidden, out_spec, out_exact,
-                                        rel_l2, commit, y, workspace, workspace_bytes, stream,
-                                        trace_ns or None))
+                                        rel_l2, commit, y, gate, workspace, workspace_bytes,
+                                        stream, trace_ns or None))
 
 
 def alspec_decode_noalloc(desc: alspec_desc, q: int, k_cache: int, v_cache: int, seq_lens: int,
@@ -316,10 +321,12 @@ class Decoder:
         _check(st, "alspec_decode")
         return out
 
-    def decode_oproj(self, q, k, v, seq_lens, lam, w_o, out=None, stream=None, trace=None):
+    def decode_oproj(self, q, k, v, seq_lens, lam, w_o, out=None, stream=None, trace=None,
+                     gate="kernel"):
         """decode() plus y = o_proj(commit ? O_spec : O_exact) with w_o bf16
         [hidden, Hq * d]; out gains "y" (fp32 [B, hidden]).  trace: None or
-        a zeroed int64 device tensor of 3 elements."""
+        a zeroed int64 device tensor of 3 elements; gate: "kernel" or
+        "graph_conditional"."""
         t = self.torch
         out = out if out is not None else self.alloc_outputs()
         hidden = int(w_o.shape[0])
@@ -330,7 +337,7 @@ class Decoder:
                                  seq_lens.data_ptr(), self.n_sink, self.window, float(lam),
                                  w_o.data_ptr(), hidden, out["out_spec"].data_ptr(),
                                  out["out_exact"].data_ptr(), out["rel_l2"].data_ptr(),
-                                 out["commit"].data_ptr(), out["y"].data_ptr(),
+                                 out["commit"].data_ptr(), out["y"].data_ptr(), GATES[gate],
                                  self.workspace.data_ptr(), self.workspace_bytes, s.cuda_stream,
                                  trace.data_ptr() if trace is not None else 0)
         _check(st, "alspec_decode_oproj")

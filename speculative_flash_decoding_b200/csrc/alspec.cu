@@ -62,6 +62,7 @@ int round_up(int a, int b) { return ceil_div(a, b) * b; }
 struct DeviceState {
     bool ready = false;
     cudaStream_t hi = nullptr;
+    cudaStream_t lo = nullptr;    // lowest priority: speculative post-attention work
     cudaEvent_t fork = nullptr;
     cudaEvent_t join = nullptr;
     cudaEvent_t join2 = nullptr;  // after the speculative output projection
@@ -83,6 +84,7 @@ alspec_status get_device_state(DeviceState** out) {
         if (!ok(cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev)) ||
             !ok(cudaDeviceGetStreamPriorityRange(&lo, &hi)) ||
             !ok(cudaStreamCreateWithPriority(&d.hi, cudaStreamNonBlocking, hi)) ||
+            !ok(cudaStreamCreateWithPriority(&d.lo, cudaStreamNonBlocking, lo)) ||
             !ok(cudaEventCreateWithFlags(&d.fork, cudaEventDisableTiming)) ||
             !ok(cudaEventCreateWithFlags(&d.join, cudaEventDisableTiming)) ||
             !ok(cudaEventCreateWithFlags(&d.join2, cudaEventDisableTiming))) {
@@ -322,12 +324,10 @@ alspec_status encode_kv_map(CUtensorMap* map, const void* base, const alspec_des
     return r == CUDA_SUCCESS ? ALSPEC_OK : ALSPEC_ERR_INVALID_ARG;
 }
 
-alspec_status ensure_smem_attr(DeviceState* ds, KernelFn fn, int bytes) {
+alspec_status ensure_smem_attr(DeviceState* ds, const void* key, int bytes) {
     std::lock_guard<std::mutex> lock(g_mutex);
-    const void* key = reinterpret_cast<const void*>(fn);
     if (ds->attr_done.count(key)) return ALSPEC_OK;
-    if (!ok(cudaFuncSetAttribute(reinterpret_cast<const void*>(fn),
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, bytes)))
+    if (!ok(cudaFuncSetAttribute(key, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes)))
         return ALSPEC_ERR_CUDA;
     ds->attr_done.insert(key);
     return ALSPEC_OK;
@@ -430,6 +430,7 @@ struct OprojReq {
     const void* w;  // bf16 [hidden][Hq * d]
     int hidden;
     float* y;       // fp32 [B][hidden]
+    int gate;       // alspec_gate
 };
 
 bool oproj_args_ok(const float* x, const void* w, const float* y, int batch, int k, int n) {
@@ -438,8 +439,11 @@ bool oproj_args_ok(const float* x, const void* w, const float* y, int batch, int
 }
 
 OprojParams oproj_params(const float* x, const void* w, float* y, const uint8_t* skip, int batch,
-                         int k, int n, unsigned long long* trace) {
+                         int k, int n, unsigned long long* trace, unsigned* err = nullptr,
+                         unsigned long long timeout_ns = 2000000000ull) {
     OprojParams o{};
+    o.err = err;
+    o.timeout_ns = timeout_ns;
     o.x = x;
     o.w = static_cast<const uint4*>(w);
     o.y = y;
@@ -451,7 +455,17 @@ OprojParams oproj_params(const float* x, const void* w, float* y, const uint8_t*
     return o;
 }
 
-dim3 oproj_grid(int n) { return dim3((unsigned)ceil_div(n, kOprojWarps * kOprojRows)); }
+dim3 oproj_grid(int n) { return dim3((unsigned)ceil_div(n, kOprojWarps)); }
+
+// Foreground projection: the bulk-copy kernel, one CTA per SM (at most one
+// per output row).
+alspec_status launch_oproj_bulk(DeviceState* ds, const OprojParams& o, cudaStream_t s) {
+    const OprojFn fn = oproj_bulk_kernel_for(o.B);
+    alspec_status st = ensure_smem_attr(ds, reinterpret_cast<const void*>(fn), kObSmem);
+    if (st != ALSPEC_OK) return st;
+    fn<<<std::min(ds->sm_count, o.N), kObThreads, kObSmem, s>>>(o);
+    return ok(cudaGetLastError()) ? ALSPEC_OK : ALSPEC_ERR_CUDA;
+}
 
 alspec_status decode_impl(const alspec_desc* desc, const void* q, const void* k_cache,
                           const void* v_cache, const int32_t* seq_lens, int n_sink, int window,
@@ -477,8 +491,12 @@ alspec_status decode_impl(const alspec_desc* desc, const void* q, const void* k_
     const int G = desc->n_q_heads / desc->n_kv_heads;
     KernelSet ks{};
     if (!pick(desc->dtype, desc->head_dim, G, pl.engine, &ks)) return ALSPEC_ERR_UNSUPPORTED;
-    if ((st = ensure_smem_attr(ds, ks.spec, ks.smem_spec)) != ALSPEC_OK) return st;
-    if ((st = ensure_smem_attr(ds, ks.mid, ks.smem_mid)) != ALSPEC_OK) return st;
+    if ((st = ensure_smem_attr(ds, reinterpret_cast<const void*>(ks.spec), ks.smem_spec)) !=
+        ALSPEC_OK)
+        return st;
+    if ((st = ensure_smem_attr(ds, reinterpret_cast<const void*>(ks.mid), ks.smem_mid)) !=
+        ALSPEC_OK)
+        return st;
 
     char* ws = static_cast<char*>(workspace);
     Params p{};
@@ -534,11 +552,15 @@ alspec_status decode_impl(const alspec_desc* desc, const void* q, const void* k_
     if (!ok(cudaEventRecord(ds->join, ds->hi))) return ALSPEC_ERR_CUDA;
     const int kdim = desc->n_q_heads * desc->head_dim;
     if (op) {
-        // Speculative output projection of O_spec, beside the exact path.
+        // Speculative output projection of O_spec, beside the exact path, on
+        // the lowest-priority stream: it has until the merge to finish, and
+        // the middle kernel's CTAs come first.
         const OprojParams o = oproj_params(out_spec, op->w, op->y, nullptr, desc->batch, kdim,
-                                           op->hidden, trace_ns ? trace_ns + 2 : nullptr);
-        oproj_kernel<<<oproj_grid(op->hidden), kOprojWarps * 32, 0, ds->hi>>>(o);
-        if (!ok(cudaGetLastError()) || !ok(cudaEventRecord(ds->join2, ds->hi)))
+                                           op->hidden, trace_ns ? trace_ns + 2 : nullptr,
+                                           p.ctr + kCtrError, p.timeout_ns);
+        if (!ok(cudaStreamWaitEvent(ds->lo, ds->join, 0))) return ALSPEC_ERR_CUDA;
+        oproj_kernel_for(o.B)<<<oproj_grid(op->hidden), kOprojWarps * 32, 0, ds->lo>>>(o);
+        if (!ok(cudaGetLastError()) || !ok(cudaEventRecord(ds->join2, ds->lo)))
             return ALSPEC_ERR_CUDA;
     }
 #ifdef ALSPEC_SPEC_SERIAL
@@ -559,12 +581,12 @@ alspec_status decode_impl(const alspec_desc* desc, const void* q, const void* k_
         mk = pl.tt == 32 ? merge_kernel<128, 32> : merge_kernel<128, 16>;
     else
         mk = pl.tt == 32 ? merge_kernel<64, 32> : merge_kernel<64, 16>;
-    // Inside a stream capture the recomputation of discarded tokens' output
-    // projection is a conditional node: the merge kernel sets its condition
-    // when it discards a token.
+    // With ALSPEC_GATE_GRAPH_CONDITIONAL, inside a stream capture the
+    // recomputation of discarded tokens' output projection is a conditional
+    // node: the merge kernel sets its condition when it discards a token.
     bool capturing = false;
     cudaGraphConditionalHandle cond = 0;
-    if (op) {
+    if (op && op->gate == ALSPEC_GATE_GRAPH_CONDITIONAL) {
         cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
         cudaGraph_t cg = nullptr;
         if (!ok(cudaStreamGetCaptureInfo(s, &cs, nullptr, &cg, nullptr, nullptr)))
@@ -589,7 +611,11 @@ alspec_status decode_impl(const alspec_desc* desc, const void* q, const void* k_
         // speculative one (both write y).
         if (!ok(cudaStreamWaitEvent(s, ds->join2, 0))) return ALSPEC_ERR_CUDA;
         OprojParams r = oproj_params(out_exact, op->w, op->y, commit, desc->batch, kdim,
-                                     op->hidden, trace_ns ? trace_ns + 2 : nullptr);
+                                     op->hidden, trace_ns ? trace_ns + 2 : nullptr,
+                                     p.ctr + kCtrError, p.timeout_ns);
+        const OprojFn rfn = oproj_bulk_kernel_for(r.B);
+        if ((st = ensure_smem_attr(ds, reinterpret_cast<const void*>(rfn), kObSmem)) != ALSPEC_OK)
+            return st;
         if (capturing) {
             cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
             cudaGraph_t g = nullptr;
@@ -606,10 +632,10 @@ alspec_status decode_impl(const alspec_desc* desc, const void* q, const void* k_
             if (!ok(cudaGraphAddNode(&cn, g, deps, ndeps, &cp))) return ALSPEC_ERR_CUDA;
             cudaGraphNodeParams kp{};
             kp.type = cudaGraphNodeTypeKernel;
-            kp.kernel.func = reinterpret_cast<void*>(oproj_kernel);
-            kp.kernel.gridDim = oproj_grid(op->hidden);
-            kp.kernel.blockDim = dim3(kOprojWarps * 32);
-            kp.kernel.sharedMemBytes = 0;
+            kp.kernel.func = reinterpret_cast<void*>(rfn);
+            kp.kernel.gridDim = dim3((unsigned)std::min(ds->sm_count, op->hidden));
+            kp.kernel.blockDim = dim3(kObThreads);
+            kp.kernel.sharedMemBytes = kObSmem;
             void* args[] = {&r};
             kp.kernel.kernelParams = args;
             cudaGraphNode_t kn = nullptr;
@@ -618,8 +644,7 @@ alspec_status decode_impl(const alspec_desc* desc, const void* q, const void* k_
                                                         cudaStreamSetCaptureDependencies)))
                 return ALSPEC_ERR_CUDA;
         } else {
-            oproj_kernel<<<oproj_grid(op->hidden), kOprojWarps * 32, 0, s>>>(r);
-            if (!ok(cudaGetLastError())) return ALSPEC_ERR_CUDA;
+            if ((st = launch_oproj_bulk(ds, r, s)) != ALSPEC_OK) return st;
         }
     }
     if (!prof(4, s)) return ALSPEC_ERR_CUDA;
@@ -654,18 +679,21 @@ alspec_status alspec_decode_traced(const alspec_desc* desc, const void* q, const
 }
 
 alspec_status alspec_oproj(const float* x, const void* w, float* y, const uint8_t* skip, int batch,
-                           int k, int n, void* stream) {
-    if (!oproj_args_ok(x, w, y, batch, k, n)) return ALSPEC_ERR_INVALID_ARG;
-    const OprojParams o = oproj_params(x, w, y, skip, batch, k, n, nullptr);
-    oproj_kernel<<<oproj_grid(n), kOprojWarps * 32, 0, static_cast<cudaStream_t>(stream)>>>(o);
-    return ok(cudaGetLastError()) ? ALSPEC_OK : ALSPEC_ERR_CUDA;
+                           int k, int n, uint32_t* err, void* stream) {
+    if (!oproj_args_ok(x, w, y, batch, k, n) || (reinterpret_cast<uintptr_t>(err) & 3u))
+        return ALSPEC_ERR_INVALID_ARG;
+    DeviceState* ds = nullptr;
+    alspec_status st = get_device_state(&ds);
+    if (st != ALSPEC_OK) return st;
+    const OprojParams o = oproj_params(x, w, y, skip, batch, k, n, nullptr, err);
+    return launch_oproj_bulk(ds, o, static_cast<cudaStream_t>(stream));
 }
 
 alspec_status alspec_decode_oproj(const alspec_desc* desc, const void* q, const void* k_cache,
                                   const void* v_cache, const int32_t* seq_lens, int n_sink,
                                   int window, float lambda, const void* w_o, int hidden,
                                   float* out_spec, float* out_exact, float* rel_l2,
-                                  uint8_t* commit, float* y, void* workspace,
+                                  uint8_t* commit, float* y, int gate, void* workspace,
                                   size_t workspace_bytes, void* stream,
                                   unsigned long long* trace_ns) {
     if (!desc) return ALSPEC_ERR_INVALID_ARG;
@@ -673,7 +701,9 @@ alspec_status alspec_decode_oproj(const alspec_desc* desc, const void* q, const 
     if (!oproj_args_ok(out_spec, w_o, y, desc->batch, kdim, hidden) || !out_exact ||
         !aligned16(out_exact))
         return ALSPEC_ERR_INVALID_ARG;
-    const OprojReq op{w_o, hidden, y};
+    if (gate != ALSPEC_GATE_KERNEL && gate != ALSPEC_GATE_GRAPH_CONDITIONAL)
+        return ALSPEC_ERR_INVALID_ARG;
+    const OprojReq op{w_o, hidden, y, gate};
     return decode_impl(desc, q, k_cache, v_cache, seq_lens, n_sink, window, lambda, out_spec,
                        out_exact, rel_l2, commit, workspace, workspace_bytes, stream, nullptr,
                        nullptr, trace_ns, &op);
@@ -748,6 +778,7 @@ alspec_status alspec_shutdown(void) {
         cudaEventDestroy(s.join);
         if (s.join2) cudaEventDestroy(s.join2);
         cudaStreamDestroy(s.hi);
+        if (s.lo) cudaStreamDestroy(s.lo);
         s = DeviceState{};
     }
     if (have_cur) cudaSetDevice(cur);

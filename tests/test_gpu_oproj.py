@@ -49,13 +49,13 @@ def test_oproj_matches_oracle(cuda_device, B, K, N):
             assert torch.equal(y2[b], y[b])
 
 
-def _pipeline(wl, data, w, lam, device, graph=False):
+def _pipeline(wl, data, w, lam, device, graph=False, gate="kernel"):
     import speculative_flash_decoding_b200 as sfd
     dec = sfd.Decoder(wl.B, wl.Hq, wl.Hkv, wl.d, wl.L, wl.dtype, wl.S, wl.W, device=device)
     trace = torch.zeros(3, dtype=torch.int64, device=device)
     if not graph:
         out = dec.decode_oproj(data["q"], data["k"], data["v"], data["seq_lens"], lam, w,
-                               trace=trace)
+                               trace=trace, gate=gate)
         torch.cuda.synchronize()
         return {k: v.cpu() for k, v in out.items()}, trace.cpu().numpy()
     # A first call outside the capture creates the library's stream and events.
@@ -67,7 +67,7 @@ def _pipeline(wl, data, w, lam, device, graph=False):
     with torch.cuda.stream(stream):
         assert sfd.alspec_graph_begin(stream.cuda_stream) == 0
         dec.decode_oproj(data["q"], data["k"], data["v"], data["seq_lens"], lam, w, out=out,
-                         stream=stream, trace=trace)
+                         stream=stream, trace=trace, gate=gate)
         st, g = sfd.alspec_graph_end(stream.cuda_stream)
         assert st == 0 and g
         for _ in range(2):
@@ -79,16 +79,17 @@ def _pipeline(wl, data, w, lam, device, graph=False):
     return {k: v.cpu() for k, v in out.items()}, trace.cpu().numpy()
 
 
-@pytest.mark.parametrize("graph", [False, True])
+@pytest.mark.parametrize("graph,gate", [(False, "kernel"), (True, "kernel"),
+                                        (True, "graph_conditional")])
 @pytest.mark.parametrize("lam", [0.1, 1.0])
-def test_speculative_projection_with_gating(cuda_device, graph, lam):
+def test_speculative_projection_with_gating(cuda_device, graph, gate, lam):
     """y = o_proj(commit ? O_spec : O_exact): against the oracle's chain, and
     exactly the projection of the device's own O_spec / O_exact rows."""
     wl = workloads.COMMIT_VARIANT.replace(L=8192, ragged=(6000, 8192))
     data = workloads.make_layer(wl, device=cuda_device)
     hidden = 1000
     w = _bf16_weights(hidden, wl.Hq * wl.d, 99, cuda_device)
-    out, tr = _pipeline(wl, data, w, lam, cuda_device, graph=graph)
+    out, tr = _pipeline(wl, data, w, lam, cuda_device, graph=graph, gate=gate)
     commit = out["commit"].numpy()
     if lam == 1.0:
         assert commit.all()
@@ -110,13 +111,14 @@ def test_speculative_projection_with_gating(cuda_device, graph, lam):
     assert tr[0] > 0 and tr[1] > tr[0] and tr[2] > 0
 
 
-def test_graph_with_all_committed_skips_the_recomputation(cuda_device):
-    """With every token committed the conditional body does not run: y is the
+@pytest.mark.parametrize("gate", ["kernel", "graph_conditional"])
+def test_graph_with_all_committed_skips_the_recomputation(cuda_device, gate):
+    """With every token committed the recomputation writes nothing: y is the
     projection of O_spec (bit-identical to the eager result)."""
     wl = workloads.COMMIT_VARIANT.replace(L=8192, ragged=(6000, 8192))
     data = workloads.make_layer(wl, device=cuda_device)
     w = _bf16_weights(512, wl.Hq * wl.d, 5, cuda_device)
     eager, _ = _pipeline(wl, data, w, 1.0, cuda_device)
-    graph, _ = _pipeline(wl, data, w, 1.0, cuda_device, graph=True)
+    graph, _ = _pipeline(wl, data, w, 1.0, cuda_device, graph=True, gate=gate)
     for k in ("out_spec", "out_exact", "rel_l2", "commit", "y"):
         assert torch.equal(eager[k], graph[k]), k
