@@ -225,8 +225,9 @@ alspec_status alspec_oproj(const float* x, const void* w, float* y, const uint8_
  *            ALSPEC_GATE_KERNEL: it is always launched and reads the flags
  *            (it exits at once when every token committed);
  *            ALSPEC_GATE_GRAPH_CONDITIONAL: inside a stream capture it is an
- *            IF conditional node of the graph, which the merge kernel enables
- *            when it discards a token (outside a capture as GATE_KERNEL).
+ *            IF conditional node of the graph, enabled by a one-warp kernel
+ *            after the merge when a token was discarded (outside a capture
+ *            as GATE_KERNEL).
  *            Evaluating the conditional node was measured at ~7 us per layer
  *            on B200, more than the kernel launch it saves.
  *   trace_ns NULL, or device 3 x uint64 zeroed by the caller: [0] and [1] as

@@ -583,7 +583,7 @@ alspec_status decode_impl(const alspec_desc* desc, const void* q, const void* k_
         mk = pl.tt == 32 ? merge_kernel<64, 32> : merge_kernel<64, 16>;
     // With ALSPEC_GATE_GRAPH_CONDITIONAL, inside a stream capture the
     // recomputation of discarded tokens' output projection is a conditional
-    // node: the merge kernel sets its condition when it discards a token.
+    // node, enabled by a one-warp kernel that reads the flags.
     bool capturing = false;
     cudaGraphConditionalHandle cond = 0;
     if (op && op->gate == ALSPEC_GATE_GRAPH_CONDITIONAL) {
@@ -592,12 +592,9 @@ alspec_status decode_impl(const alspec_desc* desc, const void* q, const void* k_
         if (!ok(cudaStreamGetCaptureInfo(s, &cs, nullptr, &cg, nullptr, nullptr)))
             return ALSPEC_ERR_CUDA;
         capturing = cs == cudaStreamCaptureStatusActive;
-        if (capturing) {
-            if (!ok(cudaGraphConditionalHandleCreate(&cond, cg, 0, cudaGraphCondAssignDefault)))
-                return ALSPEC_ERR_CUDA;
-            p.cond = static_cast<unsigned long long>(cond);
-            p.cond_on = 1;
-        }
+        if (capturing &&
+            !ok(cudaGraphConditionalHandleCreate(&cond, cg, 0, cudaGraphCondAssignDefault)))
+            return ALSPEC_ERR_CUDA;
     }
     // Programmatic launch right behind the middle kernel (when there is one
     // and no profiling event sits between them).
@@ -617,6 +614,8 @@ alspec_status decode_impl(const alspec_desc* desc, const void* q, const void* k_
         if ((st = ensure_smem_attr(ds, reinterpret_cast<const void*>(rfn), kObSmem)) != ALSPEC_OK)
             return st;
         if (capturing) {
+            set_discard_condition<<<1, 32, 0, s>>>(commit, desc->batch, cond);
+            if (!ok(cudaGetLastError())) return ALSPEC_ERR_CUDA;
             cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
             cudaGraph_t g = nullptr;
             const cudaGraphNode_t* deps = nullptr;

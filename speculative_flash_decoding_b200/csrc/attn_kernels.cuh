@@ -47,7 +47,6 @@
 #pragma once
 
 #include <cuda.h>
-#include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
 #include <cstdint>
@@ -132,8 +131,6 @@ struct Params {
     uint8_t* commit;
     unsigned long long timeout_ns;
     unsigned long long* trace;  // optional: [0] O_spec, [1] O_exact published (ns)
-    unsigned long long cond;    // graph conditional handle (cond_on != 0): set to 1
-    int cond_on;                // when a token is discarded
 };
 
 // Optional publication time stamps: after this thread's writes (and those
@@ -1331,12 +1328,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const __grid_const
                     r = sqrt(D2 / N2);
                 }
                 p.rel_l2[b] = (float)r;
-                const bool keep = r <= (double)p.lambda;
-                p.commit[b] = keep ? 1 : 0;
-                // Discarded: the graph's recomputation of what followed
-                // attention speculatively must run.
-                if (p.cond_on && !keep)
-                    cudaGraphSetConditional(static_cast<cudaGraphConditionalHandle>(p.cond), 1u);
+                p.commit[b] = r <= (double)p.lambda ? 1 : 0;
             }
         }
         if (lane == 0) trace_publish(p, 1);

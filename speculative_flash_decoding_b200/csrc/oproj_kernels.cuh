@@ -16,6 +16,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_runtime.h>
 
 #include <cstdint>
 
@@ -294,6 +295,15 @@ __global__ void __launch_bounds__(kObThreads, 1) oproj_bulk_kernel(const __grid_
         __threadfence();
         atomicMax(p.trace, (unsigned long long)global_ns());
     }
+}
+
+// Graph gating: enable the conditional node that redoes the projection when
+// any token of the batch was discarded (kept out of the merge kernel, which
+// the profiler could not capture while it could set a conditional handle).
+__global__ void __launch_bounds__(32) set_discard_condition(const uint8_t* commit, int B,
+                                                            cudaGraphConditionalHandle h) {
+    const bool discard = (int)threadIdx.x < B && commit[threadIdx.x] == 0;
+    if (__any_sync(0xffffffffu, discard) && threadIdx.x == 0) cudaGraphSetConditional(h, 1u);
 }
 
 using OprojFn = void (*)(OprojParams);
