@@ -246,6 +246,18 @@ alspec_status alspec_decode_oproj(const alspec_desc* desc,
                                   void* stream, unsigned long long* trace_ns);
 
 /*
+ * Read-bandwidth probe (a measurement aid, not part of the decode path):
+ * streams `bytes` of `buf` from HBM into shared memory with the same 1-D
+ * bulk copies and mbarrier ring the attention kernels use, one CTA per SM,
+ * and does nothing else.  Timing it gives the rate a pure streaming read
+ * reaches on this GPU.
+ *   buf    device, 16-byte aligned;  bytes a positive multiple of 16
+ *   err    device uint32 or NULL: ALSPEC_DEVERR_TIMEOUT on a wait timeout
+ * Asynchronous on `stream`.
+ */
+alspec_status alspec_read_probe(const void* buf, size_t bytes, uint32_t* err, void* stream);
+
+/*
  * Work plan the library would use (host only, no CUDA call except the SM
  * count query).  info[] receives, in order:
  *   0 tokens per sink-set work item      1 sink-set items per (b, kv head)

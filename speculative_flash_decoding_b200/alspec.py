@@ -73,6 +73,7 @@ SIGNATURES = {
     "alspec_decode_traced": (_i, [_descp, _vp, _vp, _vp, _vp, _i, _i, _f, _vp, _vp, _vp, _vp,
                                   _vp, _sz, _vp, _vp]),
     "alspec_oproj": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp]),
+    "alspec_read_probe": (_i, [_vp, _sz, _vp, _vp]),
     "alspec_decode_oproj": (_i, [_descp, _vp, _vp, _vp, _vp, _i, _i, _f, _vp, _i, _vp, _vp,
                                  _vp, _vp, _vp, _i, _vp, _sz, _vp, _vp]),
 }
@@ -161,6 +162,11 @@ def alspec_decode_oproj(desc: alspec_desc, q: int, k_cache: int, v_cache: int, s
                                         n_sink, window, lam, w_o, hidden, out_spec, out_exact,
                                         rel_l2, commit, y, gate, workspace, workspace_bytes,
                                         stream, trace_ns or None))
+
+
+def alspec_read_probe(buf: int, nbytes: int, stream: int, err: int = 0) -> int:
+    """Stream nbytes of buf from HBM (bandwidth probe)."""
+    return int(_lib.alspec_read_probe(buf, nbytes, err or None, stream))
 
 
 def alspec_decode_noalloc(desc: alspec_desc, q: int, k_cache: int, v_cache: int, seq_lens: int,

@@ -18,6 +18,7 @@
 #include "alspec.h"
 #include "attn_kernels.cuh"
 #include "oproj_kernels.cuh"
+#include "probe_kernels.cuh"
 
 namespace alspec {
 namespace {
@@ -706,6 +707,25 @@ alspec_status alspec_decode_oproj(const alspec_desc* desc, const void* q, const 
     return decode_impl(desc, q, k_cache, v_cache, seq_lens, n_sink, window, lambda, out_spec,
                        out_exact, rel_l2, commit, workspace, workspace_bytes, stream, nullptr,
                        nullptr, trace_ns, &op);
+}
+
+alspec_status alspec_read_probe(const void* buf, size_t bytes, uint32_t* err, void* stream) {
+    if (!buf || !aligned16(buf) || bytes == 0 || bytes % 16 != 0 ||
+        (reinterpret_cast<uintptr_t>(err) & 3u))
+        return ALSPEC_ERR_INVALID_ARG;
+    DeviceState* ds = nullptr;
+    alspec_status st = get_device_state(&ds);
+    if (st != ALSPEC_OK) return st;
+    if ((st = ensure_smem_attr(ds, reinterpret_cast<const void*>(read_probe_kernel), kRpSmem)) !=
+        ALSPEC_OK)
+        return st;
+    ReadProbeParams rp{};
+    rp.buf = static_cast<const unsigned char*>(buf);
+    rp.bytes = bytes;
+    rp.err = err;
+    rp.timeout_ns = 2000000000ull;
+    read_probe_kernel<<<ds->sm_count, 64, kRpSmem, static_cast<cudaStream_t>(stream)>>>(rp);
+    return ok(cudaGetLastError()) ? ALSPEC_OK : ALSPEC_ERR_CUDA;
 }
 
 alspec_status alspec_get_device_error(void* workspace, size_t workspace_bytes, void* stream,

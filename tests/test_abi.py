@@ -147,3 +147,9 @@ def test_traced_decode_rejects_bad_trace_buffer(trace, code):
     st = sfd.alspec_decode_traced(d, fake, fake, fake, fake, 4, 64, 0.1, fake, fake, fake, fake,
                                   fake, sfd.alspec_workspace_size(d, 4, 64), 0, trace)
     assert st == code
+
+
+@pytest.mark.parametrize("buf,nbytes", [(0, 1024), ((1 << 20) + 8, 1024), (1 << 20, 1000),
+                                        (1 << 20, 0)])
+def test_read_probe_rejects_bad_buffers(buf, nbytes):
+    assert sfd.alspec_read_probe(buf, nbytes, 0) == ab.ALSPEC_ERR_INVALID_ARG
