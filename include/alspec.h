@@ -246,6 +246,17 @@ alspec_status alspec_decode_oproj(const alspec_desc* desc,
                                   void* stream, unsigned long long* trace_ns);
 
 /*
+ * Test hook for failure detection: launches one CTA whose two bounded waits
+ * (written like the attention kernels' producer and consumer waits) target
+ * mbarriers that nothing ever arrives on.  The waits give up after
+ * timeout_ms (1..10000), ALSPEC_DEVERR_TIMEOUT is ORed into the workspace's
+ * device error word (read it with alspec_get_device_error), and the kernel
+ * returns: no trap, no fault.  Asynchronous on `stream`.
+ */
+alspec_status alspec_test_wait_timeout(void* workspace, size_t workspace_bytes, int timeout_ms,
+                                       void* stream);
+
+/*
  * Read-bandwidth probe (a measurement aid, not part of the decode path):
  * streams `bytes` of `buf` from HBM into shared memory with the same 1-D
  * bulk copies and mbarrier ring the attention kernels use, one CTA per SM,

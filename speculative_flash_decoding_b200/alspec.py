@@ -74,6 +74,7 @@ SIGNATURES = {
                                   _vp, _sz, _vp, _vp]),
     "alspec_oproj": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp]),
     "alspec_read_probe": (_i, [_vp, _sz, _vp, _vp]),
+    "alspec_test_wait_timeout": (_i, [_vp, _sz, _i, _vp]),
     "alspec_decode_oproj": (_i, [_descp, _vp, _vp, _vp, _vp, _i, _i, _f, _vp, _i, _vp, _vp,
                                  _vp, _vp, _vp, _i, _vp, _sz, _vp, _vp]),
 }
@@ -162,6 +163,12 @@ def alspec_decode_oproj(desc: alspec_desc, q: int, k_cache: int, v_cache: int, s
                                         n_sink, window, lam, w_o, hidden, out_spec, out_exact,
                                         rel_l2, commit, y, gate, workspace, workspace_bytes,
                                         stream, trace_ns or None))
+
+
+def alspec_test_wait_timeout(workspace: int, workspace_bytes: int, timeout_ms: int,
+                             stream: int) -> int:
+    """Test hook: a kernel whose waits can never complete must give up."""
+    return int(_lib.alspec_test_wait_timeout(workspace, workspace_bytes, timeout_ms, stream))
 
 
 def alspec_read_probe(buf: int, nbytes: int, stream: int, err: int = 0) -> int:

@@ -709,6 +709,19 @@ alspec_status alspec_decode_oproj(const alspec_desc* desc, const void* q, const 
                        nullptr, trace_ns, &op);
 }
 
+alspec_status alspec_test_wait_timeout(void* workspace, size_t workspace_bytes, int timeout_ms,
+                                       void* stream) {
+    if (!workspace || !aligned16(workspace) ||
+        workspace_bytes < (size_t)kCtrFixed * sizeof(unsigned) || timeout_ms < 1 ||
+        timeout_ms > 10000)
+        return ALSPEC_ERR_INVALID_ARG;
+    Params p{};
+    p.ctr = static_cast<unsigned*>(workspace);
+    p.timeout_ns = (unsigned long long)timeout_ms * 1000000ull;
+    stalled_wait_kernel<<<1, 64, 0, static_cast<cudaStream_t>(stream)>>>(p);
+    return ok(cudaGetLastError()) ? ALSPEC_OK : ALSPEC_ERR_CUDA;
+}
+
 alspec_status alspec_read_probe(const void* buf, size_t bytes, uint32_t* err, void* stream) {
     if (!buf || !aligned16(buf) || bytes == 0 || bytes % 16 != 0 ||
         (reinterpret_cast<uintptr_t>(err) & 3u))

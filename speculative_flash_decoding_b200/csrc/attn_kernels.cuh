@@ -379,6 +379,29 @@ __device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, volati
     }
 }
 
+// Test hook for the timeout path: both waits target mbarriers that nothing
+// ever arrives on.  The producer-style wait gives up at p.timeout_ns, sets
+// the abort flag and ORs the timeout bit into the error word; the
+// consumer-style wait sees the abort and returns.  Nothing traps or faults.
+__global__ void __launch_bounds__(64) stalled_wait_kernel(const __grid_constant__ Params p) {
+    __shared__ uint64_t bar[2];
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar[0], 1);
+        mbar_init(&bar[1], 1);
+        abort_flag = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+    volatile int* abort = &abort_flag;
+    const int lane = threadIdx.x & 31;
+    if (threadIdx.x < 32) {
+        if (lane == 0) (void)wait_one(&bar[0], 0, abort, p);
+    } else {
+        (void)wait_warp(&bar[1], 0, abort, p, lane);
+    }
+}
+
 // Weight of a partial with max m against the merged max M: exactly 1 when
 // m == M, so merging one partial with empty ones reproduces it bit for bit.
 __device__ __forceinline__ float merge_weight(float m, float M) {

@@ -153,3 +153,9 @@ def test_traced_decode_rejects_bad_trace_buffer(trace, code):
                                         (1 << 20, 0)])
 def test_read_probe_rejects_bad_buffers(buf, nbytes):
     assert sfd.alspec_read_probe(buf, nbytes, 0) == ab.ALSPEC_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("ws,nbytes,ms", [(0, 4096, 1), (1 << 20, 4096, 0), (1 << 20, 4096, 20000),
+                                          (1 << 20, 4, 1), ((1 << 20) + 4, 4096, 1)])
+def test_wait_timeout_hook_rejects_bad_arguments(ws, nbytes, ms):
+    assert sfd.alspec_test_wait_timeout(ws, nbytes, ms, 0) == ab.ALSPEC_ERR_INVALID_ARG

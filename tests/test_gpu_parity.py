@@ -289,3 +289,30 @@ def test_full_size_70b_layer(cuda_device):
     _, out = gpu_decode(wl, data, cuda_device)
     ref = oracle_decode(wl, data, batch=[0])
     assert_parity(out, ref, wl.lam, batch=[0], what="cfg4 full b0")
+
+
+def test_wait_that_never_completes_gives_up_and_reports(cuda_device):
+    """Failure detection without a fault: waits on barriers nothing arrives
+    on give up after a 1 ms limit and raise the timeout bit, which
+    alspec_get_device_error reports (and clears)."""
+    import time
+    import speculative_flash_decoding_b200 as sfd
+    wl = _small(1)
+    dec = sfd.Decoder(wl.B, wl.Hq, wl.Hkv, wl.d, wl.L, wl.dtype, wl.S, wl.W, device=cuda_device)
+    s = torch.cuda.current_stream()
+    t0 = time.perf_counter()
+    assert sfd.alspec_test_wait_timeout(dec.workspace.data_ptr(), dec.workspace_bytes, 1,
+                                        s.cuda_stream) == 0
+    torch.cuda.synchronize()
+    assert time.perf_counter() - t0 < 5.0
+    st, err = dec.device_error()
+    assert st == sfd.ALSPEC_ERR_TIMEOUT and err & sfd.ALSPEC_DEVERR_TIMEOUT
+    assert dec.device_error() == (0, 0)
+
+
+def test_one_millisecond_limit_does_not_fire_on_normal_work(cuda_device):
+    wl = _small(2)
+    data = workloads.make_layer(wl, device=cuda_device)
+    dec, out = gpu_decode(wl, data, cuda_device, timeout_ms=1)
+    assert dec.device_error() == (0, 0)
+    assert_parity(out, oracle_decode(wl, data), wl.lam, what="1 ms wait limit")
