@@ -384,8 +384,10 @@ def run_alspec(args, wl):
     t_end = torch.cuda.Event(enable_timing=True)
     step_begin = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     step_end = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    nvtx = torch.cuda.nvtx
     with ClockSampler(uuid) as clocks:
         barrier()
+        nvtx.range_push("timed steps")
         t_start.record(stream)
         for i in range(args.steps):
             if flush:
@@ -398,24 +400,29 @@ def run_alspec(args, wl):
             step_end[i].record(stream)
         t_end.record(stream)
         barrier()
+        nvtx.range_pop()
     per_step = [step_begin[i].elapsed_time(step_end[i]) for i in range(args.steps)]
     ms_total = sum(per_step) if flush else t_start.elapsed_time(t_end)
     ms_per_step = ranks.max(ms_total / args.steps)
 
     # Profiled pass: same step with per-layer events captured in the graphs.
     barrier()
+    nvtx.range_push("profiled pass (per-layer events)")
     with torch.cuda.stream(stream):
         for g in prof_graphs:
             assert sfd.alspec_graph_launch(g, stream.cuda_stream) == 0
     barrier()
+    nvtx.range_pop()
 
     # Latency pass.
     barrier()
+    nvtx.range_push("latency pass (kernel time stamps)")
     traces.zero_()
     with torch.cuda.stream(stream):
         for g in lat:
             assert sfd.alspec_graph_launch(g, stream.cuda_stream) == 0
     barrier()
+    nvtx.range_pop()
     tr = traces.cpu().numpy().astype("int64")
     t_spec, t_exact = [], []
     for j in range(prof_steps):
@@ -450,6 +457,7 @@ def run_alspec(args, wl):
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         barrier()
+        nvtx.range_push("end to end (host buffers)")
         with torch.cuda.stream(stream):
             e0.record(stream)
             for i in range(args.steps):
@@ -461,6 +469,7 @@ def run_alspec(args, wl):
                 stream.synchronize()
             e1.record(stream)
         barrier()
+        nvtx.range_pop()
         e2e_ms = ranks.max(e0.elapsed_time(e1) / args.steps)
         h2d = q_host.numel() * q_host.element_size() + lens_host.numel() * lens_host.element_size()
         d2h = rel_host.numel() * rel_host.element_size() + com_host.numel() * com_host.element_size()

@@ -69,9 +69,9 @@ constexpr int kMaxSpecCtas = 8;
 #endif
 
 // Stages per token slot of the tensor-core middle kernel: 3 stages of 16 KB
-// per consumer warp keep up to 192 KB in flight per SM -- well above the HBM
-// bandwidth-latency product -- so the producer keeps streaming through the
-// few microseconds an item's end (merging the warps' states) takes.
+// per consumer warp keep up to 192 KB in flight per SM (a warp holds one of
+// its stages for the ~0.8 us its tile's math takes), so the producer keeps
+// streaming through the few microseconds an item's end takes.
 #ifndef ALSPEC_MID_SPW
 #define ALSPEC_MID_SPW 3
 #endif
@@ -306,6 +306,12 @@ struct Cfg {
     static constexpr int kSpwBudget =
         (kSmemLimit - 1024 - kDepositBytes - 4096 - 768 - kGatherBytes) / (NTW * kStageBytes);
     static constexpr int SPW = kSpwBudget < 1 ? 1 : (kSpwBudget > kSpwMax ? kSpwMax : kSpwBudget);
+    // Tile t goes to stage t mod STAGES and to consumer warp t mod NTW, so
+    // with STAGES a multiple of NTW every stage has one consumer warp, which
+    // waits for its stage's fills in order.  That is what makes the
+    // phase-parity waits sound: a waiter is never a ring lap ahead of the
+    // stage's previous fill (with a stage shared by several warps, a fast
+    // warp could pass the parity test on the previous fill's phase).
     static constexpr int STAGES = NTW * SPW;
     // Dynamic shared memory layout (offsets from a 1024-byte aligned base;
     // every region starts on a 128-byte boundary: the stage metadata are
@@ -328,6 +334,7 @@ struct Cfg {
     static_assert(!MMA || (sizeof(T) == 2 && G <= 8), "tensor-core engine: bf16, g <= 8");
     static_assert(kSmemBytes <= kSmemLimit, "shared memory budget");
     static_assert(NTW >= 1 && NCW <= 8, "warp split");
+    static_assert(STAGES % NTW == 0, "each stage must belong to one consumer warp");
 };
 
 // ---------------------------------------------------------------- waiting
