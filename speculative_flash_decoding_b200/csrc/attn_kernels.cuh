@@ -460,6 +460,13 @@ struct CoreEngine {
     }
 
     // One 16-token tile: lanes 8u..8u+7 ("group" u) own rows 4u..4u+3.
+    // One step: the CUDA-core engine reads the stage to the end of the tile.
+    __device__ __forceinline__ void tile_load(char* ks, char* vs, int nvalid, int lane,
+                                              float qscale) {
+        tile(ks, vs, nvalid, lane, qscale);
+    }
+    __device__ __forceinline__ void tile_finish(int, int, float) {}
+
     __device__ __forceinline__ void tile(char* ks, char* vs, int nvalid, int lane, float) {
         const int grp = lane >> 3;
         const int li = lane & 7;
@@ -614,6 +621,8 @@ struct MmaEngine {
     float o[NT][4];      // P V accumulators: rows g (high part of P) and g+8 (residual)
     float m;             // running max of row g (log2 domain)
     float l;             // this lane's share of the exponential sum of row g
+    float s[TT / 8][4];  // the current tile's scores (between tile_load and tile_finish)
+    uint32_t vf[TT / 16][NT / 2][4];  // the current tile's V fragments
 
     __device__ __forceinline__ void reset() {
         m = -INFINITY;
@@ -644,10 +653,9 @@ struct MmaEngine {
         return base + (uint32_t)((c >> 3) * kHalf) + swz(r, c & 7);
     }
 
-    __device__ __forceinline__ void tile(char* ks, char* vs, int nvalid, int lane, float qscale) {
-        const int g = lane >> 2;
-        const int r = lane & 3;
-        const unsigned full = 0xffffffffu;
+    // Everything that reads the stage: clear padded rows, S^T = Q K^T, and
+    // V's fragments into registers.  The stage can be released after this.
+    __device__ __forceinline__ void tile_load(char* ks, char* vs, int nvalid, int lane, float) {
         // Rows past the end of the item may hold anything (even NaN): zero
         // their values so that 0 * V stays 0 in the P V products.
         if (nvalid < TT) {
@@ -666,7 +674,6 @@ struct MmaEngine {
 
         // S^T = Q K^T: 4 n-tiles of 8 tokens.  Even and odd k-steps go to
         // separate accumulators (half-length MMA dependency chains).
-        float s[TT / 8][4];
 #pragma unroll
         for (int j = 0; j < TT / 8; ++j) {
             float s2[4] = {0.f, 0.f, 0.f, 0.f};
@@ -681,7 +688,22 @@ struct MmaEngine {
 #pragma unroll
             for (int i = 0; i < 4; ++i) s[j][i] += s2[i];
         }
+        // V as the B operand of P V (transposed 8x8 loads), 2 k-steps of 16.
+#pragma unroll
+        for (int t2 = 0; t2 < TT / 16; ++t2)
+#pragma unroll
+            for (int jp = 0; jp < NT / 2; ++jp) {
+                const int row = 16 * t2 + ((lane >> 3) & 1) * 8 + (lane & 7);
+                ldsm_x4_t(addr(vb, row, 2 * jp + (lane >> 4)), vf[t2][jp][0], vf[t2][jp][1],
+                          vf[t2][jp][2], vf[t2][jp][3]);
+            }
+    }
 
+    // The rest of the tile, from registers: online softmax and O += P V.
+    __device__ __forceinline__ void tile_finish(int nvalid, int lane, float qscale) {
+        const int g = lane >> 2;
+        const int r = lane & 3;
+        const unsigned full = 0xffffffffu;
         // Online softmax on row g (lanes 4g..4g+3 hold its 32 scores).
         float mx = -INFINITY;
 #pragma unroll
@@ -729,11 +751,10 @@ struct MmaEngine {
         for (int t2 = 0; t2 < TT / 16; ++t2) {
 #pragma unroll
             for (int jp = 0; jp < NT / 2; ++jp) {
-                uint32_t b0, b1, b2, b3;
-                const int row = 16 * t2 + ((lane >> 3) & 1) * 8 + (lane & 7);
-                ldsm_x4_t(addr(vb, row, 2 * jp + (lane >> 4)), b0, b1, b2, b3);
-                mma_bf16_16816(o[2 * jp], pa[t2][0], pa[t2][1], pa[t2][2], pa[t2][3], b0, b1);
-                mma_bf16_16816(o[2 * jp + 1], pa[t2][0], pa[t2][1], pa[t2][2], pa[t2][3], b2, b3);
+                mma_bf16_16816(o[2 * jp], pa[t2][0], pa[t2][1], pa[t2][2], pa[t2][3],
+                               vf[t2][jp][0], vf[t2][jp][1]);
+                mma_bf16_16816(o[2 * jp + 1], pa[t2][0], pa[t2][1], pa[t2][2], pa[t2][3],
+                               vf[t2][jp][2], vf[t2][jp][3]);
             }
         }
     }
@@ -1045,10 +1066,13 @@ __device__ __forceinline__ void consume(const Params& p, unsigned char* smem, fl
         }
         if (mt.z > 0) {
             char* ks = reinterpret_cast<char*>(smem) + s * C::kStageBytes;
-            st.tile(ks, ks + C::kTileBytes, mt.z, lane, p.qscale);
+            st.tile_load(ks, ks + C::kTileBytes, mt.z, lane, p.qscale);
         }
+        // The stage is released as soon as nothing more reads it (the
+        // tensor-core engine holds the tile's V fragments in registers).
         __syncwarp();
         if (lane == 0) mbar_arrive(empty_bar + s);
+        if (mt.z > 0) st.tile_finish(mt.z, lane, p.qscale);
         if (!(mt.w & kLastTileFlag)) continue;
 
         // ---- end of this item: combine the warps' states into one partial.
