@@ -122,13 +122,15 @@ __global__ void __launch_bounds__(kOprojWarps * 32) oproj_kernel(const __grid_co
 // Foreground form: a persistent kernel, one CTA per SM, that streams the
 // weight rows with 1-D bulk copies (TMA, evict-first) into a ring of
 // 8 KB shared-memory stages -- so the bytes in flight are not bounded by the
-// L1's outstanding-miss tracking, which held plain loads near 2 TB/s.  CTA c
+// L1's outstanding-miss tracking, which held plain loads near 2 TB/s; with
+// 24 stages (192 KB) nearly an SM's whole share of a 4096 x 4096 matrix is
+// in flight at once.  CTA c
 // owns rows [c * R, (c + 1) * R); a row is P = 2K / 8192 stages; consumer
 // warp w owns the CTA's rows w, w + 8, ...; one producer lane fills the
 // stages in order; for B <= 2 each lane loads four chunks (and their x)
 // before it computes on any of them.  Every wait is bounded: on expiry the kernel ORs the
 // timeout bit into p.err, stops, lets its copies land (bounded) and returns.
-constexpr int kObStages = 12;
+constexpr int kObStages = 24;
 constexpr int kObPiece = 8192;   // bytes per stage
 constexpr int kObConsumers = 8;
 constexpr int kObThreads = (kObConsumers + 1) * 32;
