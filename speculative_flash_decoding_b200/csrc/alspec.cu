@@ -26,6 +26,18 @@ namespace {
 constexpr int kMaxDevices = 64;
 constexpr int kMaxSpecItems = kMaxSpecCtas;  // sink-set CTAs per (sequence, KV head)
 
+// Share of the SMs the sink-set CTAs may take together (NUM / DEN).  More
+// sink-set CTAs per head bring O_spec sooner but hold SMs the middle kernel
+// would stream with: 3/4 keeps the 70B shape (32 heads, 4100-row sink set)
+// at 3 CTAs per head (O_spec at 0.074 of the layer instead of 0.10, layer
+// +0.7%); the whole GPU would give the 64-head ragged batch 2 CTAs per head
+// (0.095 instead of 0.15) for 5% of its throughput.
+#ifndef ALSPEC_SPEC_SM_SHARE_NUM
+#define ALSPEC_SPEC_SM_SHARE_NUM 3
+#endif
+#ifndef ALSPEC_SPEC_SM_SHARE_DEN
+#define ALSPEC_SPEC_SM_SHARE_DEN 4
+#endif
 // Smallest middle chunk of the guided self-scheduled split, in tiles.
 #ifndef ALSPEC_GSS_MIN_TILES
 #define ALSPEC_GSS_MIN_TILES 16
@@ -170,8 +182,9 @@ void make_plan(const alspec_desc& d, int S, int W, int sms, Plan* pl) {
     const int tiles_max = ceil_div(std::min(S, L), TT) + ceil_div(std::min(W, L), TT);
     // CTAs per head for the sink set (one thread-block cluster): about
     // ALSPEC_SPEC_TILES tiles each, at most 8 (the portable cluster size),
-    // and all heads together within half of the SMs.
-    const int room1 = std::max(1, sms / 2 / std::max(1, heads));
+    // and all heads together within ALSPEC_SPEC_SM_SHARE of the SMs.
+    const int room1 = std::max(1, sms * ALSPEC_SPEC_SM_SHARE_NUM / ALSPEC_SPEC_SM_SHARE_DEN /
+                                      std::max(1, heads));
     pl->n1 = std::max(1, std::min({kMaxSpecItems, room1, ceil_div(tiles_max, ALSPEC_SPEC_TILES)}));
     const int tiles_per_item = ceil_div(tiles_max, pl->n1);
     pl->c1 = tiles_per_item * TT;
