@@ -577,9 +577,6 @@ alspec_status decode_impl(const alspec_desc* desc, const void* q, const void* k_
         if (!ok(cudaGetLastError()) || !ok(cudaEventRecord(ds->join2, ds->lo)))
             return ALSPEC_ERR_CUDA;
     }
-#ifdef ALSPEC_SPEC_SERIAL
-    if (!ok(cudaStreamWaitEvent(s, ds->join, 0))) return ALSPEC_ERR_CUDA;
-#endif
     // The middle of every sequence on the caller's stream.
     if (!prof(2, s)) return ALSPEC_ERR_CUDA;
     if (pl.n2 > 0) {
