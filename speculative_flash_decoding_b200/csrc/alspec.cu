@@ -769,8 +769,8 @@ alspec_status alspec_get_device_error(void* workspace, size_t workspace_bytes, v
 }
 
 alspec_status alspec_graph_begin(void* stream) {
-    return cudaStreamBeginCapture(static_cast<cudaStream_t>(stream),
-                                  cudaStreamCaptureModeThreadLocal) == cudaSuccess
+    return ok(cudaStreamBeginCapture(static_cast<cudaStream_t>(stream),
+                                     cudaStreamCaptureModeThreadLocal))
                ? ALSPEC_OK
                : ALSPEC_ERR_CUDA;
 }
@@ -778,29 +778,29 @@ alspec_status alspec_graph_begin(void* stream) {
 alspec_status alspec_graph_end(void* stream, void** graph) {
     if (!graph) return ALSPEC_ERR_INVALID_ARG;
     cudaGraph_t g = nullptr;
-    if (cudaStreamEndCapture(static_cast<cudaStream_t>(stream), &g) != cudaSuccess || !g)
+    if (!ok(cudaStreamEndCapture(static_cast<cudaStream_t>(stream), &g)) || !g)
         return ALSPEC_ERR_CUDA;
     cudaGraphExec_t exec = nullptr;
-    const cudaError_t e = cudaGraphInstantiateWithFlags(&exec, g, cudaGraphInstantiateFlagUseNodePriority);
+    const bool inst =
+        ok(cudaGraphInstantiateWithFlags(&exec, g, cudaGraphInstantiateFlagUseNodePriority));
     cudaGraphDestroy(g);
-    if (e != cudaSuccess) return ALSPEC_ERR_CUDA;
+    if (!inst) return ALSPEC_ERR_CUDA;
     *graph = exec;
     return ALSPEC_OK;
 }
 
 alspec_status alspec_graph_launch(void* graph, void* stream) {
     if (!graph) return ALSPEC_ERR_INVALID_ARG;
-    return cudaGraphLaunch(static_cast<cudaGraphExec_t>(graph), static_cast<cudaStream_t>(stream)) ==
-                   cudaSuccess
+    return ok(cudaGraphLaunch(static_cast<cudaGraphExec_t>(graph),
+                              static_cast<cudaStream_t>(stream)))
                ? ALSPEC_OK
                : ALSPEC_ERR_CUDA;
 }
 
 alspec_status alspec_graph_destroy(void* graph) {
     if (!graph) return ALSPEC_ERR_INVALID_ARG;
-    return cudaGraphExecDestroy(static_cast<cudaGraphExec_t>(graph)) == cudaSuccess
-               ? ALSPEC_OK
-               : ALSPEC_ERR_CUDA;
+    return ok(cudaGraphExecDestroy(static_cast<cudaGraphExec_t>(graph))) ? ALSPEC_OK
+                                                                         : ALSPEC_ERR_CUDA;
 }
 
 alspec_status alspec_shutdown(void) {
@@ -816,6 +816,7 @@ alspec_status alspec_shutdown(void) {
             continue;
         }
         if (cudaStreamSynchronize(s.hi) != cudaSuccess) st = ALSPEC_ERR_CUDA;
+        if (s.lo && cudaStreamSynchronize(s.lo) != cudaSuccess) st = ALSPEC_ERR_CUDA;
         cudaEventDestroy(s.fork);
         cudaEventDestroy(s.join);
         if (s.join2) cudaEventDestroy(s.join2);
@@ -840,7 +841,7 @@ const char* alspec_status_string(alspec_status status) {
     }
 }
 
-int alspec_version(void) { return 100; }
+int alspec_version(void) { return 200; }
 
 int alspec_last_cuda_error(void) { return (int)t_last_error; }
 
