@@ -29,6 +29,10 @@
  *   - Arguments that can be checked on the host are checked before anything
  *     is launched; a failed check returns a status and launches nothing.
  *     Nothing aborts, traps or exits.
+ *   - Calls may come from several host threads: each call enqueues its work
+ *     on the library's shared streams under a per-device lock.  While one
+ *     thread captures calls into a graph, no other thread may issue calls on
+ *     the same device (the shared streams join that capture).
  */
 #ifndef ALSPEC_H
 #define ALSPEC_H

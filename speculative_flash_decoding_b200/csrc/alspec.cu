@@ -86,6 +86,10 @@ struct DeviceState {
 
 std::mutex g_mutex;
 DeviceState g_dev[kMaxDevices];
+// One per device: a call's event records, waits and launches on the shared
+// streams are enqueued as one unit, so calls from several host threads do
+// not interleave their fork / join events.
+std::mutex g_call_mutex[kMaxDevices];
 
 alspec_status get_device_state(DeviceState** out) {
     int dev = 0;
@@ -502,6 +506,7 @@ alspec_status decode_impl(const alspec_desc* desc, const void* q, const void* k_
     if (workspace_bytes < pl.total) return ALSPEC_ERR_WORKSPACE;
     DeviceState* ds = nullptr;
     if ((st = get_device_state(&ds)) != ALSPEC_OK) return st;
+    std::lock_guard<std::mutex> call_lock(g_call_mutex[ds - g_dev]);
     const int G = desc->n_q_heads / desc->n_kv_heads;
     KernelSet ks{};
     if (!pick(desc->dtype, desc->head_dim, G, pl.engine, &ks)) return ALSPEC_ERR_UNSUPPORTED;

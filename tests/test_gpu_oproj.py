@@ -133,3 +133,40 @@ def test_read_probe_streams_without_error(cuda_device):
                                  err.data_ptr()) == 0
     torch.cuda.synchronize()
     assert err.item() == 0
+
+
+def test_speculative_projection_over_layers_in_one_graph(cuda_device):
+    """Three layers of decode + speculative projection captured in one graph
+    (each layer's own weights), replayed: every layer's y is the gated
+    projection of its own attention outputs."""
+    import speculative_flash_decoding_b200 as sfd
+    wl = workloads.COMMIT_VARIANT.replace(L=8192, ragged=(6000, 8192))
+    layers = [workloads.make_layer(wl, layer=i, device=cuda_device) for i in range(3)]
+    ws = [_bf16_weights(768, wl.Hq * wl.d, 50 + i, cuda_device) for i in range(3)]
+    dec = sfd.Decoder(wl.B, wl.Hq, wl.Hkv, wl.d, wl.L, wl.dtype, wl.S, wl.W, device=cuda_device)
+    dec.decode(layers[0]["q"], layers[0]["k"], layers[0]["v"], layers[0]["seq_lens"], wl.lam)
+    torch.cuda.synchronize()
+    outs = []
+    for _ in layers:
+        o = dec.alloc_outputs()
+        o["y"] = torch.full((wl.B, 768), 7.0, device=cuda_device)
+        outs.append(o)
+    stream = torch.cuda.Stream(cuda_device)
+    with torch.cuda.stream(stream):
+        assert sfd.alspec_graph_begin(stream.cuda_stream) == 0
+        for d, o, w in zip(layers, outs, ws):
+            dec.decode_oproj(d["q"], d["k"], d["v"], d["seq_lens"], wl.lam, w, out=o,
+                             stream=stream)
+        st, g = sfd.alspec_graph_end(stream.cuda_stream)
+        assert st == 0 and g
+        for _ in range(2):
+            assert sfd.alspec_graph_launch(g, stream.cuda_stream) == 0
+        stream.synchronize()
+        assert sfd.alspec_graph_destroy(g) == 0
+    for d, o, w in zip(layers, outs, ws):
+        commit = o["commit"].cpu().numpy()
+        mine = oracle.oproj_gated(o["out_spec"].cpu().numpy().reshape(wl.B, -1),
+                                  o["out_exact"].cpu().numpy().reshape(wl.B, -1), commit,
+                                  workloads.to_numpy_bits(w))
+        assert _row_rel(o["y"].cpu().numpy(), mine).max() < ROW_TOL
+    assert dec.device_error() == (0, 0)

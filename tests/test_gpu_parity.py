@@ -316,3 +316,49 @@ def test_one_millisecond_limit_does_not_fire_on_normal_work(cuda_device):
     dec, out = gpu_decode(wl, data, cuda_device, timeout_ms=1)
     assert dec.device_error() == (0, 0)
     assert_parity(out, oracle_decode(wl, data), wl.lam, what="1 ms wait limit")
+
+
+def test_calls_from_two_host_threads(cuda_device):
+    """Two threads, each with its own decoder and stream, decode at the same
+    time; every output equals the single-threaded result bit for bit."""
+    import threading
+    import speculative_flash_decoding_b200 as sfd
+    wl = _small(2)
+    layers = [workloads.make_layer(wl, layer=i, device=cuda_device) for i in range(4)]
+    ref = []
+    dec0 = sfd.Decoder(wl.B, wl.Hq, wl.Hkv, wl.d, wl.L, wl.dtype, wl.S, wl.W, device=cuda_device)
+    for d in layers:
+        o = dec0.decode(d["q"], d["k"], d["v"], d["seq_lens"], wl.lam)
+        torch.cuda.synchronize()
+        ref.append({k: v.clone() for k, v in o.items()})
+    got = [None] * len(layers)
+    errors = []
+
+    def work(idx):
+        try:
+            torch.cuda.set_device(cuda_device)
+            dec = sfd.Decoder(wl.B, wl.Hq, wl.Hkv, wl.d, wl.L, wl.dtype, wl.S, wl.W,
+                              device=cuda_device)
+            stream = torch.cuda.Stream(cuda_device)
+            with torch.cuda.stream(stream):
+                for rep in range(20):
+                    for i in idx:
+                        d = layers[i]
+                        o = dec.decode(d["q"], d["k"], d["v"], d["seq_lens"], wl.lam,
+                                       stream=stream)
+                        if rep == 19:
+                            stream.synchronize()
+                            got[i] = {k: v.clone() for k, v in o.items()}
+                stream.synchronize()
+        except Exception as e:  # reported below
+            errors.append(e)
+
+    threads = [threading.Thread(target=work, args=(ix,)) for ix in ([0, 1], [2, 3])]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join()
+    assert not errors, errors
+    for r, g in zip(ref, got):
+        for k in r:
+            assert torch.equal(r[k], g[k]), k
