@@ -33,6 +33,7 @@ METRIC = "KV GB/s (fraction of HBM peak) and µs/decode-step to commit flag at 1
 FALLBACK_HBM_GBS = 6650.0
 MID_KERNEL_SRC = os.path.join(ROOT, "speculative_flash_decoding_b200", "csrc", "attn_kernels.cuh")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_mid_llama8b_128k_traffic.md")
+FUSED_TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_fused_llama8b_128k_traffic.md")
 
 
 NOMINAL_HBM_GBS = 8000.0  # the HBM3e figure the target is stated against
@@ -53,6 +54,9 @@ def parse_args():
     ap.add_argument("--split-tokens", type=int, default=0,
                     help="exact-path item size for the longest sequence (0 = library's choice)")
     ap.add_argument("--engine", default="auto", choices=["auto", "cuda_cores", "tensor_cores"])
+    ap.add_argument("--schedule", default="auto", choices=["auto", "streams", "fused"],
+                    help="launch schedule: streams (sink set on a high-priority stream, three "
+                         "kernels) or fused (one persistent launch); auto = streams")
     ap.add_argument("--oproj", action="store_true",
                     help="speculative output projection against the serial one (32 x 128K)")
     ap.add_argument("--lambda-sweep", action="store_true",
@@ -121,11 +125,11 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def stored_traffic():
-    """DRAM bytes per launch of the middle kernel from the committed ncu summary,
-    or None when the kernel source changed since it was captured."""
+def stored_traffic(path):
+    """DRAM bytes per launch of the dominant kernel from a committed ncu
+    summary, or None when the kernel source changed since it was captured."""
     try:
-        text = open(TRAFFIC_FILE).read()
+        text = open(path).read()
     except OSError:
         return None
     m_hash = re.search(r"source_sha256:\s*([0-9a-f]{64})", text)
@@ -294,8 +298,9 @@ def run_alspec(args, wl):
         d["seq_lens"] = lens_all[i]
     kv_bytes = sum(workloads.kv_bytes(wl, d["lens"]) for d in layers)
     dec = sfd.Decoder(wl.B, wl.Hq, wl.Hkv, wl.d, wl.L, wl.dtype, wl.S, wl.W, device=device,
-                      split_tokens=args.split_tokens, engine=args.engine)
+                      split_tokens=args.split_tokens, engine=args.engine, schedule=args.schedule)
     plan = dec.plan()
+    fused = plan["schedule"] == sfd.ALSPEC_SCHEDULE_FUSED
     out_spec = torch.empty(n_layers, wl.B, wl.Hq, wl.d, dtype=torch.float32, device=device)
     out_exact = torch.empty_like(out_spec)
     rel_all = torch.empty(n_layers, wl.B, dtype=torch.float32, device=device)
@@ -500,12 +505,16 @@ def run_alspec(args, wl):
         read_probe = {"gbs": probe_gbs, "bytes_per_launch": nbytes, "launches": 5}
         del buf
     peak, peak_kind = measured_peak()
+    # The dominant kernel: the middle kernel (two-stream schedule) or the one
+    # kernel of the one-launch schedule, which reads every cache row.
     mid_bytes = sum(
         (max(0, L - wl.W - min(wl.S, L)) if L > wl.S + wl.W else 0) * wl.Hkv * wl.d * 2 *
         wl.elem_bytes for L in layers[0]["lens"])
+    if fused:
+        mid_bytes = workloads.kv_bytes(wl, layers[0]["lens"])
     mid_avg_ms = sum(mid_ms) / len(mid_ms)
     achieved = mid_bytes / (mid_avg_ms * 1e-3) / 1e9
-    traffic = stored_traffic()
+    traffic = stored_traffic(FUSED_TRAFFIC_FILE if fused else TRAFFIC_FILE)
     value = job_throughput(kv_bytes, world, ms_per_step)
 
     cpu = None
@@ -543,10 +552,11 @@ def run_alspec(args, wl):
                    "timing": "CUDA graph per step, CUDA events on the launch stream; "
                              "per-kernel times from a second pass of graphs with per-layer "
                              "events",
+                   "schedule": "fused" if fused else "streams",
                    "plan": plan},
         "roofline": {"bound": "hbm",
-                     "kernel": "attn_kernel<%s,%d,%d,middle,%s>" % (
-                         wl.dtype, wl.d, wl.g,
+                     "kernel": "attn_kernel<%s,%d,%d,%s,%s>" % (
+                         wl.dtype, wl.d, wl.g, "fused" if fused else "middle",
                          {1: "cuda_cores", 2: "tensor_cores"}.get(plan["engine"], "?")),
                      "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_kind": peak_kind,
@@ -575,7 +585,7 @@ def run_alspec(args, wl):
         "hit_rate": hit_rate,
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": args.steps * n_layers * (3 if plan["n2"] > 0 else 2),
+        "gpu_launches": args.steps * n_layers * (1 if fused else (3 if plan["n2"] > 0 else 2)),
         "clocks": clocks.summary(),
     }
     print(json.dumps(line), flush=True)

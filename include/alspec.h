@@ -66,6 +66,26 @@ typedef enum {
     ALSPEC_ENGINE_TENSOR_CORES = 2   /* bf16 m16n8k16 MMAs; bf16 only             */
 } alspec_engine;
 
+/*
+ * Launch schedule of one decode call (alspec_desc.schedule).
+ *   STREAMS: the sink-set kernel on a high-priority stream forked from the
+ *            caller's (O_spec early, marked by spec_event), the exact-path
+ *            kernel on the caller's stream, then a merge kernel that also
+ *            writes rel_l2 and the flags: three launches and a fork/join.
+ *   FUSED:   one persistent launch on the caller's stream.  The sink-set
+ *            work items come first in the same work queue as the exact
+ *            path's; the CTA that completes a (sequence, KV head) writes its
+ *            O_spec and O_exact, and the CTA that completes a sequence
+ *            writes rel_l2 and the flag (ticket counters in the workspace).
+ *            O_spec is complete only when the launch ends (spec_event marks
+ *            that point); alspec_decode_oproj is not available with it.
+ */
+typedef enum {
+    ALSPEC_SCHEDULE_AUTO = 0,     /* STREAMS */
+    ALSPEC_SCHEDULE_STREAMS = 1,
+    ALSPEC_SCHEDULE_FUSED = 2
+} alspec_schedule;
+
 /* Gating of the recomputation in alspec_decode_oproj. */
 typedef enum {
     ALSPEC_GATE_KERNEL = 0,             /* a kernel that reads the flags           */
@@ -102,6 +122,7 @@ typedef struct {
     int split_tokens;   /* 0 = automatic */
     int timeout_ms;     /* bound on any in-kernel wait; 0 = 2000 ms */
     int engine;         /* alspec_engine; 0 = automatic */
+    int schedule;       /* alspec_schedule; 0 = automatic */
 } alspec_desc;
 
 /*
@@ -281,8 +302,10 @@ alspec_status alspec_read_probe(const void* buf, size_t bytes, uint32_t* err, vo
  *   4 persistent CTAs of the exact path  5 threads per CTA
  *   6 dynamic shared memory per CTA      7 pipeline stages
  *   8 engine (alspec_engine, resolved)
- * (entries 5-7 describe the exact-path kernel).  n_info is the capacity of
- * info (9 fills all).
+ *   9 schedule (alspec_schedule, resolved)
+ * (entries 4-7 describe the exact-path kernel, or with the FUSED schedule
+ * the one kernel, whose queue holds both kinds of items).  n_info is the
+ * capacity of info (10 fills all).
  */
 alspec_status alspec_query_plan(const alspec_desc* desc, int n_sink, int window,
                                 int* info, int n_info);

@@ -42,11 +42,15 @@ ALSPEC_ENGINE_AUTO = 0
 ALSPEC_ENGINE_CUDA_CORES = 1
 ALSPEC_ENGINE_TENSOR_CORES = 2
 
+ALSPEC_SCHEDULE_AUTO = 0
+ALSPEC_SCHEDULE_STREAMS = 1
+ALSPEC_SCHEDULE_FUSED = 2
+
 
 class alspec_desc(ctypes.Structure):
     _fields_ = [("batch", _i), ("n_q_heads", _i), ("n_kv_heads", _i), ("head_dim", _i),
                 ("max_seq_len", _i), ("dtype", _i), ("split_tokens", _i), ("timeout_ms", _i),
-                ("engine", _i)]
+                ("engine", _i), ("schedule", _i)]
 
 
 _descp = ctypes.POINTER(alspec_desc)
@@ -188,9 +192,9 @@ def alspec_decode_noalloc(desc: alspec_desc, q: int, k_cache: int, v_cache: int,
 
 
 def alspec_query_plan(desc: alspec_desc, n_sink: int, window: int):
-    info = (ctypes.c_int * 9)()
-    st = int(_lib.alspec_query_plan(ctypes.byref(desc), n_sink, window, info, 9))
-    keys = ("c1", "n1", "c2", "n2", "grid2", "threads", "smem", "stages", "engine")
+    info = (ctypes.c_int * 10)()
+    st = int(_lib.alspec_query_plan(ctypes.byref(desc), n_sink, window, info, 10))
+    keys = ("c1", "n1", "c2", "n2", "grid2", "threads", "smem", "stages", "engine", "schedule")
     return st, dict(zip(keys, list(info)))
 
 
@@ -248,14 +252,17 @@ def alspec_last_cuda_error() -> int:
 
 ENGINES = {"auto": ALSPEC_ENGINE_AUTO, "cuda_cores": ALSPEC_ENGINE_CUDA_CORES,
            "tensor_cores": ALSPEC_ENGINE_TENSOR_CORES}
+SCHEDULES = {"auto": ALSPEC_SCHEDULE_AUTO, "streams": ALSPEC_SCHEDULE_STREAMS,
+             "fused": ALSPEC_SCHEDULE_FUSED}
 
 
 def make_desc(batch, n_q_heads, n_kv_heads, head_dim, max_seq_len, dtype, split_tokens=0,
-              timeout_ms=0, engine="auto") -> alspec_desc:
+              timeout_ms=0, engine="auto", schedule="auto") -> alspec_desc:
     code = {"bf16": ALSPEC_BF16, "f32": ALSPEC_F32}.get(dtype, dtype)
     eng = ENGINES.get(engine, engine)
+    sch = SCHEDULES.get(schedule, schedule)
     return alspec_desc(batch, n_q_heads, n_kv_heads, head_dim, max_seq_len, int(code),
-                       split_tokens, timeout_ms, int(eng))
+                       split_tokens, timeout_ms, int(eng), int(sch))
 
 
 def _check(status: int, where: str):
@@ -272,11 +279,12 @@ class Decoder:
     """
 
     def __init__(self, batch, n_q_heads, n_kv_heads, head_dim, max_seq_len, dtype, n_sink,
-                 window, device=None, split_tokens=0, timeout_ms=0, engine="auto"):
+                 window, device=None, split_tokens=0, timeout_ms=0, engine="auto",
+                 schedule="auto"):
         import torch
         self.torch = torch
         self.desc = make_desc(batch, n_q_heads, n_kv_heads, head_dim, max_seq_len, dtype,
-                              split_tokens, timeout_ms, engine)
+                              split_tokens, timeout_ms, engine, schedule)
         self.n_sink, self.window = int(n_sink), int(window)
         nbytes = alspec_workspace_size(self.desc, self.n_sink, self.window)
         if nbytes == 0:

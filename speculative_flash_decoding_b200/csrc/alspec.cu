@@ -45,6 +45,10 @@ constexpr int kMaxSpecItems = kMaxSpecCtas;  // sink-set CTAs per (sequence, KV 
 #ifndef ALSPEC_MID_SM_RESERVE
 #define ALSPEC_MID_SM_RESERVE 0
 #endif
+// One-launch schedule: tiles per sink-set item at least (one round of the
+// tensor-core kernel's consumer warps), items per head at most.
+constexpr int kFusedSpecMinTiles = 4;
+constexpr int kFusedSpecMaxItems = kMaxSpecItemsFused;
 constexpr size_t kAlign = 256;
 
 thread_local cudaError_t t_last_error = cudaSuccess;
@@ -126,16 +130,23 @@ int sm_count_for_plan() {
 
 struct Plan {
     int engine;   // ALSPEC_ENGINE_CUDA_CORES or ALSPEC_ENGINE_TENSOR_CORES
+    int schedule; // ALSPEC_SCHEDULE_STREAMS or ALSPEC_SCHEDULE_FUSED
     int tt;       // tokens per pipeline tile of that engine
-    int c1, n1;   // sink-set tokens per CTA and CTAs (one cluster) per (sequence, KV head)
+    int c1, n1;   // sink-set tokens per item and items per (sequence, KV head): CTAs of
+                  // one cluster (STREAMS), queue items (FUSED)
     int c2, n2;   // first middle chunk (tokens, longest sequence) and chunks per head
     unsigned fq[kMaxChunks + 1];
     int grid1, grid2;
     int threads, smem, stages;
-    size_t off_ctr, off_spec_ml, off_spec_o, off_mid_ml, off_mid_o, off_dn, total;
+    size_t off_ctr, off_spec_ml, off_spec_o, off_spec_pml, off_spec_po, off_mid_ml, off_mid_o,
+        off_dn, total;
 };
 
 bool supported_g(int g) { return g == 1 || g == 2 || g == 4 || g == 8; }
+
+int resolve_schedule(const alspec_desc* d) {
+    return d->schedule == ALSPEC_SCHEDULE_FUSED ? ALSPEC_SCHEDULE_FUSED : ALSPEC_SCHEDULE_STREAMS;
+}
 
 int resolve_engine(const alspec_desc* d) {
     if (d->engine == ALSPEC_ENGINE_AUTO)
@@ -152,6 +163,8 @@ alspec_status check_desc(const alspec_desc* d, int S, int W) {
     if (d->dtype != ALSPEC_F32 && d->dtype != ALSPEC_BF16) return ALSPEC_ERR_INVALID_ARG;
     if (d->engine < ALSPEC_ENGINE_AUTO || d->engine > ALSPEC_ENGINE_TENSOR_CORES)
         return ALSPEC_ERR_INVALID_ARG;
+    if (d->schedule < ALSPEC_SCHEDULE_AUTO || d->schedule > ALSPEC_SCHEDULE_FUSED)
+        return ALSPEC_ERR_INVALID_ARG;
     if (d->head_dim != 64 && d->head_dim != 128) return ALSPEC_ERR_UNSUPPORTED;
     if (!supported_g(d->n_q_heads / d->n_kv_heads)) return ALSPEC_ERR_UNSUPPORTED;
     if (resolve_engine(d) == ALSPEC_ENGINE_TENSOR_CORES && d->dtype != ALSPEC_BF16)
@@ -163,7 +176,8 @@ alspec_status check_desc(const alspec_desc* d, int S, int W) {
     return ALSPEC_OK;
 }
 
-void kernel_shape(int dtype, int D, int G, int engine, int* threads, int* smem, int* stages);
+void kernel_shape(int dtype, int D, int G, int engine, bool fused, int* threads, int* smem,
+                  int* stages);
 
 // Item sizes.  The sink-set list (at most S + W tokens per head, tiled as a
 // sink run and a window run) gets one item per head when it is short (at
@@ -177,8 +191,13 @@ void kernel_shape(int dtype, int D, int G, int engine, int* threads, int* smem, 
 // fractions of each sequence's own middle, so ragged batches get the same
 // number of (proportionally smaller) items.  A caller-given split_tokens
 // instead cuts the longest middle into equal chunks of that size.
+// The one-launch schedule cuts each sink set into items of at least
+// kFusedSpecMinTiles tiles, as many per head as one CTA each in the first
+// wave allows; they precede the middle chunks in the same queue.
 void make_plan(const alspec_desc& d, int S, int W, int sms, Plan* pl) {
     pl->engine = resolve_engine(&d);
+    pl->schedule = resolve_schedule(&d);
+    const bool fused = pl->schedule == ALSPEC_SCHEDULE_FUSED;
     const int TT = pl->engine == ALSPEC_ENGINE_TENSOR_CORES ? 32 : 16;
     pl->tt = TT;
     const int heads = d.batch * d.n_kv_heads;
@@ -190,6 +209,9 @@ void make_plan(const alspec_desc& d, int S, int W, int sms, Plan* pl) {
     const int room1 = std::max(1, sms * ALSPEC_SPEC_SM_SHARE_NUM / ALSPEC_SPEC_SM_SHARE_DEN /
                                       std::max(1, heads));
     pl->n1 = std::max(1, std::min({kMaxSpecItems, room1, ceil_div(tiles_max, ALSPEC_SPEC_TILES)}));
+    if (fused)
+        pl->n1 = std::max(1, std::min({kFusedSpecMaxItems, ceil_div(tiles_max, kFusedSpecMinTiles),
+                                       std::max(1, sms / std::max(1, heads))}));
     const int tiles_per_item = ceil_div(tiles_max, pl->n1);
     pl->c1 = tiles_per_item * TT;
     pl->n1 = ceil_div(tiles_max, tiles_per_item);  // no CTA without tiles at L_max
@@ -235,10 +257,10 @@ void make_plan(const alspec_desc& d, int S, int W, int sms, Plan* pl) {
     pl->c2 = pl->n2 > 0
                  ? (int)(((unsigned long long)mid_tiles * pl->fq[1]) >> kFracBits) * TT
                  : 0;
-    const long long items2 = (long long)heads * pl->n2;
+    const long long items2 = (long long)heads * (pl->n2 + (fused ? pl->n1 : 0));
     pl->grid2 = (int)std::min<long long>(P, items2);
     const int G = d.n_q_heads / d.n_kv_heads;
-    kernel_shape(d.dtype, d.head_dim, G, pl->engine, &pl->threads, &pl->smem, &pl->stages);
+    kernel_shape(d.dtype, d.head_dim, G, pl->engine, fused, &pl->threads, &pl->smem, &pl->stages);
 
     const size_t B = d.batch, Hq = d.n_q_heads, D = d.head_dim;
     const size_t n2 = std::max(pl->n2, 1);
@@ -251,6 +273,9 @@ void make_plan(const alspec_desc& d, int S, int W, int sms, Plan* pl) {
     pl->off_ctr = take((size_t)ctr_words(d.batch, d.n_kv_heads) * sizeof(unsigned));
     pl->off_spec_ml = take(B * Hq * 2 * sizeof(float));
     pl->off_spec_o = take(B * Hq * D * sizeof(float));
+    const size_t n1p = fused ? (size_t)pl->n1 : 0;
+    pl->off_spec_pml = take(B * Hq * n1p * 2 * sizeof(float));
+    pl->off_spec_po = take(B * Hq * n1p * D * sizeof(float));
     pl->off_mid_ml = take(B * Hq * n2 * 2 * sizeof(float));
     pl->off_mid_o = take(B * Hq * n2 * D * sizeof(float));
     pl->off_dn = take(B * Hq * merge_splits(D) * 2 * sizeof(float));
@@ -264,17 +289,28 @@ using KernelFn = void (*)(Params);
 struct KernelSet {
     KernelFn spec;
     KernelFn mid;
-    int smem_spec, smem_mid;
-    int threads_spec, threads_mid;
-    int stages_mid;
+    KernelFn fused;  // the one-launch schedule's kernel
+    int smem_spec, smem_mid, smem_fused;
+    int threads_spec, threads_mid, threads_fused;
+    int stages_mid, stages_fused;
 };
 
 template <typename T, int D, int G, bool MMA>
 KernelSet kernels_for() {
     using CS = Cfg<T, D, G, true, MMA>;
     using CM = Cfg<T, D, G, false, MMA>;
-    return KernelSet{attn_kernel<T, D, G, true, MMA>, attn_kernel<T, D, G, false, MMA>,
-                     CS::kSmemBytes, CM::kSmemBytes, CS::kThreads, CM::kThreads, CM::STAGES};
+    using CF = Cfg<T, D, G, false, MMA, true>;
+    return KernelSet{attn_kernel<T, D, G, true, MMA>,
+                     attn_kernel<T, D, G, false, MMA>,
+                     attn_kernel<T, D, G, false, MMA, true>,
+                     CS::kSmemBytes,
+                     CM::kSmemBytes,
+                     CF::kSmemBytes,
+                     CS::kThreads,
+                     CM::kThreads,
+                     CF::kThreads,
+                     CM::STAGES,
+                     CF::STAGES};
 }
 
 template <typename T, int D, bool MMA>
@@ -305,12 +341,13 @@ bool pick(int dtype, int D, int G, int engine, KernelSet* ks) {
     return false;
 }
 
-void kernel_shape(int dtype, int D, int G, int engine, int* threads, int* smem, int* stages) {
+void kernel_shape(int dtype, int D, int G, int engine, bool fused, int* threads, int* smem,
+                  int* stages) {
     KernelSet ks{};
     const bool found = pick(dtype, D, G, engine, &ks);
-    *threads = found ? ks.threads_mid : 0;
-    *smem = found ? ks.smem_mid : 0;
-    *stages = found ? ks.stages_mid : 0;
+    *threads = found ? (fused ? ks.threads_fused : ks.threads_mid) : 0;
+    *smem = found ? (fused ? ks.smem_fused : ks.smem_mid) : 0;
+    *stages = found ? (fused ? ks.stages_fused : ks.stages_mid) : 0;
 }
 
 // cuTensorMapEncodeTiled from the driver, looked up once.
@@ -417,9 +454,9 @@ alspec_status alspec_query_plan(const alspec_desc* desc, int n_sink, int window,
     if (!info || n_info < 0) return ALSPEC_ERR_INVALID_ARG;
     Plan pl{};
     make_plan(*desc, n_sink, window, sm_count_for_plan(), &pl);
-    const int vals[9] = {pl.c1,      pl.n1,      pl.c2,   pl.n2,     pl.grid2,
-                         pl.threads, pl.smem,    pl.stages, pl.engine};
-    for (int i = 0; i < n_info && i < 9; ++i) info[i] = vals[i];
+    const int vals[10] = {pl.c1,      pl.n1,   pl.c2,     pl.n2,     pl.grid2,
+                          pl.threads, pl.smem, pl.stages, pl.engine, pl.schedule};
+    for (int i = 0; i < n_info && i < 10; ++i) info[i] = vals[i];
     return ALSPEC_OK;
 }
 
@@ -504,18 +541,27 @@ alspec_status decode_impl(const alspec_desc* desc, const void* q, const void* k_
     Plan pl{};
     make_plan(*desc, n_sink, window, sm_count_for_plan(), &pl);
     if (workspace_bytes < pl.total) return ALSPEC_ERR_WORKSPACE;
+    const bool fused = pl.schedule == ALSPEC_SCHEDULE_FUSED;
+    // The speculative projection needs O_spec before the launch ends.
+    if (fused && op) return ALSPEC_ERR_UNSUPPORTED;
     DeviceState* ds = nullptr;
     if ((st = get_device_state(&ds)) != ALSPEC_OK) return st;
     std::lock_guard<std::mutex> call_lock(g_call_mutex[ds - g_dev]);
     const int G = desc->n_q_heads / desc->n_kv_heads;
     KernelSet ks{};
     if (!pick(desc->dtype, desc->head_dim, G, pl.engine, &ks)) return ALSPEC_ERR_UNSUPPORTED;
-    if ((st = ensure_smem_attr(ds, reinterpret_cast<const void*>(ks.spec), ks.smem_spec)) !=
-        ALSPEC_OK)
-        return st;
-    if ((st = ensure_smem_attr(ds, reinterpret_cast<const void*>(ks.mid), ks.smem_mid)) !=
-        ALSPEC_OK)
-        return st;
+    if (fused) {
+        if ((st = ensure_smem_attr(ds, reinterpret_cast<const void*>(ks.fused), ks.smem_fused)) !=
+            ALSPEC_OK)
+            return st;
+    } else {
+        if ((st = ensure_smem_attr(ds, reinterpret_cast<const void*>(ks.spec), ks.smem_spec)) !=
+            ALSPEC_OK)
+            return st;
+        if ((st = ensure_smem_attr(ds, reinterpret_cast<const void*>(ks.mid), ks.smem_mid)) !=
+            ALSPEC_OK)
+            return st;
+    }
 
     char* ws = static_cast<char*>(workspace);
     Params p{};
@@ -542,6 +588,8 @@ alspec_status decode_impl(const alspec_desc* desc, const void* q, const void* k_
     p.ctr = reinterpret_cast<unsigned*>(ws + pl.off_ctr);
     p.spec_ml = reinterpret_cast<float*>(ws + pl.off_spec_ml);
     p.spec_o = reinterpret_cast<float*>(ws + pl.off_spec_o);
+    p.spec_pml = reinterpret_cast<float*>(ws + pl.off_spec_pml);
+    p.spec_po = reinterpret_cast<float*>(ws + pl.off_spec_po);
     p.mid_ml = reinterpret_cast<float*>(ws + pl.off_mid_ml);
     p.mid_o = reinterpret_cast<float*>(ws + pl.off_mid_o);
     p.dn = reinterpret_cast<float*>(ws + pl.off_dn);
@@ -558,6 +606,18 @@ alspec_status decode_impl(const alspec_desc* desc, const void* q, const void* k_
                ok(record_event(static_cast<cudaEvent_t>(prof_events[i]), on));
     };
     if (!prof(0, s)) return ALSPEC_ERR_CUDA;
+    if (fused) {
+        // One persistent launch; O_spec is complete (as everything else)
+        // when it ends.
+        if (!prof(2, s)) return ALSPEC_ERR_CUDA;
+        if ((st = launch(ks.fused, dim3(pl.grid2), dim3(ks.threads_fused), ks.smem_fused, s, p, 0,
+                         0)) != ALSPEC_OK)
+            return st;
+        if (!prof(3, s) || !prof(1, s)) return ALSPEC_ERR_CUDA;
+        if (spec_event && !ok(record_event(static_cast<cudaEvent_t>(spec_event), s)))
+            return ALSPEC_ERR_CUDA;
+        return prof(4, s) ? ALSPEC_OK : ALSPEC_ERR_CUDA;
+    }
     // Fork: the sink-set kernel runs on the high-priority stream.
     if (!ok(cudaEventRecord(ds->fork, s)) || !ok(cudaStreamWaitEvent(ds->hi, ds->fork, 0)))
         return ALSPEC_ERR_CUDA;
@@ -846,7 +906,7 @@ const char* alspec_status_string(alspec_status status) {
     }
 }
 
-int alspec_version(void) { return 200; }
+int alspec_version(void) { return 300; }
 
 int alspec_last_cuda_error(void) { return (int)t_last_error; }
 

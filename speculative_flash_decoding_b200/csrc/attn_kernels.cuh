@@ -79,9 +79,11 @@ constexpr int kMaxSpecCtas = 8;
 constexpr unsigned kErrSeqLen = 1u;   // ALSPEC_DEVERR_SEQ_LEN
 constexpr unsigned kErrTimeout = 2u;  // ALSPEC_DEVERR_TIMEOUT
 
-// Counter words at the head of the workspace, then the per-sequence head
-// tickets of the merge kernel [B].  Whoever takes the last ticket of a group
-// resets it, so the words are zero between calls.
+// Counter words at the head of the workspace, then the per-sequence
+// tickets [B] (merge kernel: one per CTA of the sequence; one-launch
+// schedule: one per KV head), and for the one-launch schedule the per-head
+// tile tickets [B * Hkv].  Whoever takes the last ticket of a group resets
+// it, so the words are zero between calls.
 constexpr int kCtrQueue = 0;
 constexpr int kCtrDone = 1;
 constexpr int kCtrError = 2;
@@ -91,11 +93,17 @@ __host__ __device__ __forceinline__ int ctr_seq(int B, int Hkv, int b) {
     (void)Hkv;
     return kCtrFixed + b;
 }
-__host__ __device__ __forceinline__ int ctr_words(int B, int Hkv) {
+__host__ __device__ __forceinline__ int ctr_head(int B, int Hkv, int bh) {
     (void)Hkv;
-    return kCtrFixed + B;
+    return kCtrFixed + B + bh;
+}
+__host__ __device__ __forceinline__ int ctr_words(int B, int Hkv) {
+    return kCtrFixed + B + B * Hkv;
 }
 
+// Stage metadata word w: bit 0 marks a consumer warp's last tile of the
+// item; bits 1.. hold the item's tile count (the one-launch schedule's
+// tickets count tiles).
 constexpr int kLastTileFlag = 1;
 
 // Middle work items: every (sequence, KV head) middle is cut at fixed
@@ -104,6 +112,8 @@ constexpr int kLastTileFlag = 1;
 // queue drains on small items and the CTAs finish together).
 constexpr int kMaxChunks = 256;
 constexpr int kFracBits = 24;
+// One-launch schedule: sink-set items per (sequence, KV head) at most.
+constexpr int kMaxSpecItemsFused = 64;
 
 struct Params {
     CUtensorMap tmap_k;  // 2-D views [rows = B*Hkv*Lmax, d] (tensor-core engine)
@@ -115,12 +125,15 @@ struct Params {
     int B, Hq, Hkv, Lmax, S, W;
     float qscale;   // log2(e) / sqrt(d): scores come out in the log2 domain
     float lambda;
-    int c1, n1;     // sink-set items: tokens per item, CTAs (cluster size) per (b, kv head)
+    int c1, n1;     // sink-set items: tokens per item, items per (b, kv head) (the
+                    // sink-set kernel: CTAs of one cluster)
     int n2;         // middle chunks per (b, kv head)
     unsigned fq[kMaxChunks + 1];  // chunk c covers middle tiles
                                   // [mt * fq[c] >> 24, mt * fq[c+1] >> 24)
     unsigned* ctr;
     float* spec_ml;   // [B][Hq][2]       merged sink-set partial
+    float* spec_pml;  // [B][Hq][n1][2]   sink-set item partials (one-launch schedule)
+    float* spec_po;   // [B][Hq][n1][D]
     float* spec_o;    // [B][Hq][D]
     float* mid_ml;    // [B][Hq][n2][2]   middle item partials
     float* mid_o;     // [B][Hq][n2][D]
@@ -189,22 +202,36 @@ struct Item {
     int b, kvh, chunk, ntiles;
     int t0, ns, ws, L;  // sink-set items
     int lo, hi;         // middle items
+    bool spec;          // a sink-set item
 };
 
-template <bool SPEC, int TT>
+// Which (sequence, KV head) and chunk a queue index names.  Sink-set items
+// of one head are consecutive (one cluster); middle items are chunk-major
+// across heads.  The one-launch schedule (FUSED) numbers the sink-set items
+// first, then the middle items.
+template <bool SPEC, bool FUSED>
+__device__ __forceinline__ void item_index(const Params& p, int item, bool& spec, int& bh,
+                                           int& chunk) {
+    const int heads = p.B * p.Hkv;
+    const int n_spec = FUSED ? heads * p.n1 : 0;
+    spec = SPEC || (FUSED && item < n_spec);
+    if (FUSED && !spec) item -= n_spec;
+    bh = spec ? item / p.n1 : item % heads;
+    chunk = spec ? item % p.n1 : item / heads;
+}
+
+template <bool SPEC, int TT, bool FUSED = false>
 __device__ __forceinline__ Item decode_item(const Params& p, int item, bool flag) {
     Item it;
-    // Sink-set items of one head are consecutive (one cluster); middle items
-    // are chunk-major across heads.
-    const int bh = SPEC ? item / p.n1 : item % (p.B * p.Hkv);
-    it.chunk = SPEC ? item % p.n1 : item / (p.B * p.Hkv);
+    int bh;
+    item_index<SPEC, FUSED>(p, item, it.spec, bh, it.chunk);
     it.b = bh / p.Hkv;
     it.kvh = bh % p.Hkv;
     const SeqGeom g = seq_geom(p, it.b, flag);
     it.ns = g.ns;
     it.ws = g.ws;
     it.L = g.L;
-    if (SPEC) {
+    if (SPEC || (FUSED && it.spec)) {
         const int per = p.c1 / TT;
         it.t0 = it.chunk * per;
         const int t1 = min(it.t0 + per, spec_tiles(g, TT));
@@ -222,9 +249,9 @@ __device__ __forceinline__ Item decode_item(const Params& p, int item, bool flag
 }
 
 // First cache row (within the head) and valid row count of tile t.
-template <bool SPEC, int TT>
+template <bool SPEC, int TT, bool FUSED = false>
 __device__ __forceinline__ void tile_rows(const Item& it, int t, int& start, int& nvalid) {
-    if (SPEC) {
+    if (SPEC || (FUSED && it.spec)) {
         const int tg = it.t0 + t;
         const int tsink = cdiv(it.ns, TT);
         if (tg < tsink) {
@@ -275,7 +302,7 @@ struct Elem<__nv_bfloat16> {
 //   TT    tokens per stage            GW   heads a consumer warp holds
 //   NHW   warps sharing a stage       NTW  token slots (stages per round)
 //   SPW   stages per token slot
-template <typename T, int D, int G, bool SPEC, bool MMA>
+template <typename T, int D, int G, bool SPEC, bool MMA, bool FUSED = false>
 struct Cfg {
     static constexpr int kRowBytes = D * (int)sizeof(T);
     static constexpr int TT = MMA ? 32 : 16;
@@ -302,9 +329,18 @@ struct Cfg {
     static constexpr int kGatherFloats = G * (D + 2);
     static constexpr int kGatherStride = (kGatherFloats + 3) / 4 * 4;
     static constexpr int kGatherBytes = SPEC ? kMaxSpecCtas * kGatherStride * 4 : 0;
+    // One-launch schedule: scratch for the merges done inside the kernel --
+    // the list of a sequence's non-empty middle chunks, one merge weight per
+    // (query head of the group, chunk), (weight of the sink-set partial,
+    // normaliser) per query head, the list's length, and a copy of the chunk
+    // boundary table (read with a different index per lane, which parameter
+    // space serialises).
+    static constexpr int kScratchFloats = kMaxChunks * (G + 1) + 2 * G + 4 + kMaxChunks + 4;
+    static constexpr int kScratchBytes = FUSED ? kScratchFloats * 4 : 0;
 
     static constexpr int kSpwBudget =
-        (kSmemLimit - 1024 - kDepositBytes - 4096 - 768 - kGatherBytes) / (NTW * kStageBytes);
+        (kSmemLimit - 1024 - kDepositBytes - 4096 - 768 - kGatherBytes - kScratchBytes) /
+        (NTW * kStageBytes);
     static constexpr int SPW = kSpwBudget < 1 ? 1 : (kSpwBudget > kSpwMax ? kSpwMax : kSpwBudget);
     // Tile t goes to stage t mod STAGES and to consumer warp t mod NTW, so
     // with STAGES a multiple of NTW every stage has one consumer warp, which
@@ -320,10 +356,12 @@ struct Cfg {
     static constexpr int kOffDeposit = STAGES * kStageBytes;
     static constexpr int kOffMeta = align128(kOffDeposit + kDepositBytes);
     static constexpr int kOffBar = align128(kOffMeta + STAGES * 16);
-    static constexpr int kNumBars = 2 * STAGES + 3;
+    static constexpr int kNumBars = 2 * STAGES + 4;
     static constexpr int kOffMisc = align128(kOffBar + kNumBars * 8);
     static constexpr int kOffGather = align128(kOffMisc + 16);
-    static constexpr int kSmemBytes = kOffGather + kGatherBytes + 1024;  // + alignment slack
+    static constexpr int kOffScratch = align128(kOffGather + kGatherBytes);
+    static constexpr int kSmemBytes = (FUSED ? kOffScratch + kScratchBytes : kOffGather + kGatherBytes) +
+                                      1024;  // + alignment slack
     static_assert(kOffDeposit % 1024 == 0 && kStageBytes % 1024 == 0 && kTileBytes % 1024 == 0,
                   "TMA destinations with 128-byte swizzle need 1024-byte alignment");
     static_assert(kOffMeta % 16 == 0 && kOffBar % 8 == 0 && kOffMisc % 16 == 0 &&
@@ -335,12 +373,15 @@ struct Cfg {
     static_assert(kSmemBytes <= kSmemLimit, "shared memory budget");
     static_assert(NTW >= 1 && NCW <= 8, "warp split");
     static_assert(STAGES % NTW == 0, "each stage must belong to one consumer warp");
+    static_assert(!(SPEC && FUSED), "the one-launch kernel is a middle-kernel variant");
 };
 
 // ---------------------------------------------------------------- waiting
 
 struct Shared {
     int abort;
+    int merge;  // one-launch schedule: KV head whose merges this CTA owns, or -1
+    int pad[2];
 };
 
 // Producer-side bounded wait (one thread).
@@ -892,18 +933,60 @@ __device__ __forceinline__ void cluster_gather(const Params& p, const float* dep
     cluster_wait();
 }
 
+// ------------------------------------------- relative L2 and the flag
+
+constexpr int kMergeCols = 32;  // output columns per (squared distance, squared norm) slot
+
+// Number of (squared distance, squared norm) slots per query head.
+__host__ __device__ constexpr int merge_splits(int d) { return d / kMergeCols; }
+
+// One warp, once every slot of sequence b is written and lane 0 has
+// acquired them (the sequence's last ticket):
+// rel_l2 = sqrt(sum of squared distances / sum of squared norms) over the
+// sequence's H_q * d outputs (fp64, fixed order), and the commit flag
+// rel_l2 <= lambda.  No distance and no norm gives 0 (commit); a distance
+// with a zero norm gives infinity (discard); NaN compares false (discard).
+template <int D>
+__device__ __forceinline__ void write_flag(const Params& p, int b, int lane) {
+    constexpr int NS = merge_splits(D);
+    __syncwarp();  // orders lane 0's acquire of the ticket before every lane's loads
+    double D2 = 0.0, N2 = 0.0;
+    const float2* dn = reinterpret_cast<const float2*>(p.dn) + (size_t)b * p.Hq * NS;
+    for (int i = lane; i < p.Hq * NS; i += 32) {
+        const float2 x = __ldcg(dn + i);
+        D2 += (double)x.x;
+        N2 += (double)x.y;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        D2 += __shfl_xor_sync(0xffffffffu, D2, o);
+        N2 += __shfl_xor_sync(0xffffffffu, N2, o);
+    }
+    if (lane == 0) {
+        double r;
+        if (N2 == 0.0) {
+            r = D2 == 0.0 ? 0.0 : (double)INFINITY;
+        } else {
+            r = sqrt(D2 / N2);
+        }
+        p.rel_l2[b] = (float)r;
+        p.commit[b] = r <= (double)p.lambda ? 1 : 0;
+    }
+}
+
 // Fill stage s with tile t of item `item` (meta word, barrier arrival with
 // the expected bytes, the K and V copies).  Any lane may fill any stage.
-template <typename T, int D, int G, bool SPEC, bool MMA>
+template <typename T, int D, int G, bool SPEC, bool MMA, bool FUSED>
 __device__ __forceinline__ void fill_stage(const Params& p, unsigned char* smem, int4* meta,
                                            uint64_t* full_bar, int s, int item, const Item& it,
                                            int t, int ntiles) {
-    using C = Cfg<T, D, G, SPEC, MMA>;
+    using C = Cfg<T, D, G, SPEC, MMA, FUSED>;
     constexpr int TT = C::TT;
     const int head_row = (it.b * p.Hkv + it.kvh) * p.Lmax;
     int start = 0, nvalid = 0;
-    if (t < it.ntiles) tile_rows<SPEC, TT>(it, t, start, nvalid);
-    meta[s] = make_int4(item, t, nvalid, t >= ntiles - C::NTW ? kLastTileFlag : 0);
+    if (t < it.ntiles) tile_rows<SPEC, TT, FUSED>(it, t, start, nvalid);
+    meta[s] = make_int4(item, t, nvalid,
+                        (it.ntiles << 1) | (t >= ntiles - C::NTW ? kLastTileFlag : 0));
     if (nvalid == 0) {
         mbar_arrive(full_bar + s);
         return;
@@ -934,18 +1017,19 @@ __device__ __forceinline__ void fill_stage(const Params& p, unsigned char* smem,
 // CTA's init barrier) fills the untouched stages one tile per lane, so the
 // first copies leave within a few hundred cycles; lane 0 alone continues
 // with the rest, waiting for each stage to be released.
-template <typename T, int D, int G, bool SPEC, bool MMA>
+template <typename T, int D, int G, bool SPEC, bool MMA, bool FUSED>
 __device__ __forceinline__ void produce(const Params& p, unsigned char* smem, int4* meta,
                                         uint64_t* full_bar, uint64_t* empty_bar,
                                         volatile int* abort, int lane, int item0,
                                         const Item& it0) {
-    using C = Cfg<T, D, G, SPEC, MMA>;
-    const int n_items = p.B * p.Hkv * (SPEC ? p.n1 : p.n2);
+    using C = Cfg<T, D, G, SPEC, MMA, FUSED>;
+    const int n_items = p.B * p.Hkv * (SPEC ? p.n1 : (FUSED ? p.n1 + p.n2 : p.n2));
     auto rounded = [](const Item& it) { return (it.ntiles + C::NTW - 1) / C::NTW * C::NTW; };
     const bool have0 = item0 < n_items && it0.ntiles > 0;
     const int fresh = have0 ? min(rounded(it0), C::STAGES) : 0;
     for (int t = lane; t < fresh; t += 32)
-        fill_stage<T, D, G, SPEC, MMA>(p, smem, meta, full_bar, t, item0, it0, t, rounded(it0));
+        fill_stage<T, D, G, SPEC, MMA, FUSED>(p, smem, meta, full_bar, t, item0, it0, t,
+                                              rounded(it0));
     if (lane != 0) return;
 
     uint32_t gt = (uint32_t)fresh;
@@ -959,7 +1043,7 @@ __device__ __forceinline__ void produce(const Params& p, unsigned char* smem, in
                 ok = false;
                 return;
             }
-            fill_stage<T, D, G, SPEC, MMA>(p, smem, meta, full_bar, s, item, it, t, ntiles);
+            fill_stage<T, D, G, SPEC, MMA, FUSED>(p, smem, meta, full_bar, s, item, it, t, ntiles);
         }
     };
     if (have0) run(item0, it0, fresh);
@@ -967,7 +1051,7 @@ __device__ __forceinline__ void produce(const Params& p, unsigned char* smem, in
         while (ok) {
             const int item = (int)atomicAdd(p.ctr + kCtrQueue, 1u);
             if (item >= n_items || *abort) break;
-            const Item it = decode_item<SPEC, C::TT>(p, item, true);
+            const Item it = decode_item<SPEC, C::TT, FUSED>(p, item, true);
             if (it.ntiles > 0) run(item, it, 0);
         }
     }
@@ -1005,15 +1089,346 @@ __device__ __forceinline__ void produce(const Params& p, unsigned char* smem, in
     }
 }
 
+// ------------------------------------------------ one-launch schedule merges
+//
+// In the one-launch schedule each (sequence, KV head) has a tile ticket in
+// the workspace: every item, sink-set or middle, adds its tile count when
+// its partial is written.  The CTA that completes a head merges, for the
+// group's G query heads, the sink-set item partials into O_spec (and the
+// merged sink-set partial) and that with the middle partials into O_exact,
+// writes their (squared distance, squared norm) slots, then takes a
+// per-sequence ticket; the CTA that takes a sequence's last one writes
+// rel_l2 and the flag.  Every merge runs in a fixed order, so results do
+// not depend on which CTA does it.  (O_spec is thus written at the end of
+// the head's work, not early: in one launch, nothing outside the kernel
+// could use it before the launch ends.)
+//
+// The merges run on the consumer warps of one CTA (`sync` is their barrier;
+// every consumer thread calls with the same arguments).  Tickets are taken
+// with acquire-release atomics after a barrier over the writing threads, so
+// the partials of every contributor are visible to the merging CTA (loads go
+// to L2).
+
+__device__ __forceinline__ float warp_max(float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+    return x;
+}
+// Butterfly sum: every lane ends with the same value (each step adds the
+// same two operands on both partner lanes).
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+// O_spec of one (sequence, KV head) from its sink-set item partials: per
+// query head M = max m_j, f_j = 2^(m_j - M), l = sum f_j l_j, o = sum f_j o_j
+// (items in order), O_spec = o / l; (M, l, o) is also stored as the merged
+// sink-set partial for the exact merge.
+template <class C, int D, int G, class Sync>
+__device__ __forceinline__ bool fused_spec_merge(const Params& p, int b, int kvh, float* scratch,
+                                                 int warp, int lane, Sync& sync) {
+    constexpr int NCT = C::NCW * 32;
+    constexpr int NQ = D / 4;               // float4 columns per head
+    constexpr int kJ = kMaxSpecItemsFused;  // items per head at most
+    const int ctid = warp * 32 + lane;
+    const int per = p.c1 / C::TT;
+    const int n = cdiv(spec_tiles(seq_geom(p, b, false), C::TT), per);  // items with rows
+    float* w = scratch + kMaxChunks;  // [G][kMaxChunks]
+    float* fl = w + G * kMaxChunks;   // [G][2]: M, l
+    const size_t bq0 = (size_t)b * p.Hq + kvh * G;
+    for (int hh = warp; hh < G; hh += C::NCW) {
+        const float2* ml = reinterpret_cast<const float2*>(p.spec_pml) + (bq0 + hh) * p.n1;
+        float2 x[kJ / 32];
+        float M = -INFINITY;
+#pragma unroll
+        for (int k = 0; k < kJ / 32; ++k) {
+            const int j = lane + 32 * k;
+            x[k] = j < n ? __ldcg(ml + j) : make_float2(-INFINITY, 0.f);
+            M = fmaxf(M, x[k].x);
+        }
+        M = warp_max(M);
+        float lsum = 0.f;
+#pragma unroll
+        for (int k = 0; k < kJ / 32; ++k) {
+            const int j = lane + 32 * k;
+            if (j < n) {
+                const float f = merge_weight(x[k].x, M);
+                w[hh * kMaxChunks + j] = f;
+                lsum = fmaf(f, x[k].y, lsum);
+            }
+        }
+        lsum = warp_sum(lsum);
+        if (lane == 0) {
+            fl[2 * hh] = M;
+            fl[2 * hh + 1] = lsum;
+        }
+    }
+    if (!sync()) return false;
+    // Lane j of the CTA owns 4 consecutive columns of one head; all of its
+    // item loads are issued before the sums (items in order).
+    constexpr int kB = 16;
+    for (int j = ctid; j < G * NQ; j += NCT) {
+        const int hh = j / NQ;
+        const int e4 = j % NQ;
+        const size_t bq = bq0 + hh;
+        const float4* o = reinterpret_cast<const float4*>(p.spec_po + bq * p.n1 * D) + e4;
+        const float* wh = w + hh * kMaxChunks;
+        float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int j0 = 0; j0 < n; j0 += kB) {
+            float4 v[kB];
+#pragma unroll
+            for (int u = 0; u < kB; ++u)
+                v[u] = j0 + u < n ? __ldcg(o + (size_t)(j0 + u) * NQ) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int u = 0; u < kB; ++u) {
+                if (j0 + u < n) {
+                    const float f = wh[j0 + u];
+                    O.x = fmaf(f, v[u].x, O.x);
+                    O.y = fmaf(f, v[u].y, O.y);
+                    O.z = fmaf(f, v[u].z, O.z);
+                    O.w = fmaf(f, v[u].w, O.w);
+                }
+            }
+        }
+        const float L = fl[2 * hh + 1];
+        if (e4 == 0) {
+            p.spec_ml[bq * 2] = fl[2 * hh];
+            p.spec_ml[bq * 2 + 1] = L;
+        }
+        reinterpret_cast<float4*>(p.spec_o + bq * D)[e4] = O;
+        // (out_spec need not be 16-byte aligned.)
+        float* os = p.out_spec + bq * D + 4 * e4;
+        os[0] = __fdiv_rn(O.x, L);
+        os[1] = __fdiv_rn(O.y, L);
+        os[2] = __fdiv_rn(O.z, L);
+        os[3] = __fdiv_rn(O.w, L);
+    }
+    return sync();
+}
+
+// O_exact of one (sequence, KV head): the merged sink-set partial and the
+// sequence's non-empty middle chunks (in chunk order) by the log-sum-exp
+// rule, O_exact = o / l per query head; then each head's (squared distance,
+// squared norm) against O_spec per 32 columns, and the sequence ticket.
+// With no middle chunk the sink-set partial's weight is exactly 1, so
+// O_exact is O_spec bit for bit.
+//
+// `ring` (optional): the CTA's idle stage ring (after its last item) of
+// `ring_bytes`, and `mbar` a fresh mbarrier.  When the group's middle
+// partials fit, they are pulled in with bulk copies -- loads through the
+// registers of one SM reach only a few tens of GB/s, so a head's ~180 KB
+// of partials took several microseconds that way -- and read from there.
+template <class C, int D, int G, class Sync>
+__device__ __forceinline__ bool fused_head_merge(const Params& p, int bh, float* scratch,
+                                                 int warp, int lane, Sync& sync,
+                                                 unsigned char* ring = nullptr,
+                                                 size_t ring_bytes = 0, uint64_t* mbar = nullptr,
+                                                 volatile int* abort = nullptr) {
+    constexpr int NCT = C::NCW * 32;
+    constexpr int NQ = D / 4;  // float4 columns per head
+    constexpr int NS = merge_splits(D);
+    constexpr int kU = 16;     // chunk loads each thread keeps in flight
+    constexpr int kS = 4;      // independent partial sums per column
+    static_assert(NQ % 8 == 0, "a 32-column slot is 8 lanes of float4 columns");
+    const int b = bh / p.Hkv;
+    const int kvh = bh % p.Hkv;
+    int* list = reinterpret_cast<int*>(scratch);  // [kMaxChunks]
+    float* w = scratch + kMaxChunks;               // [G][kMaxChunks]
+    float* fl = w + G * kMaxChunks;                // [G][2]: weight of the sink-set partial, l
+    int* nlist = reinterpret_cast<int*>(fl + 2 * G);
+    const unsigned* fq = reinterpret_cast<const unsigned*>(nlist + 4);  // chunk table copy
+    const size_t bq0 = (size_t)b * p.Hq + kvh * G;
+    // The group's partials [G][n2][D] are contiguous in the workspace.
+    const size_t blk_bytes = (size_t)G * p.n2 * D * sizeof(float);
+    const bool bulk = ring != nullptr && p.n2 > 0 && blk_bytes <= ring_bytes;
+    if (bulk && warp == 0) {
+        constexpr uint32_t kPiece = 16384;
+        const char* src = reinterpret_cast<const char*>(p.mid_o + bq0 * p.n2 * D);
+        // The partials were acquired through the generic proxy (ticket).
+        fence_proxy_async_global();
+        if (lane == 0) mbar_arrive_expect_tx(mbar, (uint32_t)blk_bytes);
+        __syncwarp();
+        const uint64_t pol = l2_evict_first_policy();
+        for (size_t off = (size_t)lane * kPiece; off < blk_bytes; off += 32 * (size_t)kPiece) {
+            const uint32_t nb = (uint32_t)(blk_bytes - off < kPiece ? blk_bytes - off : kPiece);
+            bulk_load(ring + off, src + off, nb, mbar, pol);
+        }
+    }
+    // O_spec and the merged sink-set partial, while the copies land.
+    if (!fused_spec_merge<C, D, G>(p, b, kvh, scratch, warp, lane, sync)) return false;
+    if (warp == 0 && lane == 0) trace_publish(p, 0);
+
+    // Non-empty chunks of this sequence's middle, in order (warp 0).
+    if (warp == 0) {
+        const int mid_tiles = cdiv(seq_geom(p, b, false).mid_len, C::TT);
+        int count = 0;
+        for (int c0 = 0; c0 < p.n2; c0 += 32) {
+            const int c = c0 + lane;
+            bool ne = false;
+            if (c < p.n2) {
+                const int lo = (int)(((unsigned long long)mid_tiles * fq[c]) >> kFracBits);
+                const int hi = (int)(((unsigned long long)mid_tiles * fq[c + 1]) >> kFracBits);
+                ne = hi > lo;
+            }
+            const unsigned bal = __ballot_sync(0xffffffffu, ne);
+            if (ne) list[count + __popc(bal & ((1u << lane) - 1u))] = c;
+            count += __popc(bal);
+        }
+        if (lane == 0) *nlist = count;
+    }
+    if (!sync()) return false;
+    const int n = *nlist;
+
+    // Per query head (one warp each): max, weights, normaliser.
+    for (int hh = warp; hh < G; hh += C::NCW) {
+        const float2 sml = __ldcg(reinterpret_cast<const float2*>(p.spec_ml) + bq0 + hh);
+        const float2* ml = reinterpret_cast<const float2*>(p.mid_ml) + (bq0 + hh) * p.n2;
+        float2 x[kMaxChunks / 32];
+        float M = sml.x;
+#pragma unroll
+        for (int k = 0; k < kMaxChunks / 32; ++k) {
+            const int i = lane + 32 * k;
+            x[k] = i < n ? __ldcg(ml + list[i]) : make_float2(-INFINITY, 0.f);
+            M = fmaxf(M, x[k].x);
+        }
+        M = warp_max(M);
+        float lsum = 0.f;
+#pragma unroll
+        for (int k = 0; k < kMaxChunks / 32; ++k) {
+            const int i = lane + 32 * k;
+            if (i < n) {
+                const float f = merge_weight(x[k].x, M);
+                w[hh * kMaxChunks + i] = f;
+                lsum = fmaf(f, x[k].y, lsum);
+            }
+        }
+        lsum = warp_sum(lsum);
+        if (lane == 0) {
+            const float f0 = merge_weight(sml.x, M);
+            fl[2 * hh] = f0;
+            fl[2 * hh + 1] = fmaf(f0, sml.y, lsum);
+        }
+    }
+    if (!sync()) return false;
+    if (bulk && !wait_warp(mbar, 0, abort, p, lane)) return false;
+
+    // Columns: lane j of the CTA owns 4 consecutive columns of one head; the
+    // 8 lanes of a 32-column slot reduce its distance and norm.
+    for (int j0 = warp * 32; j0 < G * NQ; j0 += NCT) {
+        const int j = j0 + lane;
+        const bool act = j < G * NQ;
+        const int hh = act ? j / NQ : 0;
+        const int e4 = act ? j % NQ : 0;
+        const size_t bq = bq0 + hh;
+        float dd = 0.f, nn = 0.f;
+        if (act) {
+            const float4 so = __ldcg(reinterpret_cast<const float4*>(p.spec_o + bq * D) + e4);
+            const float sl = __ldcg(p.spec_ml + bq * 2 + 1);
+            const float f0 = fl[2 * hh];
+            const float L = fl[2 * hh + 1];
+            const float* wh = w + hh * kMaxChunks;
+            float4 a = make_float4(f0 * so.x, f0 * so.y, f0 * so.z, f0 * so.w);
+            // kS interleaved sums (list position i goes to sum i mod kS),
+            // added in a fixed tree at the end: the same order on both
+            // paths, so the bits do not depend on which one the merging
+            // CTA takes.
+            float4 acc[kS];
+            acc[0] = a;
+#pragma unroll
+            for (int k = 1; k < kS; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+            auto add = [&](float4& t, float f, const float4& v) {
+                t.x = fmaf(f, v.x, t.x);
+                t.y = fmaf(f, v.y, t.y);
+                t.z = fmaf(f, v.z, t.z);
+                t.w = fmaf(f, v.w, t.w);
+            };
+            if (bulk) {
+                const float4* mo = reinterpret_cast<const float4*>(ring) + (size_t)hh * p.n2 * NQ + e4;
+                int i = 0;
+                for (; i + kS <= n; i += kS) {
+                    float4 v[kS];
+#pragma unroll
+                    for (int k = 0; k < kS; ++k) v[k] = mo[(size_t)list[i + k] * NQ];
+#pragma unroll
+                    for (int k = 0; k < kS; ++k) add(acc[k], wh[i + k], v[k]);
+                }
+#pragma unroll
+                for (int k = 0; k < kS - 1; ++k)
+                    if (i + k < n) add(acc[k], wh[i + k], mo[(size_t)list[i + k] * NQ]);
+            }
+            if (!bulk) {
+                static_assert(kU % kS == 0, "batches start at sum 0");
+                const float4* mo = reinterpret_cast<const float4*>(p.mid_o + bq * p.n2 * D) + e4;
+                for (int i0 = 0; i0 < n; i0 += kU) {
+                    float4 v[kU];
+#pragma unroll
+                    for (int u = 0; u < kU; ++u) {
+                        const int i = i0 + u;
+                        v[u] = i < n ? __ldcg(mo + (size_t)list[i] * NQ)
+                                     : make_float4(0.f, 0.f, 0.f, 0.f);
+                    }
+#pragma unroll
+                    for (int u = 0; u < kU; ++u) {
+                        const int i = i0 + u;
+                        if (i < n) add(acc[u % kS], wh[i], v[u]);
+                    }
+                }
+            }
+            static_assert(kS == 4, "the final tree below");
+            a.x = (acc[0].x + acc[1].x) + (acc[2].x + acc[3].x);
+            a.y = (acc[0].y + acc[1].y) + (acc[2].y + acc[3].y);
+            a.z = (acc[0].z + acc[1].z) + (acc[2].z + acc[3].z);
+            a.w = (acc[0].w + acc[1].w) + (acc[2].w + acc[3].w);
+            const float4 oe = make_float4(__fdiv_rn(a.x, L), __fdiv_rn(a.y, L), __fdiv_rn(a.z, L),
+                                          __fdiv_rn(a.w, L));
+            const float4 os = make_float4(__fdiv_rn(so.x, sl), __fdiv_rn(so.y, sl),
+                                          __fdiv_rn(so.z, sl), __fdiv_rn(so.w, sl));
+            // (out_exact need not be 16-byte aligned.)
+            float* ox = p.out_exact + bq * D + 4 * e4;
+            ox[0] = oe.x;
+            ox[1] = oe.y;
+            ox[2] = oe.z;
+            ox[3] = oe.w;
+            const float d0 = oe.x - os.x, d1 = oe.y - os.y, d2 = oe.z - os.z, d3 = oe.w - os.w;
+            dd = d0 * d0 + d1 * d1 + d2 * d2 + d3 * d3;
+            nn = oe.x * oe.x + oe.y * oe.y + oe.z * oe.z + oe.w * oe.w;
+        }
+#pragma unroll
+        for (int o = 1; o < 8; o <<= 1) {
+            dd += __shfl_xor_sync(0xffffffffu, dd, o);
+            nn += __shfl_xor_sync(0xffffffffu, nn, o);
+        }
+        if (act && (lane & 7) == 0)
+            *reinterpret_cast<float2*>(p.dn + (bq * NS + e4 / 8) * 2) = make_float2(dd, nn);
+    }
+    // Every slot of this head is written once this passes.
+    if (!sync()) return false;
+    if (warp == 0) {
+        unsigned last = 0;
+        if (lane == 0) {
+            unsigned* word = p.ctr + ctr_seq(p.B, p.Hkv, b);
+            const unsigned t = atom_add_acq_rel_gpu(word, 1u);
+            last = t == (unsigned)(p.Hkv - 1);
+            if (last) atomicExch(word, 0u);
+        }
+        if (__shfl_sync(0xffffffffu, last, 0)) write_flag<D>(p, b, lane);
+        if (lane == 0) trace_publish(p, 1);
+    }
+    return true;
+}
+
 // Consumer warps: compute tiles; at each item's end merge the warps' states
 // and write the item's partial (or, for the sink set, O_spec / this CTA's
 // share of it).
-template <typename T, int D, int G, bool SPEC, bool MMA>
+template <typename T, int D, int G, bool SPEC, bool MMA, bool FUSED>
 __device__ __forceinline__ void consume(const Params& p, unsigned char* smem, float* deposit,
                                         int4* meta, uint64_t* full_bar,
                                         uint64_t* empty_bar, uint64_t* dep_bar, uint64_t* free_bar,
-                                        volatile int* abort) {
-    using C = Cfg<T, D, G, SPEC, MMA>;
+                                        uint64_t* merge_bar, volatile int* abort, Shared* sh,
+                                        float* scratch) {
+    using C = Cfg<T, D, G, SPEC, MMA, FUSED>;
     using Engine = typename EngineOf<C, T, D, G, MMA>::type;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -1030,8 +1445,37 @@ __device__ __forceinline__ void consume(const Params& p, unsigned char* smem, fl
         if (lane == 0) mbar_arrive(bar);
         return wait_warp(bar, (ph++) & 1, abort, p, lane);
     };
+    auto sync = [&]() { return sync_on(dep_bar, ph_dep); };
+    const int ctid = warp * 32 + lane;
     uint32_t gt = tw;
     int b = 0, kvh = 0, chunk = 0;
+    bool spec_item = SPEC;
+    if (FUSED) {
+        // The chunk boundary table, for the merges' per-lane lookups.
+        unsigned* fq = reinterpret_cast<unsigned*>(scratch) + kMaxChunks * (G + 1) + 2 * G + 4;
+        for (int i = ctid; i <= kMaxChunks; i += C::NCW * 32) fq[i] = p.fq[i];
+    }
+    // One-launch schedule: thread 0's head ticket still in flight (taken at
+    // an item's end, looked at by the next one), and its resolution into
+    // sh->merge (the head whose merges this CTA owns, or -1).
+    int pend_bh = -1;
+    unsigned pend_old = 0, pend_target = 0;
+    auto take_head_ticket = [&](int bh, int bb, unsigned add) {
+        const SeqGeom g = seq_geom(p, bb, false);
+        const unsigned total = (unsigned)(cdiv(g.mid_len, C::TT) + spec_tiles(g, C::TT));
+        pend_old = atom_add_acq_rel_gpu(p.ctr + ctr_head(p.B, p.Hkv, bh), add);
+        pend_target = total - add;
+        pend_bh = bh;
+    };
+    auto resolve_head_ticket = [&]() {
+        int m = -1;
+        if (pend_bh >= 0 && pend_old == pend_target) {
+            atomicExch(p.ctr + ctr_head(p.B, p.Hkv, pend_bh), 0u);
+            m = pend_bh;
+        }
+        pend_bh = -1;
+        sh->merge = m;
+    };
     if (SPEC && p.n1 > 1) {
         // Empty state (m = -inf, l = 0, o = 0) in this warp's deposit slot:
         // a CTA whose slice of a short sink set has no tiles contributes
@@ -1058,8 +1502,8 @@ __device__ __forceinline__ void consume(const Params& p, unsigned char* smem, fl
         const int4 mt = meta[s];
         if (mt.x < 0) break;
         if (!SPEC && mt.y < C::NTW) {
-            const int bh = mt.x % (p.B * p.Hkv);
-            chunk = mt.x / (p.B * p.Hkv);
+            int bh;
+            item_index<SPEC, FUSED>(p, mt.x, spec_item, bh, chunk);
             b = bh / p.Hkv;
             kvh = bh % p.Hkv;
             st.load_query(p, b, kvh * G + hw * C::GW, lane);
@@ -1083,12 +1527,16 @@ __device__ __forceinline__ void consume(const Params& p, unsigned char* smem, fl
             __syncwarp();
             continue;
         }
+        if (FUSED && ctid == 0) resolve_head_ticket();
         if (!sync_on(dep_bar, ph_dep)) break;
+        // Read before the next barrier: thread 0 rewrites it only after that.
+        const int merge_bh = FUSED ? sh->merge : -1;
         {
-            const int ctid = warp * 32 + lane;
-            float* part_ml = p.mid_ml;
-            float* part_o = p.mid_o;
-            const int per = SPEC ? p.n1 : p.n2;
+            // The one-launch schedule keeps sink-set item partials apart.
+            const bool sp = FUSED && spec_item;
+            float* part_ml = sp ? p.spec_pml : p.mid_ml;
+            float* part_o = sp ? p.spec_po : p.mid_o;
+            const int per = SPEC || sp ? p.n1 : p.n2;
             for (int idx = ctid; idx < G * D; idx += C::NCW * 32) {
                 const int hh = idx / D;
                 const int e = idx % D;
@@ -1128,15 +1576,35 @@ __device__ __forceinline__ void consume(const Params& p, unsigned char* smem, fl
         // Every consumer thread's partial is written (and the deposit slots
         // are free again) once this sync passes.
         if (!sync_on(free_bar, ph_free)) break;
+        if (FUSED) {
+            // A head completed by this CTA's previous item: merge it now (the
+            // ring is busy; rare, heads complete at the end of the queue).
+            if (merge_bh >= 0 && !fused_head_merge<C, D, G>(p, merge_bh, scratch, warp, lane, sync))
+                break;
+            if (ctid == 0) take_head_ticket(b * p.Hkv + kvh, b, (unsigned)mt.w >> 1);
+        }
         st.reset();
+    }
+    if (FUSED) {
+        // The head ticket of this CTA's last item may be the last one.
+        if (ctid == 0) resolve_head_ticket();
+        if (sync()) {
+            // The producer has stopped and every stage was consumed: the
+            // ring is free for the merge's bulk copies.
+            const int merge_bh = sh->merge;
+            if (merge_bh >= 0)
+                (void)fused_head_merge<C, D, G>(p, merge_bh, scratch, warp, lane, sync, smem,
+                                                (size_t)C::STAGES * C::kStageBytes, merge_bar,
+                                                abort);
+        }
     }
 }
 // ------------------------------------------------------------ the kernel
 
-template <typename T, int D, int G, bool SPEC, bool MMA>
-__global__ void __launch_bounds__(Cfg<T, D, G, SPEC, MMA>::kThreads, 1)
+template <typename T, int D, int G, bool SPEC, bool MMA, bool FUSED = false>
+__global__ void __launch_bounds__(Cfg<T, D, G, SPEC, MMA, FUSED>::kThreads, 1)
     attn_kernel(const __grid_constant__ Params p) {
-    using C = Cfg<T, D, G, SPEC, MMA>;
+    using C = Cfg<T, D, G, SPEC, MMA, FUSED>;
     extern __shared__ unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -1147,9 +1615,11 @@ __global__ void __launch_bounds__(Cfg<T, D, G, SPEC, MMA>::kThreads, 1)
     uint64_t* dep_bar = empty_bar + C::STAGES;  // consumer warps: phase sync
     uint64_t* free_bar = dep_bar + 1;           // consumer warps: writes done
     uint64_t* gather_bar = free_bar + 1;        // sink-set cluster leader: partials in
+    uint64_t* merge_bar = gather_bar + 1;       // one-launch schedule: final merge's copies
     Shared* sh = reinterpret_cast<Shared*>(smem + C::kOffMisc);
     volatile int* abort = &sh->abort;
     float* gather = reinterpret_cast<float*>(smem + C::kOffGather);
+    float* scratch = reinterpret_cast<float*>(smem + C::kOffScratch);
     // Sink-set kernel with several CTAs per head: those CTAs are one cluster.
     const bool clustered = SPEC && p.n1 > 1;
 
@@ -1164,15 +1634,17 @@ __global__ void __launch_bounds__(Cfg<T, D, G, SPEC, MMA>::kThreads, 1)
         mbar_init(dep_bar, C::NCW);
         mbar_init(free_bar, C::NCW);
         mbar_init(gather_bar, 1);
+        mbar_init(merge_bar, 1);
         // Every CTA of a cluster receives every CTA's slot as transaction bytes.
         if (clustered) mbar_arrive_expect_tx(gather_bar, (uint32_t)(p.n1 * C::kGatherStride * 4));
         sh->abort = 0;
+        sh->merge = -1;
         fence_barrier_init();
     }
     // The producer warp fetches the tensor maps and takes its first item now,
     // so that those loads, the queue ticket and the sequence-length load
     // overlap the barrier set-up.
-    const int n_items = p.B * p.Hkv * (SPEC ? p.n1 : p.n2);
+    const int n_items = p.B * p.Hkv * (SPEC ? p.n1 : (FUSED ? p.n1 + p.n2 : p.n2));
     int item0 = n_items;
     Item it0{};
     if (warp == C::NCW) {
@@ -1187,23 +1659,24 @@ __global__ void __launch_bounds__(Cfg<T, D, G, SPEC, MMA>::kThreads, 1)
             if (lane == 0) v = atomicAdd(p.ctr + kCtrQueue, 1u);
             item0 = (int)__shfl_sync(0xffffffffu, v, 0);
         }
-        if (item0 < n_items) it0 = decode_item<SPEC, C::TT>(p, item0, lane == 0);
+        if (item0 < n_items) it0 = decode_item<SPEC, C::TT, FUSED>(p, item0, lane == 0);
     }
     // The merge kernel that follows this (middle) kernel may be resident
     // already: it only prepares until this grid has completed.
-    if (!SPEC) pdl_launch_dependents();
+    if (!SPEC && !FUSED) pdl_launch_dependents();
     __syncthreads();
     if (clustered) cluster_arrive_relaxed();  // this CTA's barriers are set up
 
     if (warp == C::NCW) {
         // ---------------------------------------------------- producer
-        produce<T, D, G, SPEC, MMA>(p, smem, meta, full_bar, empty_bar, abort, lane, item0, it0);
+        produce<T, D, G, SPEC, MMA, FUSED>(p, smem, meta, full_bar, empty_bar, abort, lane, item0,
+                                           it0);
         if (!clustered) return;
         cluster_wait_any();  // the cluster's barriers are set up
         __syncwarp();  // the warp waits for its producer lane, then joins the cluster merge
     } else {
-        consume<T, D, G, SPEC, MMA>(p, smem, deposit, meta, full_bar, empty_bar, dep_bar,
-                                    free_bar, abort);
+        consume<T, D, G, SPEC, MMA, FUSED>(p, smem, deposit, meta, full_bar, empty_bar, dep_bar,
+                                           free_bar, merge_bar, abort, sh, scratch);
     }
     if (SPEC && !clustered && warp < C::NCW && p.trace) {
         // One CTA per head: its consumer warps wrote O_spec.
@@ -1219,13 +1692,10 @@ __global__ void __launch_bounds__(Cfg<T, D, G, SPEC, MMA>::kThreads, 1)
 
 // ------------------------------------------------------- merge + verify
 
-constexpr int kMergeCols = 32;   // output columns per CTA (one per lane)
 constexpr int kMergeParts = 8;   // warps per CTA, each over every 8th chunk
 constexpr int kMergeBatch = 32;  // chunk loads each thread keeps in flight
 constexpr int kMergeThreads = kMergeCols * kMergeParts;
 
-// Number of (squared distance, squared norm) slots per query head.
-__host__ __device__ constexpr int merge_splits(int d) { return d / kMergeCols; }
 
 // One CTA per (32 output columns of a query head, sequence): lane e of warp
 // `part` owns column split * 32 + e over the chunks list[part],
@@ -1361,30 +1831,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const __grid_const
             last = t == (unsigned)(p.Hq * NS - 1);
             if (last) atomicExch(word, 0u);
         }
-        if (__shfl_sync(0xffffffffu, lane == 0 ? last : 0, 0)) {
-            double D2 = 0.0, N2 = 0.0;
-            const float2* dn = reinterpret_cast<const float2*>(p.dn) + (size_t)b * p.Hq * NS;
-            for (int i = lane; i < p.Hq * NS; i += 32) {
-                const float2 x = __ldcg(dn + i);
-                D2 += (double)x.x;
-                N2 += (double)x.y;
-            }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                D2 += __shfl_xor_sync(0xffffffffu, D2, o);
-                N2 += __shfl_xor_sync(0xffffffffu, N2, o);
-            }
-            if (lane == 0) {
-                double r;
-                if (N2 == 0.0) {
-                    r = D2 == 0.0 ? 0.0 : (double)INFINITY;
-                } else {
-                    r = sqrt(D2 / N2);
-                }
-                p.rel_l2[b] = (float)r;
-                p.commit[b] = r <= (double)p.lambda ? 1 : 0;
-            }
-        }
+        if (__shfl_sync(0xffffffffu, lane == 0 ? last : 0, 0)) write_flag<D>(p, b, lane);
         if (lane == 0) trace_publish(p, 1);
     }
 }

@@ -33,7 +33,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_version_and_status_strings():
-    assert sfd.alspec_version() == 200
+    assert sfd.alspec_version() == 300
     for st in range(7):
         assert sfd.alspec_status_string(st) and "unknown" not in sfd.alspec_status_string(st)
     assert "unknown" in sfd.alspec_status_string(99)

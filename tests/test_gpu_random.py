@@ -3,7 +3,7 @@
 Each case draws a batch, KV head count, group size, head size, dtype and
 engine, a ragged set of lengths (1 token and up), a sink and a window (either
 may be 0), a split size and a threshold, and compares the CUDA path with the
-fp64 oracle on the same bits.
+fp64 oracle on the same bits, under both launch schedules.
 """
 import numpy as np
 import pytest
@@ -38,8 +38,9 @@ def _case(seed):
     return wl, lens, engine, split
 
 
+@pytest.mark.parametrize("schedule", ["streams", "fused"])
 @pytest.mark.parametrize("seed", range(24))
-def test_random_shapes_match_oracle(cuda_device, seed):
+def test_random_shapes_match_oracle(cuda_device, seed, schedule):
     wl, lens, engine, split = _case(seed)
     data = workloads.make_layer(wl, device=cuda_device, poison_tail=True)
     data["lens"] = lens
@@ -48,8 +49,9 @@ def test_random_shapes_match_oracle(cuda_device, seed):
     for b, L in enumerate(lens):
         data["k"][b, :, L:, :] = float("nan")
         data["v"][b, :, L:, :] = float("nan")
-    dec, out = gpu_decode(wl, data, cuda_device, engine=engine, split_tokens=split)
-    what = (f"seed {seed}: B{wl.B} Hkv{wl.Hkv} g{wl.g} d{wl.d} {wl.dtype} {engine} "
+    dec, out = gpu_decode(wl, data, cuda_device, engine=engine, split_tokens=split,
+                          schedule=schedule)
+    what = (f"{schedule} seed {seed}: B{wl.B} Hkv{wl.Hkv} g{wl.g} d{wl.d} {wl.dtype} {engine} "
             f"L{lens} S{wl.S} W{wl.W} split {split} lam {wl.lam}")
     assert_parity(out, oracle_decode(wl, data), wl.lam, what=what)
     for b, L in enumerate(lens):
