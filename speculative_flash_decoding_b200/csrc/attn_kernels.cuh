@@ -102,7 +102,7 @@ __host__ __device__ __forceinline__ int ctr_words(int B, int Hkv) {
 }
 
 // Stage metadata word w: bit 0 marks a consumer warp's last tile of the
-// item; bits 1.. hold the item's tile count (the one-launch schedule's
+// item; in the one-launch schedule bits 1.. hold the item's tile count (its
 // tickets count tiles).
 constexpr int kLastTileFlag = 1;
 
@@ -986,7 +986,7 @@ __device__ __forceinline__ void fill_stage(const Params& p, unsigned char* smem,
     int start = 0, nvalid = 0;
     if (t < it.ntiles) tile_rows<SPEC, TT, FUSED>(it, t, start, nvalid);
     meta[s] = make_int4(item, t, nvalid,
-                        (it.ntiles << 1) | (t >= ntiles - C::NTW ? kLastTileFlag : 0));
+                        (FUSED ? it.ntiles << 1 : 0) | (t >= ntiles - C::NTW ? kLastTileFlag : 0));
     if (nvalid == 0) {
         mbar_arrive(full_bar + s);
         return;
