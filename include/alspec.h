@@ -175,10 +175,12 @@ alspec_status alspec_workspace_init(void* workspace, size_t workspace_bytes, voi
  *               [1]-[0] is the latency of O_spec, [3]-[2] the duration of
  *               the middle kernel, [4]-[0] the latency of the whole step.
  *
- * The sink-set attention runs on a high-priority stream forked from
- * `stream` with events; the rest runs on `stream`.  Safe to capture in a
- * CUDA graph (no host synchronization, no allocation).  With
- * L_b <= S + W the two outputs are bit-identical and rel_l2 is exactly 0.
+ * STREAMS schedule: the sink-set attention runs on a high-priority stream
+ * forked from `stream` with events; the rest runs on `stream`.  FUSED
+ * schedule: one launch on `stream`; spec_event and prof_events [1]-[3] are
+ * recorded around it.  Safe to capture in a CUDA graph (no host
+ * synchronization, no allocation).  With L_b <= S + W the two outputs are
+ * bit-identical and rel_l2 is exactly 0.
  */
 alspec_status alspec_decode(const alspec_desc* desc,
                             const void* q, const void* k_cache, const void* v_cache,
