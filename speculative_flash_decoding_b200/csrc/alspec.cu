@@ -38,9 +38,24 @@ constexpr int kMaxSpecItems = kMaxSpecCtas;  // sink-set CTAs per (sequence, KV 
 #ifndef ALSPEC_SPEC_SM_SHARE_DEN
 #define ALSPEC_SPEC_SM_SHARE_DEN 4
 #endif
-// Smallest middle chunk of the guided self-scheduled split, in tiles.
+// Smallest middle chunk of the guided self-scheduled split, in tiles, and
+// the divisor of its chunk size (chunk c takes H * r_c / (DIV * P) of each
+// head's middle): DIV_SINGLE for a batch of one sequence, DIV otherwise.
+// Chunk boundaries are fractions of each sequence's own middle and the plan
+// sees only max_seq_len, so in a batch the longest sequence's first chunks
+// exceed a CTA's fair share of the real work by L_max / L_mean; DIV 1.5
+// leaves room for that.  One sequence cannot be ragged, and there a first
+// chunk of a whole fair share (DIV 1) means fewer items and partials:
+// measured on the 32 x 128K step 2760 us against 2823 us with 1.5, while
+// 1.0 cost 16% on the ragged batch of 8 (16K-64K).
 #ifndef ALSPEC_GSS_MIN_TILES
 #define ALSPEC_GSS_MIN_TILES 16
+#endif
+#ifndef ALSPEC_GSS_DIV
+#define ALSPEC_GSS_DIV 1.5
+#endif
+#ifndef ALSPEC_GSS_DIV_SINGLE
+#define ALSPEC_GSS_DIV_SINGLE 1.0
 #endif
 #ifndef ALSPEC_MID_SM_RESERVE
 #define ALSPEC_MID_SM_RESERVE 0
@@ -180,13 +195,15 @@ void kernel_shape(int dtype, int D, int G, int engine, bool fused, int* threads,
                   int* stages);
 
 // Item sizes.  The sink-set list (at most S + W tokens per head, tiled as a
-// sink run and a window run) gets one item per head when it is short (at
-// most 64 tiles): that CTA publishes O_spec with no cross-CTA merge.  Long
-// sink sets are cut into a few items, with at most a quarter of the SMs for
-// the sink-set kernel overall.  The persistent middle kernel takes the
-// remaining SMs (at least three quarters), so both kernels start at once.
+// sink run and a window run) is cut into n1 items of about
+// ALSPEC_SPEC_TILES tiles, one CTA each, the n1 CTAs of a head forming one
+// thread-block cluster (n1 <= 8, the portable cluster size), with all heads
+// together within ALSPEC_SPEC_SM_SHARE of the SMs; n1 = 1 needs no
+// cross-CTA merge.  The persistent middle kernel takes every SM: its CTAs
+// that find an SM busy with the (short) sink-set kernel start when it is
+// done, and its atomic queue balances the work.
 // Middle chunks follow guided self-scheduling: with H heads sharing each
-// chunk index and P CTAs, chunk c takes H * r_c / (1.5 P) of what is left
+// chunk index and P CTAs, chunk c takes H * r_c / (DIV P) of what is left
 // of a head's middle (r_c), never less than 16 tiles; chunk boundaries are
 // fractions of each sequence's own middle, so ragged batches get the same
 // number of (proportionally smaller) items.  A caller-given split_tokens
@@ -232,9 +249,10 @@ void make_plan(const alspec_desc& d, int S, int W, int sms, Plan* pl) {
             for (int c = 0; c < n; ++c) sizes.push_back((double)ct / mid_tiles);
         } else {
             const double smin = std::min(1.0, (double)ALSPEC_GSS_MIN_TILES / mid_tiles);
+            const double div = d.batch == 1 ? ALSPEC_GSS_DIV_SINGLE : ALSPEC_GSS_DIV;
             double r = 1.0;
             while (r > 1e-9 && (int)sizes.size() < kMaxChunks) {
-                double s = std::max((double)heads * r / (1.5 * P), smin);
+                double s = std::max((double)heads * r / (div * P), smin);
                 s = std::min(s, r);
                 sizes.push_back(s);
                 r -= s;
