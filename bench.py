@@ -31,9 +31,12 @@ sys.path.insert(0, ROOT)
 
 METRIC = "KV GB/s (fraction of HBM peak) and µs/decode-step to commit flag at 128K"
 FALLBACK_HBM_GBS = 6650.0
-MID_KERNEL_SRC = os.path.join(ROOT, "speculative_flash_decoding_b200", "csrc", "attn_kernels.cuh")
+# The sources a stored ncu traffic figure depends on: the kernels and the
+# host planner (which sets the items and partials each launch writes).
+KERNEL_SRCS = [os.path.join(ROOT, "speculative_flash_decoding_b200", "csrc", f)
+               for f in ("attn_kernels.cuh", "alspec.cu")]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_mid_llama8b_128k_traffic.md")
-FUSED_TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_fused_llama8b_128k_traffic.md")
+FUSED_TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_fused_llama8b_128k_ncu.md")
 
 
 NOMINAL_HBM_GBS = 8000.0  # the HBM3e figure the target is stated against
@@ -127,7 +130,8 @@ def measured_peak():
 
 def stored_traffic(path):
     """DRAM bytes per launch of the dominant kernel from a committed ncu
-    summary, or None when the kernel source changed since it was captured."""
+    summary, or None when the kernel or planner source changed since it was
+    captured (`source_sha256` is over the files in KERNEL_SRCS, in order)."""
     try:
         text = open(path).read()
     except OSError:
@@ -136,7 +140,10 @@ def stored_traffic(path):
     m_bytes = re.search(r"dram_bytes_per_launch:\s*([0-9]+)", text)
     if not (m_hash and m_bytes):
         return None
-    src = hashlib.sha256(open(MID_KERNEL_SRC, "rb").read()).hexdigest()
+    h = hashlib.sha256()
+    for f in KERNEL_SRCS:
+        h.update(open(f, "rb").read())
+    src = h.hexdigest()
     return int(m_bytes.group(1)) if src == m_hash.group(1) else None
 
 
