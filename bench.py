@@ -57,9 +57,11 @@ def parse_args():
     ap.add_argument("--split-tokens", type=int, default=0,
                     help="exact-path item size for the longest sequence (0 = library's choice)")
     ap.add_argument("--engine", default="auto", choices=["auto", "cuda_cores", "tensor_cores"])
-    ap.add_argument("--schedule", default="auto", choices=["auto", "streams", "fused"],
-                    help="launch schedule: streams (sink set on a high-priority stream, three "
-                         "kernels) or fused (one persistent launch); auto = streams")
+    ap.add_argument("--schedule", default="auto",
+                    choices=["auto", "streams", "fused", "sink_first"],
+                    help="launch schedule: streams (sink set on a high-priority stream beside "
+                         "the exact path, three kernels), fused (one persistent launch) or "
+                         "sink_first (sink set alone first); auto = streams")
     ap.add_argument("--oproj", action="store_true",
                     help="speculative output projection against the serial one (32 x 128K)")
     ap.add_argument("--lambda-sweep", action="store_true",
@@ -559,7 +561,7 @@ def run_alspec(args, wl):
                    "timing": "CUDA graph per step, CUDA events on the launch stream; "
                              "per-kernel times from a second pass of graphs with per-layer "
                              "events",
-                   "schedule": "fused" if fused else "streams",
+                   "schedule": {1: "streams", 2: "fused", 3: "sink_first"}[plan["schedule"]],
                    "plan": plan},
         "roofline": {"bound": "hbm",
                      "kernel": "attn_kernel<%s,%d,%d,%s,%s>" % (

@@ -79,11 +79,16 @@ typedef enum {
  *            writes rel_l2 and the flag (ticket counters in the workspace).
  *            O_spec is complete only when the launch ends (spec_event marks
  *            that point); alspec_decode_oproj is not available with it.
+ *   SINK_FIRST: as STREAMS, but the sink-set kernel runs alone first on the
+ *            caller's stream with every SM, and the exact-path kernel after
+ *            it: O_spec sooner when the sink set is large (many sequences or
+ *            a long window), at some cost in throughput.
  */
 typedef enum {
     ALSPEC_SCHEDULE_AUTO = 0,     /* STREAMS */
     ALSPEC_SCHEDULE_STREAMS = 1,
-    ALSPEC_SCHEDULE_FUSED = 2
+    ALSPEC_SCHEDULE_FUSED = 2,
+    ALSPEC_SCHEDULE_SINK_FIRST = 3
 } alspec_schedule;
 
 /* Gating of the recomputation in alspec_decode_oproj. */

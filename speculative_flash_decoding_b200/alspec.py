@@ -45,6 +45,7 @@ ALSPEC_ENGINE_TENSOR_CORES = 2
 ALSPEC_SCHEDULE_AUTO = 0
 ALSPEC_SCHEDULE_STREAMS = 1
 ALSPEC_SCHEDULE_FUSED = 2
+ALSPEC_SCHEDULE_SINK_FIRST = 3
 
 
 class alspec_desc(ctypes.Structure):
@@ -253,7 +254,7 @@ def alspec_last_cuda_error() -> int:
 ENGINES = {"auto": ALSPEC_ENGINE_AUTO, "cuda_cores": ALSPEC_ENGINE_CUDA_CORES,
            "tensor_cores": ALSPEC_ENGINE_TENSOR_CORES}
 SCHEDULES = {"auto": ALSPEC_SCHEDULE_AUTO, "streams": ALSPEC_SCHEDULE_STREAMS,
-             "fused": ALSPEC_SCHEDULE_FUSED}
+             "fused": ALSPEC_SCHEDULE_FUSED, "sink_first": ALSPEC_SCHEDULE_SINK_FIRST}
 
 
 def make_desc(batch, n_q_heads, n_kv_heads, head_dim, max_seq_len, dtype, split_tokens=0,

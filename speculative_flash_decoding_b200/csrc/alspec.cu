@@ -152,6 +152,7 @@ struct Plan {
     int c2, n2;   // first middle chunk (tokens, longest sequence) and chunks per head
     unsigned fq[kMaxChunks + 1];
     int grid1, grid2;
+    bool sink_first;  // SINK_FIRST: the sink-set kernel alone first, then the middle kernel
     int threads, smem, stages;
     size_t off_ctr, off_spec_ml, off_spec_o, off_spec_pml, off_spec_po, off_mid_ml, off_mid_o,
         off_dn, total;
@@ -160,7 +161,7 @@ struct Plan {
 bool supported_g(int g) { return g == 1 || g == 2 || g == 4 || g == 8; }
 
 int resolve_schedule(const alspec_desc* d) {
-    return d->schedule == ALSPEC_SCHEDULE_FUSED ? ALSPEC_SCHEDULE_FUSED : ALSPEC_SCHEDULE_STREAMS;
+    return d->schedule == ALSPEC_SCHEDULE_AUTO ? ALSPEC_SCHEDULE_STREAMS : d->schedule;
 }
 
 int resolve_engine(const alspec_desc* d) {
@@ -178,7 +179,7 @@ alspec_status check_desc(const alspec_desc* d, int S, int W) {
     if (d->dtype != ALSPEC_F32 && d->dtype != ALSPEC_BF16) return ALSPEC_ERR_INVALID_ARG;
     if (d->engine < ALSPEC_ENGINE_AUTO || d->engine > ALSPEC_ENGINE_TENSOR_CORES)
         return ALSPEC_ERR_INVALID_ARG;
-    if (d->schedule < ALSPEC_SCHEDULE_AUTO || d->schedule > ALSPEC_SCHEDULE_FUSED)
+    if (d->schedule < ALSPEC_SCHEDULE_AUTO || d->schedule > ALSPEC_SCHEDULE_SINK_FIRST)
         return ALSPEC_ERR_INVALID_ARG;
     if (d->head_dim != 64 && d->head_dim != 128) return ALSPEC_ERR_UNSUPPORTED;
     if (!supported_g(d->n_q_heads / d->n_kv_heads)) return ALSPEC_ERR_UNSUPPORTED;
@@ -223,8 +224,12 @@ void make_plan(const alspec_desc& d, int S, int W, int sms, Plan* pl) {
     // CTAs per head for the sink set (one thread-block cluster): about
     // ALSPEC_SPEC_TILES tiles each, at most 8 (the portable cluster size),
     // and all heads together within ALSPEC_SPEC_SM_SHARE of the SMs.
-    const int room1 = std::max(1, sms * ALSPEC_SPEC_SM_SHARE_NUM / ALSPEC_SPEC_SM_SHARE_DEN /
-                                      std::max(1, heads));
+    // SINK_FIRST: the sink-set kernel runs alone, so it may take every SM.
+    pl->sink_first = pl->schedule == ALSPEC_SCHEDULE_SINK_FIRST;
+    const int share_sms = pl->sink_first
+                              ? sms
+                              : sms * ALSPEC_SPEC_SM_SHARE_NUM / ALSPEC_SPEC_SM_SHARE_DEN;
+    const int room1 = std::max(1, share_sms / std::max(1, heads));
     pl->n1 = std::max(1, std::min({kMaxSpecItems, room1, ceil_div(tiles_max, ALSPEC_SPEC_TILES)}));
     if (fused)
         pl->n1 = std::max(1, std::min({kFusedSpecMaxItems, ceil_div(tiles_max, kFusedSpecMinTiles),
@@ -636,17 +641,21 @@ alspec_status decode_impl(const alspec_desc* desc, const void* q, const void* k_
             return ALSPEC_ERR_CUDA;
         return prof(4, s) ? ALSPEC_OK : ALSPEC_ERR_CUDA;
     }
-    // Fork: the sink-set kernel runs on the high-priority stream.
-    if (!ok(cudaEventRecord(ds->fork, s)) || !ok(cudaStreamWaitEvent(ds->hi, ds->fork, 0)))
+    // Fork: the sink-set kernel runs on the high-priority stream, beside the
+    // middle kernel -- or (SINK_FIRST) alone first on the caller's stream,
+    // the middle kernel following it there.
+    cudaStream_t ss = pl.sink_first ? s : ds->hi;
+    if (!pl.sink_first &&
+        (!ok(cudaEventRecord(ds->fork, s)) || !ok(cudaStreamWaitEvent(ds->hi, ds->fork, 0))))
         return ALSPEC_ERR_CUDA;
     const dim3 grid1(pl.grid1);
-    if ((st = launch(ks.spec, grid1, dim3(ks.threads_spec), ks.smem_spec, ds->hi, p,
-                     kLaunchHighPriority, ds->prio_hi, pl.n1)) != ALSPEC_OK)
+    if ((st = launch(ks.spec, grid1, dim3(ks.threads_spec), ks.smem_spec, ss, p,
+                     pl.sink_first ? 0 : kLaunchHighPriority, ds->prio_hi, pl.n1)) != ALSPEC_OK)
         return st;
-    if (spec_event && !ok(record_event(static_cast<cudaEvent_t>(spec_event), ds->hi)))
+    if (spec_event && !ok(record_event(static_cast<cudaEvent_t>(spec_event), ss)))
         return ALSPEC_ERR_CUDA;
-    if (!prof(1, ds->hi)) return ALSPEC_ERR_CUDA;
-    if (!ok(cudaEventRecord(ds->join, ds->hi))) return ALSPEC_ERR_CUDA;
+    if (!prof(1, ss)) return ALSPEC_ERR_CUDA;
+    if (!ok(cudaEventRecord(ds->join, ss))) return ALSPEC_ERR_CUDA;
     const int kdim = desc->n_q_heads * desc->head_dim;
     if (op) {
         // Speculative output projection of O_spec, beside the exact path, on

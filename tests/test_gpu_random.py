@@ -3,7 +3,7 @@
 Each case draws a batch, KV head count, group size, head size, dtype and
 engine, a ragged set of lengths (1 token and up), a sink and a window (either
 may be 0), a split size and a threshold, and compares the CUDA path with the
-fp64 oracle on the same bits, under both launch schedules.
+fp64 oracle on the same bits, under each launch schedule.
 """
 import numpy as np
 import pytest
@@ -38,7 +38,7 @@ def _case(seed):
     return wl, lens, engine, split
 
 
-@pytest.mark.parametrize("schedule", ["streams", "fused"])
+@pytest.mark.parametrize("schedule", ["streams", "fused", "sink_first"])
 @pytest.mark.parametrize("seed", range(24))
 def test_random_shapes_match_oracle(cuda_device, seed, schedule):
     wl, lens, engine, split = _case(seed)

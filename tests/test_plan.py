@@ -135,7 +135,7 @@ CASES = [
 
 @pytest.mark.parametrize("case", CASES)
 @pytest.mark.parametrize("engine", ["auto", "cuda_cores"])
-@pytest.mark.parametrize("schedule", ["streams", "fused"])
+@pytest.mark.parametrize("schedule", ["streams", "fused", "sink_first"])
 def test_every_row_read_exactly_once(case, engine, schedule):
     B, Hq, Hkv, d, Lmax, dtype, S, W = case
     rng = random.Random(hash(case) & 0xffff)
@@ -143,6 +143,23 @@ def test_every_row_read_exactly_once(case, engine, schedule):
         lens = [rng.randint(1, Lmax) for _ in range(B)]
         lens[0] = Lmax
         tiles_of(B, Hq, Hkv, d, Lmax, dtype, S, W, lens, engine=engine, schedule=schedule)
+
+
+def test_sink_first_plan_takes_every_sm_for_the_sink_set():
+    """SINK_FIRST runs the sink-set kernel alone, so its clusters may cover
+    every SM; the concurrent schedule keeps them within 3/4 of the SMs."""
+    for B, Hkv, W in [(8, 8, 2048), (4, 8, 4096), (1, 8, 1024)]:
+        plans = {}
+        for sch in ("streams", "sink_first"):
+            desc = sfd.make_desc(B, 4 * Hkv, Hkv, 128, 65536, "bf16", schedule=sch)
+            st, plans[sch] = sfd.alspec_query_plan(desc, 4, W)
+            assert st == 0
+        assert plans["sink_first"]["schedule"] == ab.ALSPEC_SCHEDULE_SINK_FIRST
+        heads = B * Hkv
+        assert plans["streams"]["n1"] * heads <= 148 * 3 // 4
+        assert plans["sink_first"]["n1"] * heads <= 148
+        assert plans["sink_first"]["n1"] >= plans["streams"]["n1"]
+        assert plans["sink_first"]["n2"] == plans["streams"]["n2"]
 
 
 @pytest.mark.parametrize("split", [16, 112, 1024, 100000])
