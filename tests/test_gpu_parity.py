@@ -137,6 +137,31 @@ def test_short_sequences_in_a_clustered_sink_set(cuda_device, d, engine):
     assert dec.device_error() == (0, 0)
 
 
+@pytest.mark.parametrize("schedule", ["streams", "fused", "sink_first"])
+def test_large_batch_of_short_sequences(cuda_device, schedule):
+    """64 sequences x 8 KV heads = 512 (sequence, head) pairs, more than the
+    SMs: one sink-set CTA per head in the sink-set kernel's grid, ragged
+    lengths from 1 to 3000 tokens, NaN past every length."""
+    import numpy as np
+    rng = np.random.default_rng(64)
+    lens = [int(x) for x in rng.integers(1, 3001, size=64)]
+    lens[0], lens[1] = 1, 3000
+    wl = workloads.Workload("large-batch", B=64, Hq=32, Hkv=8, d=128, L=3000, S=4, W=256,
+                            lam=0.3, dtype="bf16", seed=6464)
+    data = workloads.make_layer(wl, device=cuda_device)
+    data["lens"] = lens
+    data["seq_lens"] = torch.tensor(lens, dtype=torch.int32, device=cuda_device)
+    for b, L in enumerate(lens):
+        data["k"][b, :, L:, :] = float("nan")
+        data["v"][b, :, L:, :] = float("nan")
+    dec, out = gpu_decode(wl, data, cuda_device, schedule=schedule)
+    assert_parity(out, oracle_decode(wl, data), wl.lam, what=f"large batch {schedule}")
+    for b, L in enumerate(lens):
+        if L <= wl.S + wl.W:
+            assert torch.equal(out["out_spec"][b], out["out_exact"][b])
+    assert dec.device_error() == (0, 0)
+
+
 def test_deterministic_and_reusable_workspace(cuda_device):
     wl = _small(1)
     data = workloads.make_layer(wl, device=cuda_device)
