@@ -1,6 +1,7 @@
 // Host side of libalspec.so: argument checks, work planning, workspace
-// layout, the fork/join onto a high-priority stream, kernel launches and the
-// C ABI declared in include/alspec.h.
+// layout, the launch schedules (the sink-set kernel forked onto a
+// high-priority stream, or first on the caller's stream, or one fused
+// launch), kernel launches and the C ABI declared in include/alspec.h.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>

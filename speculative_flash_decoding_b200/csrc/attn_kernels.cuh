@@ -19,9 +19,12 @@
 //   * the middle kernel (MID) is persistent: CTAs pull items from an atomic
 //     queue and stream the cache through shared memory;
 //   * the merge kernel, after both, combines the sink-set partial with the
-//     middle partials into O_exact (one CTA per query head, the chunks split
-//     over four thread groups), and the CTA finishing a sequence's last head
-//     computes rel_l2 and the commit flag.
+//     middle partials into O_exact (one CTA per 32 output columns of a query
+//     head, its warps over interleaved chunks), and the CTA finishing a
+//     sequence's last slot computes rel_l2 and the commit flag;
+//   * the one-launch variant (FUSED) is the middle kernel with the sink-set
+//     items at the head of its queue and the merges done in the kernel, by
+//     the CTA whose tile ticket completes a (sequence, KV head).
 //
 // Inside a CTA one producer lane fills a ring of shared-memory stages with
 // K and V tiles through the TMA engine (mbarrier completion); consumer warps
