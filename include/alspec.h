@@ -310,9 +310,13 @@ alspec_status alspec_read_probe(const void* buf, size_t bytes, uint32_t* err, vo
  *   6 dynamic shared memory per CTA      7 pipeline stages
  *   8 engine (alspec_engine, resolved)
  *   9 schedule (alspec_schedule, resolved)
+ *  10 CTAs per sequence (one thread-block cluster) of the merge kernel, or
+ *     0 when the merge runs as one CTA per 32 output columns (a CTA's share
+ *     of the middle partials does not fit in shared memory; and the FUSED
+ *     schedule, which merges inside its one kernel)
  * (entries 4-7 describe the exact-path kernel, or with the FUSED schedule
  * the one kernel, whose queue holds both kinds of items).  n_info is the
- * capacity of info (10 fills all).
+ * capacity of info (11 fills all).
  */
 alspec_status alspec_query_plan(const alspec_desc* desc, int n_sink, int window,
                                 int* info, int n_info);

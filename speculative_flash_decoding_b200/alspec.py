@@ -193,9 +193,10 @@ def alspec_decode_noalloc(desc: alspec_desc, q: int, k_cache: int, v_cache: int,
 
 
 def alspec_query_plan(desc: alspec_desc, n_sink: int, window: int):
-    info = (ctypes.c_int * 10)()
-    st = int(_lib.alspec_query_plan(ctypes.byref(desc), n_sink, window, info, 10))
-    keys = ("c1", "n1", "c2", "n2", "grid2", "threads", "smem", "stages", "engine", "schedule")
+    info = (ctypes.c_int * 11)()
+    st = int(_lib.alspec_query_plan(ctypes.byref(desc), n_sink, window, info, 11))
+    keys = ("c1", "n1", "c2", "n2", "grid2", "threads", "smem", "stages", "engine", "schedule",
+            "merge_c")
     return st, dict(zip(keys, list(info)))
 
 

@@ -154,6 +154,9 @@ struct Plan {
     unsigned fq[kMaxChunks + 1];
     int grid1, grid2;
     bool sink_first;  // SINK_FIRST: the sink-set kernel alone first, then the middle kernel
+    int merge_c;      // CTAs per sequence (one cluster) of the cluster merge; 0: the
+                      // 32-column merge kernel
+    int merge_smem;   // its dynamic shared memory
     int threads, smem, stages;
     size_t off_ctr, off_spec_ml, off_spec_o, off_spec_pml, off_spec_po, off_mid_ml, off_mid_o,
         off_dn, total;
@@ -281,6 +284,29 @@ void make_plan(const alspec_desc& d, int S, int W, int sms, Plan* pl) {
     pl->c2 = pl->n2 > 0
                  ? (int)(((unsigned long long)mid_tiles * pl->fq[1]) >> kFracBits) * TT
                  : 0;
+    // Merge: the 32-column merge kernel (B * H_q * d / 32 CTAs) while it
+    // fits in one wave of CTAs; beyond that one cluster of C CTAs per
+    // sequence, when a CTA's middle partials ([H_q / C][n2][d] fp32) fit in
+    // shared memory, C the largest of 8, 4, 2, 1 dividing H_q with at most
+    // kCmMaxHeads heads per CTA.  Measured (same box): the batch of 8
+    // ragged sequences 805.7 -> 758.8 us per 4 layers, the 70B batch of 4
+    // 1299 -> 1255 us; one 128K sequence 2758 -> 2812 us per 32 layers,
+    // where the 128 small CTAs spread the loads over more SMs.
+    pl->merge_c = 0;
+    pl->merge_smem = 0;
+    const bool one_wave =
+        (long long)d.batch * d.n_q_heads * merge_splits(d.head_dim) <= (long long)sms;
+    for (int c : {8, 4, 2, 1}) {
+        if (fused || one_wave) break;
+        if (d.n_q_heads % c != 0 || d.n_q_heads / c > kCmMaxHeads) continue;
+        const long long bytes =
+            (long long)(d.n_q_heads / c) * std::max(pl->n2, 0) * d.head_dim * 4 + 128;
+        if (bytes <= kSmemLimit - kCmStatic) {
+            pl->merge_c = c;
+            pl->merge_smem = (int)bytes;
+        }
+        break;
+    }
     const long long items2 = (long long)heads * (pl->n2 + (fused ? pl->n1 : 0));
     pl->grid2 = (int)std::min<long long>(P, items2);
     const int G = d.n_q_heads / d.n_kv_heads;
@@ -478,9 +504,9 @@ alspec_status alspec_query_plan(const alspec_desc* desc, int n_sink, int window,
     if (!info || n_info < 0) return ALSPEC_ERR_INVALID_ARG;
     Plan pl{};
     make_plan(*desc, n_sink, window, sm_count_for_plan(), &pl);
-    const int vals[10] = {pl.c1,      pl.n1,   pl.c2,     pl.n2,     pl.grid2,
-                          pl.threads, pl.smem, pl.stages, pl.engine, pl.schedule};
-    for (int i = 0; i < n_info && i < 10; ++i) info[i] = vals[i];
+    const int vals[11] = {pl.c1,      pl.n1,   pl.c2,     pl.n2,     pl.grid2,   pl.threads,
+                          pl.smem,    pl.stages, pl.engine, pl.schedule, pl.merge_c};
+    for (int i = 0; i < n_info && i < 11; ++i) info[i] = vals[i];
     return ALSPEC_OK;
 }
 
@@ -681,10 +707,19 @@ alspec_status decode_impl(const alspec_desc* desc, const void* q, const void* k_
     // Join, then merge + relative L2 + flag.
     if (!ok(cudaStreamWaitEvent(s, ds->join, 0))) return ALSPEC_ERR_CUDA;
     KernelFn mk = nullptr;
-    if (desc->head_dim == 128)
+    if (pl.merge_c > 0) {
+        if (desc->head_dim == 128)
+            mk = pl.tt == 32 ? merge_cluster_kernel<128, 32> : merge_cluster_kernel<128, 16>;
+        else
+            mk = pl.tt == 32 ? merge_cluster_kernel<64, 32> : merge_cluster_kernel<64, 16>;
+        if ((st = ensure_smem_attr(ds, reinterpret_cast<const void*>(mk),
+                                   kSmemLimit - kCmStatic)) != ALSPEC_OK)
+            return st;
+    } else if (desc->head_dim == 128) {
         mk = pl.tt == 32 ? merge_kernel<128, 32> : merge_kernel<128, 16>;
-    else
+    } else {
         mk = pl.tt == 32 ? merge_kernel<64, 32> : merge_kernel<64, 16>;
+    }
     // With ALSPEC_GATE_GRAPH_CONDITIONAL, inside a stream capture the
     // recomputation of discarded tokens' output projection is a conditional
     // node, enabled by a one-warp kernel that reads the flags.
@@ -703,10 +738,15 @@ alspec_status decode_impl(const alspec_desc* desc, const void* q, const void* k_
     // Programmatic launch right behind the middle kernel (when there is one
     // and no profiling event sits between them).
     const bool pdl = pl.n2 > 0 && !prof_events;
-    if ((st = launch(mk, dim3(desc->n_q_heads * merge_splits(desc->head_dim), desc->batch),
-                     dim3(kMergeThreads),
-                     0, s, p, pdl ? kLaunchProgrammatic : 0, 0)) != ALSPEC_OK)
+    if (pl.merge_c > 0) {
+        if ((st = launch(mk, dim3(pl.merge_c, desc->batch), dim3(kCmThreads), pl.merge_smem, s, p,
+                         pdl ? kLaunchProgrammatic : 0, 0, pl.merge_c)) != ALSPEC_OK)
+            return st;
+    } else if ((st = launch(mk, dim3(desc->n_q_heads * merge_splits(desc->head_dim), desc->batch),
+                            dim3(kMergeThreads), 0, s, p, pdl ? kLaunchProgrammatic : 0, 0)) !=
+               ALSPEC_OK) {
         return st;
+    }
     if (op) {
         // Redo the projection on O_exact for the discarded tokens, after the
         // speculative one (both write y).

@@ -1839,4 +1839,202 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const __grid_const
     }
 }
 
+// ----------------------------------------- merge + verify, one cluster per sequence
+//
+// The same merge with one thread-block cluster of C CTAs per sequence
+// (C <= 8, dividing H_q): CTA r owns query heads [r * H_q / C, (r + 1) * H_q / C),
+// whose middle partials [heads][n2][d] are contiguous in the workspace and
+// arrive with bulk copies into shared memory while the chunk weights are
+// computed; its (squared distance, squared norm) sums go to CTA 0 of the
+// cluster through distributed shared memory, which writes rel_l2 and the
+// flag.  Against the 32-column merge kernel this saves the per-sequence
+// ticket and the reload of the slots (two dependent global round trips).
+// Used when a CTA's partials fit in shared memory.
+constexpr int kCmThreads = 256;
+constexpr int kCmWarps = kCmThreads / 32;
+constexpr int kCmMaxHeads = 8;     // query heads per CTA at most
+constexpr int kCmStatic = 16384;   // static shared memory, rounded up (for the host's budget)
+
+template <int D, int TT>
+__global__ void __launch_bounds__(kCmThreads, 1) merge_cluster_kernel(const __grid_constant__ Params p) {
+    extern __shared__ unsigned char cm_raw[];
+    float* blk = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(cm_raw) + 127) & ~uintptr_t(127));
+    __shared__ int list[kMaxChunks];
+    __shared__ float wts[kCmMaxHeads][kMaxChunks];
+    __shared__ float fl[kCmMaxHeads][2];    // weight of the sink-set partial, l
+    __shared__ double red[2][kCmWarps];
+    __shared__ double dn_cta[2];
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int nlist;
+    const int C = (int)gridDim.x;
+    const int rank = (int)blockIdx.x;  // the cluster spans the x dimension
+    const int b = blockIdx.y;
+    const int hpc = p.Hq / C;
+    const int h0 = rank * hpc;
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    const size_t bq0 = (size_t)b * p.Hq + h0;
+    static_assert(kMaxChunks <= kCmThreads, "one chunk per thread in the list scan");
+    static_assert(sizeof(int) * kMaxChunks + sizeof(float) * kCmMaxHeads * (kMaxChunks + 2) +
+                          sizeof(double) * (2 * kCmWarps + 2) + 8 + 4 <= kCmStatic,
+                  "static shared memory");
+
+    // Inputs only: the non-empty chunks of this sequence, in order.
+    if (tid == 0) {
+        const int mid_tiles = cdiv(seq_geom(p, b, false).mid_len, TT);
+        int count = 0, prev = 0;
+#pragma unroll 8
+        for (int c = 0; c < p.n2; ++c) {
+            const int t = (int)(((unsigned long long)mid_tiles * p.fq[c + 1]) >> kFracBits);
+            if (t > prev) list[count++] = c;
+            prev = t;
+        }
+        nlist = count;
+        mbar_init(&bar, 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    const int n = nlist;
+    // The partials are written by the kernels this one follows.
+    pdl_wait_prerequisite();
+    const size_t bytes = (size_t)hpc * p.n2 * D * sizeof(float);
+    if (warp == 0 && bytes > 0) {
+        constexpr uint32_t kPiece = 16384;
+        const char* src = reinterpret_cast<const char*>(p.mid_o + bq0 * p.n2 * D);
+        fence_proxy_async_global();
+        if (lane == 0) mbar_arrive_expect_tx(&bar, (uint32_t)bytes);
+        __syncwarp();
+        const uint64_t pol = l2_evict_first_policy();
+        for (size_t off = (size_t)lane * kPiece; off < bytes; off += 32 * (size_t)kPiece) {
+            const uint32_t nb = (uint32_t)(bytes - off < kPiece ? bytes - off : kPiece);
+            bulk_load(reinterpret_cast<unsigned char*>(blk) + off, src + off, nb, &bar, pol);
+        }
+    }
+    // Per query head (one warp each): max, weights, normaliser, while the
+    // copies land.
+    for (int hh = warp; hh < hpc; hh += kCmWarps) {
+        const float2 sml = __ldcg(reinterpret_cast<const float2*>(p.spec_ml) + bq0 + hh);
+        const float2* ml = reinterpret_cast<const float2*>(p.mid_ml) + (bq0 + hh) * p.n2;
+        float2 x[kMaxChunks / 32];
+        float M = sml.x;
+#pragma unroll
+        for (int k = 0; k < kMaxChunks / 32; ++k) {
+            const int i = lane + 32 * k;
+            x[k] = i < n ? __ldcg(ml + list[i]) : make_float2(-INFINITY, 0.f);
+            M = fmaxf(M, x[k].x);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        float lsum = 0.f;
+#pragma unroll
+        for (int k = 0; k < kMaxChunks / 32; ++k) {
+            const int i = lane + 32 * k;
+            if (i < n) {
+                const float f = merge_weight(x[k].x, M);
+                wts[hh][i] = f;
+                lsum = fmaf(f, x[k].y, lsum);
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
+        if (lane == 0) {
+            const float f0 = merge_weight(sml.x, M);
+            fl[hh][0] = f0;
+            fl[hh][1] = fmaf(f0, sml.y, lsum);
+        }
+    }
+    __syncthreads();
+    // The copies (bounded wait; on expiry the error bit is raised and the
+    // CTA waits once more, bounded, so no copy lands after it exits).
+    if (bytes > 0) {
+        bool ok = true;
+        const uint64_t t0 = global_ns();
+        while (!mbar_try_wait(&bar, 0)) {
+            if (global_ns() - t0 > p.timeout_ns) {
+                ok = false;
+                break;
+            }
+        }
+        if (!ok) {
+            if (tid == 0) atomicOr(p.ctr + kCtrError, kErrTimeout);
+            const uint64_t t1 = global_ns();
+            while (!mbar_try_wait(&bar, 0) && global_ns() - t1 < p.timeout_ns) {
+            }
+        }
+    }
+    // Columns: four interleaved sums per output (list position i goes to
+    // sum i mod 4), then a fixed tree.
+    double dd = 0.0, nn = 0.0;
+    for (int idx = tid; idx < hpc * D; idx += kCmThreads) {
+        const int hh = idx / D;
+        const int e = idx % D;
+        const size_t bq = bq0 + hh;
+        const float os = __ldcg(p.spec_o + bq * D + e);
+        const float sl = __ldcg(p.spec_ml + bq * 2 + 1);
+        const float* col = blk + (size_t)hh * p.n2 * D + e;
+        const float* wh = wts[hh];
+        float acc[4] = {fl[hh][0] * os, 0.f, 0.f, 0.f};
+        int i = 0;
+        for (; i + 4 <= n; i += 4) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) acc[k] = fmaf(wh[i + k], col[(size_t)list[i + k] * D], acc[k]);
+        }
+#pragma unroll
+        for (int k = 0; k < 3; ++k)
+            if (i + k < n) acc[k] = fmaf(wh[i + k], col[(size_t)list[i + k] * D], acc[k]);
+        const float a = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+        const float o_exact = __fdiv_rn(a, fl[hh][1]);
+        const float o_spec = __fdiv_rn(os, sl);
+        p.out_exact[bq * D + e] = o_exact;
+        const float diff = o_exact - o_spec;
+        dd += (double)(diff * diff);
+        nn += (double)(o_exact * o_exact);
+    }
+    // This CTA's sums (fixed order), then CTA 0 of the cluster adds the
+    // CTAs' sums in rank order.
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        dd += __shfl_xor_sync(0xffffffffu, dd, o);
+        nn += __shfl_xor_sync(0xffffffffu, nn, o);
+    }
+    if (lane == 0) {
+        red[0][warp] = dd;
+        red[1][warp] = nn;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        double s0 = 0.0, s1 = 0.0;
+        for (int w = 0; w < kCmWarps; ++w) {
+            s0 += red[0][w];
+            s1 += red[1][w];
+        }
+        dn_cta[0] = s0;
+        dn_cta[1] = s1;
+    }
+    cluster_sync();  // every CTA's sums and O_exact are written
+    if (rank == 0 && tid == 0) {
+        double D2 = 0.0, N2 = 0.0;
+        const uint32_t local = smem_addr(dn_cta);
+        for (int r = 0; r < C; ++r) {
+            const uint32_t a = dsmem_addr(local, (uint32_t)r);
+            double v0, v1;
+            asm volatile("ld.shared::cluster.f64 %0, [%1];" : "=d"(v0) : "r"(a) : "memory");
+            asm volatile("ld.shared::cluster.f64 %0, [%1];" : "=d"(v1) : "r"(a + 8u) : "memory");
+            D2 += v0;
+            N2 += v1;
+        }
+        double r;
+        if (N2 == 0.0) {
+            r = D2 == 0.0 ? 0.0 : (double)INFINITY;
+        } else {
+            r = sqrt(D2 / N2);
+        }
+        p.rel_l2[b] = (float)r;
+        p.commit[b] = r <= (double)p.lambda ? 1 : 0;
+    }
+    cluster_sync();  // CTA 0 has read every CTA's sums
+    if (rank == 0 && tid == 0) trace_publish(p, 1);
+}
+
 }  // namespace alspec

@@ -162,6 +162,27 @@ def test_large_batch_of_short_sequences(cuda_device, schedule):
     assert dec.device_error() == (0, 0)
 
 
+@pytest.mark.parametrize("shape", ["cluster8", "cluster4_3kv", "columns_fallback"])
+def test_merge_kernels(cuda_device, shape):
+    """Both merge kernels on the default schedule: one cluster per sequence
+    (8 CTAs of 4 heads; 4 CTAs of 3 heads with 3 KV heads), and one CTA per
+    32 columns -- for one wave of such CTAs, or when a cluster CTA's
+    partials would not fit in shared memory (2 x 64 query heads, 62 chunks
+    per head)."""
+    B, Hq, Hkv, L, split, want_c = {
+        "cluster8": (2, 32, 8, 20000, 0, 8),
+        "cluster4_3kv": (4, 12, 3, 9000, 0, 4),
+        "columns_fallback": (2, 64, 8, 32768, 512, 0),
+    }[shape]
+    wl = workloads.Workload("merge-" + shape, B=B, Hq=Hq, Hkv=Hkv, d=128, L=L, S=4, W=1024,
+                            lam=0.3, dtype="bf16", seed=808)
+    data = workloads.make_layer(wl, device=cuda_device, poison_tail=True)
+    dec, out = gpu_decode(wl, data, cuda_device, split_tokens=split)
+    assert dec.plan()["merge_c"] == want_c
+    assert_parity(out, oracle_decode(wl, data), wl.lam, what="merge " + shape)
+    assert dec.device_error() == (0, 0)
+
+
 def test_deterministic_and_reusable_workspace(cuda_device):
     wl = _small(1)
     data = workloads.make_layer(wl, device=cuda_device)
