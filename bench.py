@@ -130,17 +130,19 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def stored_traffic(path):
+def stored_traffic(path, workload):
     """DRAM bytes per launch of the dominant kernel from a committed ncu
-    summary, or None when the kernel or planner source changed since it was
-    captured (`source_sha256` is over the files in KERNEL_SRCS, in order)."""
+    summary of `workload`, or None when the summary covers another workload
+    or the kernel or planner source changed since it was captured
+    (`source_sha256` is over the files in KERNEL_SRCS, in order)."""
     try:
         text = open(path).read()
     except OSError:
         return None
     m_hash = re.search(r"source_sha256:\s*([0-9a-f]{64})", text)
     m_bytes = re.search(r"dram_bytes_per_launch:\s*([0-9]+)", text)
-    if not (m_hash and m_bytes):
+    m_work = re.search(r"traffic_workload:\s*(\S+)", text)
+    if not (m_hash and m_bytes and m_work) or m_work.group(1) != workload:
         return None
     h = hashlib.sha256()
     for f in KERNEL_SRCS:
@@ -523,7 +525,7 @@ def run_alspec(args, wl):
         mid_bytes = workloads.kv_bytes(wl, layers[0]["lens"])
     mid_avg_ms = sum(mid_ms) / len(mid_ms)
     achieved = mid_bytes / (mid_avg_ms * 1e-3) / 1e9
-    traffic = stored_traffic(FUSED_TRAFFIC_FILE if fused else TRAFFIC_FILE)
+    traffic = stored_traffic(FUSED_TRAFFIC_FILE if fused else TRAFFIC_FILE, wl.name)
     value = job_throughput(kv_bytes, world, ms_per_step)
 
     cpu = None
