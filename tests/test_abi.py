@@ -87,6 +87,8 @@ def test_workspace_size_and_plan():
     (dict(max_seq_len=0), 4, 8, ab.ALSPEC_ERR_INVALID_ARG),
     (dict(dtype=7), 4, 8, ab.ALSPEC_ERR_INVALID_ARG),
     (dict(engine=3), 4, 8, ab.ALSPEC_ERR_INVALID_ARG),
+    (dict(schedule=4), 4, 8, ab.ALSPEC_ERR_INVALID_ARG),
+    (dict(schedule=-1), 4, 8, ab.ALSPEC_ERR_INVALID_ARG),
     (dict(max_seq_len=1 << 29), 4, 8, ab.ALSPEC_ERR_UNSUPPORTED),  # rows >= 2^31
     (dict(), 0, 0, ab.ALSPEC_ERR_INVALID_ARG),                  # empty sink set
     (dict(), -1, 8, ab.ALSPEC_ERR_INVALID_ARG),
@@ -101,6 +103,21 @@ def test_bad_descriptions(kw, S, W, code):
     st = sfd.alspec_decode(d, fake, fake, fake, fake, S, W, 0.1, fake, fake, fake, fake, fake,
                            1 << 30, 0, 0, None)
     assert st == code
+
+
+def test_schedules_in_the_plan_and_workspace():
+    """AUTO resolves to STREAMS; each schedule reports itself; the one-launch
+    schedule needs room for its sink-set item partials."""
+    sizes = {}
+    for name, code in (("auto", 1), ("streams", 1), ("fused", 2), ("sink_first", 3)):
+        d = desc(schedule=name)
+        st, plan = sfd.alspec_query_plan(d, 4, 1024)
+        assert st == 0 and plan["schedule"] == code
+        sizes[name] = sfd.alspec_workspace_size(d, 4, 1024)
+        assert sizes[name] > 0
+    assert sizes["auto"] == sizes["streams"] == sizes["sink_first"] < sizes["fused"]
+    # The fused schedule merges inside its kernel: no separate merge kernel.
+    assert sfd.alspec_query_plan(desc(schedule="fused"), 4, 1024)[1]["merge_c"] == 0
 
 
 def _decode_with(**over):
