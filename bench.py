@@ -8,7 +8,12 @@ high-priority stream), the split exact-attention kernel and the merge +
 relative-L2 + flag kernel, all captured in one CUDA graph.  Layers are
 independent caches generated from the seed; inputs are resident in HBM.
 
-Output: one JSON line on rank 0 (see the keys at the end of main()).
+The other four workloads (a tiny fp32 layer, a 32K layer, a ragged batch of
+eight 16K-64K sequences, a Llama-70B-shaped batch of four 128K sequences) are
+timed the same way, a few steps each, and reported in the line's per_config
+object.
+
+Output: one JSON line on rank 0 (see the keys at the end of run_alspec()).
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl alspec|reference]
 With --impl reference the fp64 CPU oracle is timed on the host cores on a
 bounded sample of the same workload instead.
@@ -66,6 +71,10 @@ def parse_args():
                     help="speculative output projection against the serial one (32 x 128K)")
     ap.add_argument("--lambda-sweep", action="store_true",
                     help="hit rate against the threshold on the commit-mixing workload family")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the other workloads' entries (per_config) of the line")
+    ap.add_argument("--per-config-steps", type=int, default=10,
+                    help="timed steps of each other workload in per_config")
     return ap.parse_args()
 
 
@@ -278,8 +287,7 @@ def run_reference(args, wl):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": t * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": wl.name, "context": wl.L, "sink": wl.S, "window": wl.W,
-                       "lambda": wl.lam, "sample": sample},
+            "config": workload_config(wl, args.layers or wl.n_layers, world),
             "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
@@ -290,35 +298,92 @@ def run_reference(args, wl):
 
 # ---------------------------------------------------------------- GPU leg
 
-def run_alspec(args, wl):
+PROBE_LIB = os.path.join(ROOT, "speculative_flash_decoding_b200", "libalspec_read_probe.so")
+
+
+def read_probe_fn():
+    """alspec_read_probe from libalspec_read_probe.so (include/alspec_read_probe.h):
+    (buf, bytes, err, stream) -> status; a measurement aid outside the
+    decode library."""
+    import ctypes
+    lib = ctypes.CDLL(PROBE_LIB)
+    fn = lib.alspec_read_probe
+    fn.restype = ctypes.c_int
+    fn.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_void_p]
+    return lambda buf, nbytes, stream, err=0: int(fn(buf, nbytes, err or None, stream))
+
+
+def workload_config(wl, n_layers, world):
+    """The `config` object of both arms' lines: the workload, nothing about
+    how either arm runs it."""
+    return {"workload": wl.name, "layers": n_layers, "batch": wl.B, "q_heads": wl.Hq,
+            "kv_heads": wl.Hkv, "head_dim": wl.d, "context": wl.L,
+            "ragged": list(wl.ragged) if wl.ragged else None, "sink": wl.S, "window": wl.W,
+            "lambda": wl.lam, "cache_dtype": wl.dtype,
+            "parallelism": "replicas" if world > 1 else "single"}
+
+
+def middle_bytes(wl, lens, fused):
+    """Algorithmic bytes of one launch of the dominant kernel: the middle
+    rows [S, L - W) of every sequence (two-stream schedules), or every row
+    (one-launch schedule, whose kernel reads the sink set too)."""
+    import workloads
+    if fused:
+        return workloads.kv_bytes(wl, lens)
+    return sum(max(0, L - wl.W - min(wl.S, L)) * wl.Hkv * wl.d * 2 * wl.elem_bytes for L in lens)
+
+
+def quantiles_us(ms):
+    if len(ms) < 2:
+        return None
+    q = statistics.quantiles(ms, n=10)
+    return [float(q[0] * 1e3), float(statistics.median(ms) * 1e3), float(q[-1] * 1e3)]
+
+
+def measure(wl, n_layers, steps, warmup, device, ranks, args, want_e2e=True, lat_layers=4):
+    """Time one workload on this rank's GPU (every rank runs the same steps).
+
+    A step is one decode token through the workload's n_layers layers (each
+    its own seeded cache, all resident in HBM): per layer the sink-set
+    kernel on the library's high-priority stream, the exact-path (middle)
+    kernel and the merge, captured as one CUDA graph per step.  Passes:
+      timed     `steps` graph replays, CUDA events on the launch stream;
+                a step whose caches fit a few times in L2 is preceded by an
+                untimed L2 flush and timed on its own;
+      profiled  the same step with per-layer event nodes: the middle
+                kernel's duration (the roofline's denominator);
+      latency   graphs through the traced entry point (kernel-written time
+                stamps of O_spec's and O_exact's publication), over the
+                step's layers, or over `lat_layers` distinct layers when the
+                step has one, each replay timed too (per-layer time);
+      e2e       the step through the public API with host buffers.
+    Returns a dict of raw measurements (times in ms)."""
     import torch
     import workloads
     import speculative_flash_decoding_b200 as sfd
 
-    rank, world, local = dist_env()
-    device = torch.device("cuda", local)
-    torch.cuda.set_device(device)
-    ranks = Ranks("nccl", device)
-
-    n_layers = args.layers or wl.n_layers
-    layers = [workloads.make_layer(wl, layer=i, device=device) for i in range(n_layers)]
-    q_all = torch.stack([d["q"] for d in layers]).contiguous()      # [layers, B, Hq, d]
+    n_lat = n_layers if n_layers >= 2 else lat_layers
+    layers = [workloads.make_layer(wl, layer=i, device=device) for i in range(max(n_layers, n_lat))]
+    q_all = torch.stack([d["q"] for d in layers]).contiguous()            # [layers, B, Hq, d]
     lens_all = torch.stack([d["seq_lens"] for d in layers]).contiguous()  # [layers, B]
     for i, d in enumerate(layers):
         d["q"] = q_all[i]
         d["seq_lens"] = lens_all[i]
-    kv_bytes = sum(workloads.kv_bytes(wl, d["lens"]) for d in layers)
+    kv_bytes = sum(workloads.kv_bytes(wl, d["lens"]) for d in layers[:n_layers])
+    lat_kv_bytes = sum(workloads.kv_bytes(wl, d["lens"]) for d in layers[:n_lat])
     dec = sfd.Decoder(wl.B, wl.Hq, wl.Hkv, wl.d, wl.L, wl.dtype, wl.S, wl.W, device=device,
                       split_tokens=args.split_tokens, engine=args.engine, schedule=args.schedule)
     plan = dec.plan()
     fused = plan["schedule"] == sfd.ALSPEC_SCHEDULE_FUSED
-    out_spec = torch.empty(n_layers, wl.B, wl.Hq, wl.d, dtype=torch.float32, device=device)
+    n_all = len(layers)
+    out_spec = torch.empty(n_all, wl.B, wl.Hq, wl.d, dtype=torch.float32, device=device)
     out_exact = torch.empty_like(out_spec)
-    rel_all = torch.empty(n_layers, wl.B, dtype=torch.float32, device=device)
-    commit_all = torch.empty(n_layers, wl.B, dtype=torch.uint8, device=device)
+    rel_all = torch.empty(n_all, wl.B, dtype=torch.float32, device=device)
+    commit_all = torch.empty(n_all, wl.B, dtype=torch.uint8, device=device)
     outs = [dict(out_spec=out_spec[i], out_exact=out_exact[i], rel_l2=rel_all[i],
-                 commit=commit_all[i]) for i in range(n_layers)]
+                 commit=commit_all[i]) for i in range(n_all)]
     stream = torch.cuda.Stream(device)
+    step_layers = layers[:n_layers]
 
     def new_events():
         evs = [[torch.cuda.Event(enable_timing=True, external=True)
@@ -328,13 +393,15 @@ def run_alspec(args, wl):
                 e.record(stream)
         return evs
 
-    def capture(events):
+    def capture(events=None, traces=None, which=None):
+        which = step_layers if which is None else which
         with torch.cuda.stream(stream):
             st = sfd.alspec_graph_begin(stream.cuda_stream)
             assert st == 0, sfd.alspec_status_string(st)
-            for i, d in enumerate(layers):
+            for i, d in enumerate(which):
                 dec.decode(d["q"], d["k"], d["v"], d["seq_lens"], wl.lam, out=outs[i],
-                           stream=stream, prof_events=events[i] if events else None)
+                           stream=stream, prof_events=events[i] if events else None,
+                           trace=traces[i] if traces is not None else None)
             st, g = sfd.alspec_graph_end(stream.cuda_stream)
             assert st == 0, sfd.alspec_status_string(st)
         return g
@@ -346,39 +413,18 @@ def run_alspec(args, wl):
     stream.synchronize()
 
     # Timed graphs carry no profiling events (so nothing sits between the
-    # kernels); a second set of graphs with per-layer events measures the
-    # per-kernel breakdown in its own timed pass.
-    warm_graph = capture(None)
-    graphs = [capture(None) for _ in range(args.steps)]
-    prof_steps = max(3, min(args.steps, 10))
+    # kernels); separate graphs carry the events and the time stamps.
+    warm_graph = capture()
+    graphs = [capture() for _ in range(steps)]
+    prof_steps = max(3, min(steps, 10))
     step_events = [new_events() for _ in range(prof_steps)]
-    prof_graphs = [capture(ev) for ev in step_events]
+    prof_graphs = [capture(events=ev) for ev in step_events]
+    traces = torch.zeros(prof_steps, n_lat, 2, dtype=torch.int64, device=device)
+    lat = [capture(traces=traces[j], which=layers[:n_lat]) for j in range(prof_steps)]
 
-    # Latency graphs: the timed step through the traced entry point, which
-    # leaves per layer the global-timer ns at which O_spec and O_exact were
-    # published (written by the kernels; no event nodes in the graph).
-    # t_spec(l) runs from the end of layer l-1 to O_spec of layer l,
-    # t_exact(l) to the end of layer l.
-    traces = torch.zeros(prof_steps, n_layers, 2, dtype=torch.int64, device=device)
-
-    def capture_latency(tr):
-        with torch.cuda.stream(stream):
-            st = sfd.alspec_graph_begin(stream.cuda_stream)
-            assert st == 0, sfd.alspec_status_string(st)
-            for i, d in enumerate(layers):
-                dec.decode(d["q"], d["k"], d["v"], d["seq_lens"], wl.lam, out=outs[i],
-                           stream=stream, trace=tr[i])
-            st, g = sfd.alspec_graph_end(stream.cuda_stream)
-            assert st == 0, sfd.alspec_status_string(st)
-        return g
-
-    lat = [capture_latency(traces[j]) for j in range(prof_steps)]
-
-    barrier = ranks.barrier
-
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         sfd.alspec_graph_launch(warm_graph, stream.cuda_stream)
-    barrier()
+    ranks.barrier()
 
     uuid = None
     try:
@@ -393,60 +439,76 @@ def run_alspec(args, wl):
     l2_bytes = int(getattr(torch.cuda.get_device_properties(device), "L2_cache_size", 0) or
                    (126 << 20))
     flush = kv_bytes < 4 * l2_bytes
-    scrub = torch.empty(2 * l2_bytes, dtype=torch.uint8, device=device) if flush else None
-    clean = torch.ones(l2_bytes // 2, dtype=torch.int32, device=device) if flush else None
-    sink = torch.empty((), dtype=torch.int64, device=device) if flush else None
+    lat_flush = lat_kv_bytes < 4 * l2_bytes
+    scrub = clean = sink = None
+    if flush or lat_flush:
+        scrub = torch.empty(2 * l2_bytes, dtype=torch.uint8, device=device)
+        clean = torch.ones(l2_bytes // 2, dtype=torch.int32, device=device)
+        sink = torch.empty((), dtype=torch.int64, device=device)
+
+    def flush_l2():
+        with torch.cuda.stream(stream):
+            scrub.zero_()
+            torch.sum(clean, dim=0, out=sink)
+
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
-    step_begin = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    step_end = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    step_begin = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    step_end = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     nvtx = torch.cuda.nvtx
     with ClockSampler(uuid) as clocks:
-        barrier()
-        nvtx.range_push("timed steps")
+        ranks.barrier()
+        nvtx.range_push("timed steps " + wl.name)
         t_start.record(stream)
-        for i in range(args.steps):
+        for i in range(steps):
             if flush:
-                with torch.cuda.stream(stream):
-                    scrub.zero_()
-                    torch.sum(clean, dim=0, out=sink)
+                flush_l2()
             step_begin[i].record(stream)
             st = sfd.alspec_graph_launch(graphs[i], stream.cuda_stream)
             assert st == 0
             step_end[i].record(stream)
         t_end.record(stream)
-        barrier()
+        ranks.barrier()
         nvtx.range_pop()
-    per_step = [step_begin[i].elapsed_time(step_end[i]) for i in range(args.steps)]
+    per_step = [step_begin[i].elapsed_time(step_end[i]) for i in range(steps)]
     ms_total = sum(per_step) if flush else t_start.elapsed_time(t_end)
-    ms_per_step = ranks.max(ms_total / args.steps)
+    ms_per_step = ranks.max(ms_total / steps)
 
     # Profiled pass: same step with per-layer events captured in the graphs.
-    barrier()
+    ranks.barrier()
     nvtx.range_push("profiled pass (per-layer events)")
     with torch.cuda.stream(stream):
         for g in prof_graphs:
+            if flush:
+                flush_l2()
             assert sfd.alspec_graph_launch(g, stream.cuda_stream) == 0
-    barrier()
+    ranks.barrier()
     nvtx.range_pop()
 
-    # Latency pass.
-    barrier()
+    # Latency pass (each replay also timed as a whole).
+    ranks.barrier()
     nvtx.range_push("latency pass (kernel time stamps)")
     traces.zero_()
+    lat_begin = [torch.cuda.Event(enable_timing=True) for _ in lat]
+    lat_end = [torch.cuda.Event(enable_timing=True) for _ in lat]
     with torch.cuda.stream(stream):
-        for g in lat:
+        for j, g in enumerate(lat):
+            if lat_flush:
+                flush_l2()
+            lat_begin[j].record(stream)
             assert sfd.alspec_graph_launch(g, stream.cuda_stream) == 0
-    barrier()
+            lat_end[j].record(stream)
+    ranks.barrier()
     nvtx.range_pop()
+    lat_ms = [lat_begin[j].elapsed_time(lat_end[j]) / n_lat for j in range(len(lat))]
     tr = traces.cpu().numpy().astype("int64")
     t_spec, t_exact = [], []
     for j in range(prof_steps):
-        for i in range(1, n_layers):
+        for i in range(1, n_lat):
             t_spec.append((tr[j, i, 0] - tr[j, i - 1, 1]) * 1e-6)   # ms
             t_exact.append((tr[j, i, 1] - tr[j, i - 1, 1]) * 1e-6)
 
-    # Per-layer profiling events of every timed step.
+    # Per-layer profiling events of every profiled step.
     mid_ms, spec_ms, layer_ms, pre_ms, post_ms, gap_ms = [], [], [], [], [], []
     for ev in step_events:
         for i, e in enumerate(ev):
@@ -457,82 +519,167 @@ def run_alspec(args, wl):
             post_ms.append(e[3].elapsed_time(e[4]))
             if i + 1 < len(ev):
                 gap_ms.append(e[4].elapsed_time(ev[i + 1][0]))
-    hit_rate = float(commit_all.float().mean().item())
+    hit_rate = float(commit_all[:n_layers].float().mean().item())
     st, err = dec.device_error(stream)
     assert st == 0 and err == 0, f"device error word {err:#x}"
 
-    # End-to-end through the public API with host buffers: per step, copy the
+    # End to end through the public API with host buffers: per step, copy the
     # step's query vectors (all layers) and lengths in from pinned memory,
     # replay the step, read every layer's rel_l2 and flag back.
     e2e = None
-    if not args.no_e2e:
-        q_host = q_all.cpu().pin_memory()
-        lens_host = lens_all.cpu().pin_memory()
-        rel_host = torch.empty(rel_all.shape, dtype=rel_all.dtype).pin_memory()
-        com_host = torch.empty(commit_all.shape, dtype=commit_all.dtype).pin_memory()
+    if want_e2e:
+        q_host = q_all[:n_layers].cpu().pin_memory()
+        lens_host = lens_all[:n_layers].cpu().pin_memory()
+        rel_host = torch.empty((n_layers, wl.B), dtype=rel_all.dtype).pin_memory()
+        com_host = torch.empty((n_layers, wl.B), dtype=commit_all.dtype).pin_memory()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
-        barrier()
+        ranks.barrier()
         nvtx.range_push("end to end (host buffers)")
         with torch.cuda.stream(stream):
             e0.record(stream)
-            for i in range(args.steps):
-                q_all.copy_(q_host, non_blocking=True)
-                lens_all.copy_(lens_host, non_blocking=True)
+            for i in range(steps):
+                q_all[:n_layers].copy_(q_host, non_blocking=True)
+                lens_all[:n_layers].copy_(lens_host, non_blocking=True)
                 sfd.alspec_graph_launch(graphs[i], stream.cuda_stream)
-                rel_host.copy_(rel_all, non_blocking=True)
-                com_host.copy_(commit_all, non_blocking=True)
+                rel_host.copy_(rel_all[:n_layers], non_blocking=True)
+                com_host.copy_(commit_all[:n_layers], non_blocking=True)
                 stream.synchronize()
             e1.record(stream)
-        barrier()
+        ranks.barrier()
         nvtx.range_pop()
-        e2e_ms = ranks.max(e0.elapsed_time(e1) / args.steps)
+        e2e_ms = ranks.max(e0.elapsed_time(e1) / steps)
         h2d = q_host.numel() * q_host.element_size() + lens_host.numel() * lens_host.element_size()
         d2h = rel_host.numel() * rel_host.element_size() + com_host.numel() * com_host.element_size()
-        e2e = {"value": job_throughput(kv_bytes, world, e2e_ms), "unit": "GB/s",
+        e2e = {"value": job_throughput(kv_bytes, ranks.world, e2e_ms), "unit": "GB/s",
                "us_per_step": e2e_ms * 1e3, "h2d_bytes_per_step": int(h2d),
-               "d2h_bytes_per_step": int(d2h)}
+               "d2h_bytes_per_step": int(d2h),
+               "what": "per step: pinned host-to-device copy of every layer's q and seq_lens, "
+                       "the step's graph, device-to-host read of every layer's rel_l2 and "
+                       "commit flag, then a host synchronize; O_spec and O_exact stay on the "
+                       "device, where the post-attention ops that consume them run"}
 
     for g in [warm_graph] + graphs + prof_graphs + lat:
         sfd.alspec_graph_destroy(g)
+    lens0 = step_layers[0]["lens"]
+    return {
+        "plan": plan, "fused": fused, "kv_bytes": kv_bytes, "n_layers": n_layers,
+        "ms_per_step": ms_per_step, "per_step": per_step, "flush": flush, "l2_bytes": l2_bytes,
+        "mid_ms": mid_ms, "mid_bytes": middle_bytes(wl, lens0, fused), "spec_ms": spec_ms,
+        "layer_ms": layer_ms, "pre_ms": pre_ms, "post_ms": post_ms, "gap_ms": gap_ms,
+        "t_spec": t_spec, "t_exact": t_exact, "n_lat": n_lat, "lat_ms": lat_ms,
+        "lat_flush": lat_flush, "hit_rate": hit_rate, "e2e": e2e, "clocks": clocks.summary(),
+        "launches_per_layer": 1 if fused else (3 if plan["n2"] > 0 else 2),
+    }
+
+
+def spec_summary(m):
+    ratio = [s / l for s, l in zip(m["t_spec"], m["t_exact"])]
+    return {
+        "us_median": statistics.median(m["t_spec"]) * 1e3 if m["t_spec"] else None,
+        "ratio_to_layer_median": statistics.median(ratio) if ratio else None,
+        "layer_us_median": statistics.median(m["t_exact"]) * 1e3 if m["t_exact"] else None,
+        "us_p90": statistics.quantiles(m["t_spec"], n=10)[-1] * 1e3
+        if len(m["t_spec"]) > 1 else None,
+        "from": "kernel-written global-timer stamps: last write of layer l-1's outputs to the "
+                "last write of layer l's O_spec (layer: to the last write of its O_exact and "
+                "flags); graphs of %d distinct layers, layers 1..%d" % (m["n_lat"], m["n_lat"] - 1),
+    }
+
+
+def config_summary(wl, m, world, peak):
+    """One workload's entry in the line's per_config object."""
+    value = job_throughput(m["kv_bytes"], world, m["ms_per_step"])
+    mid_avg = statistics.mean(m["mid_ms"]) if m["mid_ms"] else None
+    mid_gbs = m["mid_bytes"] / (mid_avg * 1e-3) / 1e9 if mid_avg and m["mid_bytes"] else None
+    lat_layer_ms = statistics.median(m["lat_ms"])
+    return {
+        "us_per_step": m["ms_per_step"] * 1e3,
+        "us_per_step_p10_p50_p90": quantiles_us(m["per_step"]),
+        "steps": len(m["per_step"]),
+        "kv_bytes_per_step": m["kv_bytes"],
+        "kv_gbs": value,
+        "frac": value / world / peak,
+        "frac_of_nominal_8000": value / world / NOMINAL_HBM_GBS,
+        "us_per_layer_in_graph": lat_layer_ms * 1e3,
+        "frac_per_layer_in_graph": (m["kv_bytes"] / m["n_layers"]) / (lat_layer_ms * 1e-3) / 1e9
+        / peak,
+        "layer_graph": "%d distinct layers per graph%s" % (
+            m["n_lat"], ", L2 flushed before each" if m["lat_flush"] else ""),
+        "middle_kernel": {"avg_launch_us": mid_avg * 1e3 if mid_avg else None,
+                          "bytes_per_launch": m["mid_bytes"], "gbs": mid_gbs,
+                          "frac": mid_gbs / peak if mid_gbs else None},
+        "spec_latency": spec_summary(m),
+        "hit_rate": m["hit_rate"],
+        "e2e_us_per_step": m["e2e"]["us_per_step"] if m["e2e"] else None,
+        "l2": "flushed before every timed step" if m["flush"] else "inputs larger than L2",
+        "plan": m["plan"],
+        "clocks": m["clocks"],
+    }
+
+
+def run_alspec(args, wl):
+    import torch
+    import workloads
+
+    rank, world, local = dist_env()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    ranks = Ranks("nccl", device)
+    n_layers = args.layers or wl.n_layers
+    m = measure(wl, n_layers, args.steps, args.warmup, device, ranks, args,
+                want_e2e=not args.no_e2e)
+    torch.cuda.empty_cache()
+
+    # Every other workload, a few timed steps each (the same on every rank).
+    peak, peak_kind = measured_peak()
+    per_config = None
+    if not args.no_per_config and args.layers == 0:
+        per_config = {}
+        for idx in sorted(workloads.CONFIGS):
+            other = workloads.CONFIGS[idx]
+            if other.name == wl.name:
+                continue
+            mo = measure(other, other.n_layers, args.per_config_steps, max(3, args.warmup),
+                         device, ranks, args, want_e2e=not args.no_e2e)
+            per_config[other.name] = dict(workload_index=idx,
+                                          **config_summary(other, mo, world, peak))
+            del mo
+            torch.cuda.empty_cache()
     ranks.close()
     if rank != 0:
         return
 
     # Same-run read probe: a 4 GiB stream through bulk copies, nothing else.
-    read_probe = None
-    if rank == 0:
-        nbytes = 4 << 30
-        buf = torch.empty(nbytes, dtype=torch.uint8, device=device)
-        evp = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-        with torch.cuda.stream(stream):
-            for r in range(7):
-                if r == 2:
-                    evp[0].record(stream)
-                assert sfd.alspec_read_probe(buf.data_ptr(), nbytes, stream.cuda_stream) == 0
-            evp[1].record(stream)
-        stream.synchronize()
-        probe_gbs = nbytes * 5 / (evp[0].elapsed_time(evp[1]) * 1e-3) / 1e9
-        read_probe = {"gbs": probe_gbs, "bytes_per_launch": nbytes, "launches": 5}
-        del buf
-    peak, peak_kind = measured_peak()
-    # The dominant kernel: the middle kernel (two-stream schedule) or the one
-    # kernel of the one-launch schedule, which reads every cache row.
-    mid_bytes = sum(
-        (max(0, L - wl.W - min(wl.S, L)) if L > wl.S + wl.W else 0) * wl.Hkv * wl.d * 2 *
-        wl.elem_bytes for L in layers[0]["lens"])
-    if fused:
-        mid_bytes = workloads.kv_bytes(wl, layers[0]["lens"])
-    mid_avg_ms = sum(mid_ms) / len(mid_ms)
-    achieved = mid_bytes / (mid_avg_ms * 1e-3) / 1e9
+    probe = read_probe_fn()
+    nbytes = 4 << 30
+    buf = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    stream = torch.cuda.Stream(device)
+    evp = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    with torch.cuda.stream(stream):
+        for r in range(7):
+            if r == 2:
+                evp[0].record(stream)
+            assert probe(buf.data_ptr(), nbytes, stream.cuda_stream) == 0
+        evp[1].record(stream)
+    stream.synchronize()
+    probe_gbs = nbytes * 5 / (evp[0].elapsed_time(evp[1]) * 1e-3) / 1e9
+    read_probe = {"gbs": probe_gbs, "bytes_per_launch": nbytes, "launches": 5,
+                  "library": "libalspec_read_probe.so"}
+    del buf
+
+    fused = m["fused"]
+    mid_avg_ms = sum(m["mid_ms"]) / len(m["mid_ms"])
+    achieved = m["mid_bytes"] / (mid_avg_ms * 1e-3) / 1e9
     traffic = stored_traffic(FUSED_TRAFFIC_FILE if fused else TRAFFIC_FILE, wl.name)
-    value = job_throughput(kv_bytes, world, ms_per_step)
+    value = job_throughput(m["kv_bytes"], world, m["ms_per_step"])
 
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(wl.replace(n_layers=n_layers), args.cpu_seconds)
 
-    spec_ratio = [s / l for s, l in zip(t_spec, t_exact)]
+    plan = m["plan"]
+    l2_bytes = m["l2_bytes"]
     line = {
         "metric": METRIC,
         "value": value,
@@ -540,64 +687,53 @@ def run_alspec(args, wl):
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
-        "ms_per_step": ms_per_step,
-        "us_per_step": ms_per_step * 1e3,
-        "us_per_step_p10_p50_p90": [float(x * 1e3) for x in
-                                    statistics.quantiles(per_step, n=10)[::4]]
-        if len(per_step) >= 2 else None,
+        "ms_per_step": m["ms_per_step"],
+        "us_per_step": m["ms_per_step"] * 1e3,
+        "us_per_step_p10_p50_p90": quantiles_us(m["per_step"]),
         "frac_of_hbm_peak": value / world / peak,
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": wl.dtype,
         "data": "synthetic",
-        "config": {"workload": wl.name, "layers": n_layers, "batch": wl.B, "q_heads": wl.Hq,
-                   "kv_heads": wl.Hkv, "head_dim": wl.d, "context": wl.L, "sink": wl.S,
-                   "window": wl.W, "lambda": wl.lam, "kv_bytes_per_step": kv_bytes,
-                   "l2": ("L2 flushed before every timed step (untimed write of %d MB, then "
-                          "a read of %d MB of other data); %.1f MB of KV per step"
-                          % (2 * l2_bytes >> 20, 2 * l2_bytes >> 20, kv_bytes / 1e6))
-                   if flush else ("inputs larger than L2: %.1f MB of KV per step against "
-                                  "%d MB of L2; no flush" % (kv_bytes / 1e6, l2_bytes >> 20)),
-                   "parallelism": "replicas" if world > 1 else "single",
-                   "timing": "CUDA graph per step, CUDA events on the launch stream; "
-                             "per-kernel times from a second pass of graphs with per-layer "
-                             "events",
-                   "schedule": {1: "streams", 2: "fused", 3: "sink_first"}[plan["schedule"]],
-                   "plan": plan},
+        "config": workload_config(wl, n_layers, world),
+        "method": {
+            "kv_bytes_per_step": m["kv_bytes"],
+            "l2": ("L2 flushed before every timed step (untimed write of %d MB, then a read "
+                   "of %d MB of other data); %.1f MB of KV per step"
+                   % (2 * l2_bytes >> 20, 2 * l2_bytes >> 20, m["kv_bytes"] / 1e6))
+            if m["flush"] else ("inputs larger than L2: %.1f MB of KV per step against %d MB "
+                                "of L2; no flush" % (m["kv_bytes"] / 1e6, l2_bytes >> 20)),
+            "timing": "CUDA graph per step, CUDA events on the launch stream; per-kernel times "
+                      "from a second pass of graphs with per-layer events",
+            "schedule": {1: "streams", 2: "fused", 3: "sink_first"}[plan["schedule"]],
+            "plan": plan},
         "roofline": {"bound": "hbm",
                      "kernel": "attn_kernel<%s,%d,%d,%s,%s>" % (
                          wl.dtype, wl.d, wl.g, "fused" if fused else "middle",
                          {1: "cuda_cores", 2: "tensor_cores"}.get(plan["engine"], "?")),
                      "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_kind": peak_kind,
-                     "bytes_per_launch": mid_bytes, "avg_launch_us": mid_avg_ms * 1e3,
-                     "launches_measured": len(mid_ms), "traffic": traffic,
+                     "bytes_per_launch": m["mid_bytes"], "avg_launch_us": mid_avg_ms * 1e3,
+                     "launches_measured": len(m["mid_ms"]), "traffic": traffic,
                      "frac_of_nominal_8000": achieved / NOMINAL_HBM_GBS,
-                     "frac_of_same_run_read_probe": (achieved / read_probe["gbs"]
-                                                     if read_probe else None)},
+                     "frac_of_same_run_read_probe": achieved / probe_gbs},
         "read_probe": read_probe,
         "frac_of_nominal_8000": value / world / NOMINAL_HBM_GBS,
-        "spec_latency": {
-            "us_median": statistics.median(t_spec) * 1e3 if t_spec else None,
-            "ratio_to_layer_median": statistics.median(spec_ratio) if spec_ratio else None,
-            "layer_us_median": statistics.median(t_exact) * 1e3 if t_exact else None,
-            "us_p90": statistics.quantiles(t_spec, n=10)[-1] * 1e3 if len(t_spec) > 1 else None,
-            "from": "kernel-written global-timer stamps: last write of layer l-1's "
-                    "outputs to the last write of layer l's O_spec (layer: of its O_exact "
-                    "and flags); graphs as timed, layers 1..%d" % (n_layers - 1),
-            "profiled_graph_us_median": statistics.median(spec_ms) * 1e3,
-            "profiled_graph_layer_us_median": statistics.median(layer_ms) * 1e3},
+        "spec_latency": dict(spec_summary(m),
+                             profiled_graph_us_median=statistics.median(m["spec_ms"]) * 1e3,
+                             profiled_graph_layer_us_median=statistics.median(m["layer_ms"]) * 1e3),
         "layer_breakdown_us_median": {
-            "start_to_middle_kernel": statistics.median(pre_ms) * 1e3,
-            "middle_kernel": statistics.median(mid_ms) * 1e3,
-            "middle_end_to_layer_end": statistics.median(post_ms) * 1e3,
-            "between_layers": statistics.median(gap_ms) * 1e3 if gap_ms else None},
-        "hit_rate": hit_rate,
+            "start_to_middle_kernel": statistics.median(m["pre_ms"]) * 1e3,
+            "middle_kernel": statistics.median(m["mid_ms"]) * 1e3,
+            "middle_end_to_layer_end": statistics.median(m["post_ms"]) * 1e3,
+            "between_layers": statistics.median(m["gap_ms"]) * 1e3 if m["gap_ms"] else None},
+        "hit_rate": m["hit_rate"],
         "cpu_baseline": cpu,
-        "e2e": e2e,
-        "gpu_launches": args.steps * n_layers * (1 if fused else (3 if plan["n2"] > 0 else 2)),
-        "clocks": clocks.summary(),
+        "e2e": m["e2e"],
+        "gpu_launches": args.steps * n_layers * m["launches_per_layer"],
+        "clocks": m["clocks"],
+        "per_config": per_config,
     }
     print(json.dumps(line), flush=True)
 

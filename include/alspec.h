@@ -289,18 +289,6 @@ alspec_status alspec_test_wait_timeout(void* workspace, size_t workspace_bytes, 
                                        void* stream);
 
 /*
- * Read-bandwidth probe (a measurement aid, not part of the decode path):
- * streams `bytes` of `buf` from HBM into shared memory with the same 1-D
- * bulk copies and mbarrier ring the attention kernels use, one CTA per SM,
- * and does nothing else.  Timing it gives the rate a pure streaming read
- * reaches on this GPU.
- *   buf    device, 16-byte aligned;  bytes a positive multiple of 16
- *   err    device uint32 or NULL: ALSPEC_DEVERR_TIMEOUT on a wait timeout
- * Asynchronous on `stream`.
- */
-alspec_status alspec_read_probe(const void* buf, size_t bytes, uint32_t* err, void* stream);
-
-/*
  * Work plan the library would use (host only, no CUDA call except the SM
  * count query).  info[] receives, in order:
  *   0 tokens per sink-set work item      1 sink-set items per (b, kv head)
@@ -383,17 +371,21 @@ int alspec_last_cuda_error(void);
  *
  *   - A problem whose workspace (alspec_workspace_size) is larger than
  *     ALSPEC_NOALLOC_SCRATCH_BYTES is rejected with ALSPEC_ERR_WORKSPACE
- *     before anything is launched.
+ *     before anything is launched.  Every other argument is checked as by
+ *     alspec_decode, also before anything is queued: a rejected call leaves
+ *     the array untouched.
  *   - The first call on a device looks up the device address of the array
  *     (cudaGetSymbolAddress) with that device current; make that first call
- *     outside any stream capture.
+ *     outside any stream capture.  The address is kept until
+ *     alspec_shutdown, which must precede a cudaDeviceReset.
  *   - Each call clears the array's counters on `stream`, then runs exactly
  *     what alspec_decode runs.  All calls on a device share the one array:
  *     calls that overlap on the GPU (different streams without ordering
  *     between them) race and corrupt each other's results.  Calls ordered
  *     on one stream are fine.
- *   - There is no spec_event and no profiling events; the device error word
- *     is not readable (use alspec_decode with a workspace for that).
+ *   - There is no spec_event and no profiling events.  The device error
+ *     word of the array (a clamped seq_lens entry, an in-kernel wait that
+ *     gave up) is read with alspec_noalloc_device_error.
  */
 #define ALSPEC_NOALLOC_SCRATCH_BYTES (8u << 20)
 alspec_status alspec_decode_noalloc(const alspec_desc* desc,
@@ -401,6 +393,16 @@ alspec_status alspec_decode_noalloc(const alspec_desc* desc,
                                     const int32_t* seq_lens, int n_sink, int window,
                                     float lambda, float* out_spec, float* out_exact,
                                     float* rel_l2, uint8_t* commit, void* stream);
+
+/*
+ * Read (and clear) the device error word of alspec_decode_noalloc's scratch
+ * array on the current device, as alspec_get_device_error does for a
+ * workspace: synchronizes `stream`; *err (host) receives the bitwise OR of
+ * ALSPEC_DEVERR_* raised since the last read.  Returns ALSPEC_OK, or
+ * ALSPEC_ERR_DEVICE_DATA / ALSPEC_ERR_TIMEOUT when the word is non-zero,
+ * ALSPEC_ERR_INVALID_ARG for a NULL err.  Allocates nothing.
+ */
+alspec_status alspec_noalloc_device_error(void* stream, uint32_t* err);
 
 #ifdef __cplusplus
 }

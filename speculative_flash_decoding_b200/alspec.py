@@ -75,10 +75,10 @@ SIGNATURES = {
     "alspec_last_cuda_error": (_i, []),
     "alspec_decode_noalloc": (_i, [_descp, _vp, _vp, _vp, _vp, _i, _i, _f, _vp, _vp, _vp, _vp,
                                    _vp]),
+    "alspec_noalloc_device_error": (_i, [_vp, _u32p]),
     "alspec_decode_traced": (_i, [_descp, _vp, _vp, _vp, _vp, _i, _i, _f, _vp, _vp, _vp, _vp,
                                   _vp, _sz, _vp, _vp]),
     "alspec_oproj": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp]),
-    "alspec_read_probe": (_i, [_vp, _sz, _vp, _vp]),
     "alspec_test_wait_timeout": (_i, [_vp, _sz, _i, _vp]),
     "alspec_decode_oproj": (_i, [_descp, _vp, _vp, _vp, _vp, _i, _i, _f, _vp, _i, _vp, _vp,
                                  _vp, _vp, _vp, _i, _vp, _sz, _vp, _vp]),
@@ -176,11 +176,6 @@ def alspec_test_wait_timeout(workspace: int, workspace_bytes: int, timeout_ms: i
     return int(_lib.alspec_test_wait_timeout(workspace, workspace_bytes, timeout_ms, stream))
 
 
-def alspec_read_probe(buf: int, nbytes: int, stream: int, err: int = 0) -> int:
-    """Stream nbytes of buf from HBM (bandwidth probe)."""
-    return int(_lib.alspec_read_probe(buf, nbytes, err or None, stream))
-
-
 def alspec_decode_noalloc(desc: alspec_desc, q: int, k_cache: int, v_cache: int, seq_lens: int,
                           n_sink: int, window: int, lam: float, out_spec: int, out_exact: int,
                           rel_l2: int, commit: int, stream: int) -> int:
@@ -190,6 +185,14 @@ def alspec_decode_noalloc(desc: alspec_desc, q: int, k_cache: int, v_cache: int,
     return int(_lib.alspec_decode_noalloc(ctypes.byref(desc), q, k_cache, v_cache, seq_lens,
                                           n_sink, window, lam, out_spec, out_exact, rel_l2,
                                           commit, stream))
+
+
+def alspec_noalloc_device_error(stream: int):
+    """(status, error word) of alspec_decode_noalloc's scratch on the current
+    device (read and cleared; synchronizes the stream)."""
+    err = ctypes.c_uint32(0)
+    st = int(_lib.alspec_noalloc_device_error(stream, ctypes.byref(err)))
+    return st, int(err.value)
 
 
 def alspec_query_plan(desc: alspec_desc, n_sink: int, window: int):

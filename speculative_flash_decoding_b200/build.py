@@ -1,4 +1,7 @@
-"""Build libalspec.so in-tree with nvcc for sm_100a.
+"""Build the package's shared libraries in-tree with nvcc for sm_100a:
+libalspec.so (the decode library, include/alspec.h) and
+libalspec_read_probe.so (the benchmark's read-bandwidth probe,
+include/alspec_read_probe.h).
 
 Usage: python speculative_flash_decoding_b200/build.py [--force] [-v]
 (run by path: importing the package needs the built library)
@@ -12,9 +15,15 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libalspec.so")
-SOURCES = [os.path.join(CSRC, "alspec.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cuh", ".h"))] + [
-    os.path.join(INCLUDE, "alspec.h")]
+PROBE_LIB = os.path.join(PKG, "libalspec_read_probe.so")
+# (library, its source, the headers it depends on)
+TARGETS = [
+    (LIB, os.path.join(CSRC, "alspec.cu"),
+     [os.path.join(CSRC, f) for f in ("attn_kernels.cuh", "oproj_kernels.cuh", "ptx.cuh")] +
+     [os.path.join(INCLUDE, "alspec.h")]),
+    (PROBE_LIB, os.path.join(CSRC, "read_probe.cu"),
+     [os.path.join(CSRC, "ptx.cuh"), os.path.join(INCLUDE, "alspec_read_probe.h")]),
+]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -30,18 +39,23 @@ def nvcc() -> str:
     return "nvcc"
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile csrc/alspec.cu into the package's libalspec.so; return its path."""
-    if not force and os.path.exists(LIB):
-        newest = max(os.path.getmtime(p) for p in DEPS)
-        if os.path.getmtime(LIB) >= newest:
-            return LIB
-    tmp = LIB + ".tmp"
-    cmd = [nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-o", tmp, *SOURCES]
+def _build_one(lib: str, src: str, deps, force: bool, verbose: bool) -> None:
+    if not force and os.path.exists(lib):
+        newest = max(os.path.getmtime(p) for p in [src, *deps])
+        if os.path.getmtime(lib) >= newest:
+            return
+    tmp = lib + ".tmp"
+    cmd = [nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-o", tmp, src]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
+    os.replace(tmp, lib)
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    """Compile every library of the package; return the decode library's path."""
+    for lib, src, deps in TARGETS:
+        _build_one(lib, src, deps, force, verbose)
     return LIB
 
 

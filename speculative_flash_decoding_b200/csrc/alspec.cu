@@ -19,7 +19,6 @@
 #include "alspec.h"
 #include "attn_kernels.cuh"
 #include "oproj_kernels.cuh"
-#include "probe_kernels.cuh"
 
 namespace alspec {
 namespace {
@@ -475,6 +474,9 @@ alspec_status launch(KernelFn fn, dim3 grid, dim3 block, int smem, cudaStream_t 
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Forget the no-alloc scratch addresses looked up so far (alspec_shutdown).
+void noalloc_forget();
+
 }  // namespace
 }  // namespace alspec
 
@@ -577,7 +579,8 @@ alspec_status decode_impl(const alspec_desc* desc, const void* q, const void* k_
                           float lambda, float* out_spec, float* out_exact, float* rel_l2,
                           uint8_t* commit, void* workspace, size_t workspace_bytes, void* stream,
                           void* spec_event, void* const* prof_events,
-                          unsigned long long* trace_ns, const OprojReq* op = nullptr) {
+                          unsigned long long* trace_ns, const OprojReq* op = nullptr,
+                          bool clear_counters = false) {
     alspec_status st = check_desc(desc, n_sink, window);
     if (st != ALSPEC_OK) return st;
     if (reinterpret_cast<uintptr_t>(trace_ns) & 7u) return ALSPEC_ERR_INVALID_ARG;
@@ -651,6 +654,13 @@ alspec_status decode_impl(const alspec_desc* desc, const void* q, const void* k_
     p.timeout_ns = (unsigned long long)(desc->timeout_ms > 0 ? desc->timeout_ms : 2000) * 1000000ull;
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // A workspace that is not the caller's own (alspec_decode_noalloc's
+    // shared scratch) gets its counters cleared first, once every check has
+    // passed, so that a rejected call leaves nothing queued.
+    if (clear_counters &&
+        !ok(cudaMemsetAsync(p.ctr, 0, (size_t)ctr_words(desc->batch, desc->n_kv_heads) *
+                                          sizeof(unsigned), s)))
+        return ALSPEC_ERR_CUDA;
     auto prof = [&](int i, cudaStream_t on) {
         return !prof_events || !prof_events[i] ||
                ok(record_event(static_cast<cudaEvent_t>(prof_events[i]), on));
@@ -865,25 +875,6 @@ alspec_status alspec_test_wait_timeout(void* workspace, size_t workspace_bytes, 
     return ok(cudaGetLastError()) ? ALSPEC_OK : ALSPEC_ERR_CUDA;
 }
 
-alspec_status alspec_read_probe(const void* buf, size_t bytes, uint32_t* err, void* stream) {
-    if (!buf || !aligned16(buf) || bytes == 0 || bytes % 16 != 0 ||
-        (reinterpret_cast<uintptr_t>(err) & 3u))
-        return ALSPEC_ERR_INVALID_ARG;
-    DeviceState* ds = nullptr;
-    alspec_status st = get_device_state(&ds);
-    if (st != ALSPEC_OK) return st;
-    if ((st = ensure_smem_attr(ds, reinterpret_cast<const void*>(read_probe_kernel), kRpSmem)) !=
-        ALSPEC_OK)
-        return st;
-    ReadProbeParams rp{};
-    rp.buf = static_cast<const unsigned char*>(buf);
-    rp.bytes = bytes;
-    rp.err = err;
-    rp.timeout_ns = 2000000000ull;
-    read_probe_kernel<<<ds->sm_count, 64, kRpSmem, static_cast<cudaStream_t>(stream)>>>(rp);
-    return ok(cudaGetLastError()) ? ALSPEC_OK : ALSPEC_ERR_CUDA;
-}
-
 alspec_status alspec_get_device_error(void* workspace, size_t workspace_bytes, void* stream,
                                       uint32_t* err) {
     if (!workspace || !err || workspace_bytes < (kCtrFixed * sizeof(unsigned)))
@@ -937,6 +928,7 @@ alspec_status alspec_graph_destroy(void* graph) {
 }
 
 alspec_status alspec_shutdown(void) {
+    noalloc_forget();
     std::lock_guard<std::mutex> lock(g_mutex);
     int cur = 0;
     const bool have_cur = cudaGetDevice(&cur) == cudaSuccess;
@@ -982,6 +974,7 @@ int alspec_last_cuda_error(void) { return (int)t_last_error; }
 
 // ------------------------------------------------------------ no-alloc path
 
+namespace alspec {
 namespace {
 
 // Scratch space of alspec_decode_noalloc: a fixed array in this library's
@@ -990,14 +983,15 @@ namespace {
 // address looked up below.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[ALSPEC_NOALLOC_SCRATCH_BYTES];
 
+std::mutex g_noalloc_mutex;
 void* g_noalloc_ptr[kMaxDevices] = {};
 
 // Device address of the scratch array on the current device, looked up once
-// per device (with that device current).
+// per device (with that device current) and kept until alspec_shutdown.
 alspec_status noalloc_scratch(void** out) {
     int dev = 0;
     if (!ok(cudaGetDevice(&dev)) || dev < 0 || dev >= kMaxDevices) return ALSPEC_ERR_CUDA;
-    std::lock_guard<std::mutex> lock(g_mutex);
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
     if (!g_noalloc_ptr[dev]) {
         void* ptr = nullptr;
         if (!ok(cudaGetSymbolAddress(&ptr, g_noalloc_scratch)) || !ptr) return ALSPEC_ERR_CUDA;
@@ -1007,7 +1001,13 @@ alspec_status noalloc_scratch(void** out) {
     return ALSPEC_OK;
 }
 
+void noalloc_forget() {
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    for (void*& p : g_noalloc_ptr) p = nullptr;
+}
+
 }  // namespace
+}  // namespace alspec
 
 extern "C" alspec_status alspec_decode_noalloc(const alspec_desc* desc, const void* q,
                                                const void* k_cache, const void* v_cache,
@@ -1021,14 +1021,20 @@ extern "C" alspec_status alspec_decode_noalloc(const alspec_desc* desc, const vo
     }
     if (need > ALSPEC_NOALLOC_SCRATCH_BYTES) return ALSPEC_ERR_WORKSPACE;
     void* scratch = nullptr;
-    alspec_status st = noalloc_scratch(&scratch);
+    const alspec_status st = noalloc_scratch(&scratch);
     if (st != ALSPEC_OK) return st;
-    // The counters at the head of the scratch must start at zero; the rest
-    // of it is written before it is read within a call.
-    const size_t counters = (size_t)ctr_words(desc->batch, desc->n_kv_heads) * sizeof(unsigned);
-    if (!ok(cudaMemsetAsync(scratch, 0, counters, static_cast<cudaStream_t>(stream))))
-        return ALSPEC_ERR_CUDA;
-    return alspec_decode(desc, q, k_cache, v_cache, seq_lens, n_sink, window, lambda, out_spec,
-                         out_exact, rel_l2, commit, scratch, ALSPEC_NOALLOC_SCRATCH_BYTES, stream,
-                         nullptr, nullptr);
+    // The counters at the head of the scratch are cleared on `stream` once
+    // the call's arguments have passed every check; the rest of the scratch
+    // is written before it is read within a call.
+    return decode_impl(desc, q, k_cache, v_cache, seq_lens, n_sink, window, lambda, out_spec,
+                       out_exact, rel_l2, commit, scratch, ALSPEC_NOALLOC_SCRATCH_BYTES, stream,
+                       nullptr, nullptr, nullptr, nullptr, /*clear_counters=*/true);
+}
+
+extern "C" alspec_status alspec_noalloc_device_error(void* stream, uint32_t* err) {
+    if (!err) return ALSPEC_ERR_INVALID_ARG;
+    void* scratch = nullptr;
+    const alspec_status st = noalloc_scratch(&scratch);
+    if (st != ALSPEC_OK) return st;
+    return alspec_get_device_error(scratch, ALSPEC_NOALLOC_SCRATCH_BYTES, stream, err);
 }

@@ -1,12 +1,14 @@
-// Read-bandwidth probe: how fast this GPU streams a large buffer from HBM
+// libalspec_read_probe.so: a read-bandwidth probe, kept out of the decode
+// library.  It measures how fast this GPU streams a large buffer from HBM
 // into shared memory with the same machinery the attention kernels use
 // (1-D bulk copies into an mbarrier-guarded ring, one CTA per SM).  The
 // benchmark reports the middle kernel's rate against it, beside the
 // measured copy peak and the nominal HBM bandwidth.
-#pragma once
+#include <cuda_runtime.h>
 
 #include <cstdint>
 
+#include "alspec_read_probe.h"
 #include "ptx.cuh"
 
 namespace alspec {
@@ -83,3 +85,24 @@ __global__ void __launch_bounds__(64, 1) read_probe_kernel(const __grid_constant
 }
 
 }  // namespace alspec
+
+extern "C" int alspec_read_probe(const void* buf, size_t bytes, uint32_t* err, void* stream) {
+    using namespace alspec;
+    const uintptr_t a = reinterpret_cast<uintptr_t>(buf);
+    if (!buf || (a & 15u) || bytes == 0 || bytes % 16 != 0 ||
+        (reinterpret_cast<uintptr_t>(err) & 3u))
+        return 1;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaFuncSetAttribute(reinterpret_cast<const void*>(read_probe_kernel),
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, kRpSmem) != cudaSuccess)
+        return 4;
+    ReadProbeParams rp{};
+    rp.buf = static_cast<const unsigned char*>(buf);
+    rp.bytes = bytes;
+    rp.err = err;
+    rp.timeout_ns = 2000000000ull;
+    read_probe_kernel<<<sms, 64, kRpSmem, static_cast<cudaStream_t>(stream)>>>(rp);
+    return cudaGetLastError() == cudaSuccess ? 0 : 4;
+}

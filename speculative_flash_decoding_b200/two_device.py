@@ -24,7 +24,11 @@ Llama-3.1-8B shapes, tens of nanoseconds on NVLink 5 -- so both ranks post
 the same messages without reading the flags on the host.
 
 The decode and projection calls are parameters (``decode_fn``,
-``project_fn``); by default they are this library's CUDA entry points.
+``project_fn``); by default they are this library's CUDA entry points.  So
+is the transport (``send_fn`` on the attention rank, ``recv_fn`` on the
+projection rank): by default torch.distributed's point-to-point ``isend``
+and ``recv``.  A send is issued on the CUDA stream current at the call -- the
+side stream for O_spec -- and returns a handle with ``wait()``.
 """
 from __future__ import annotations
 
@@ -48,15 +52,24 @@ def _default_project(x, w, y, skip):
         raise ab.AlspecError(st, "alspec_oproj")
 
 
+def _isend(tensor, peer, group):
+    return dist.isend(tensor, peer, group=group)
+
+
+def _recv(tensor, peer, group):
+    dist.recv(tensor, peer, group=group)
+
+
 class AttentionRank:
     """The rank that owns the KV cache: decode, then stream the results to
     the projection rank ``peer``."""
 
-    def __init__(self, decoder, peer: int, group=None, decode_fn=None):
+    def __init__(self, decoder, peer: int, group=None, decode_fn=None, send_fn=None):
         self.decoder = decoder
         self.peer = peer
         self.group = group
         self.decode_fn = decode_fn
+        self.send = send_fn or _isend
         self._side = None
 
     def step(self, q, k, v, seq_lens, lam):
@@ -78,30 +91,31 @@ class AttentionRank:
                 self._side = torch.cuda.Stream(q.device, priority=-1)
             self._side.wait_event(spec_ready)
             with torch.cuda.stream(self._side):
-                works.append(dist.isend(out["out_spec"].reshape(B, -1), self.peer,
-                                        group=self.group))
+                works.append(self.send(out["out_spec"].reshape(B, -1), self.peer, self.group))
             # The messages of a pair complete in issue order; the flags and
             # O_exact follow on the caller's stream, after the decode.
             torch.cuda.current_stream(q.device).wait_stream(self._side)
         else:
-            works.append(dist.isend(out["out_spec"].reshape(B, -1).contiguous(), self.peer,
-                                    group=self.group))
-        works.append(dist.isend(out["commit"].contiguous(), self.peer, group=self.group))
-        works.append(dist.isend(out["out_exact"].reshape(B, -1).contiguous(), self.peer,
-                                group=self.group))
+            works.append(self.send(out["out_spec"].reshape(B, -1).contiguous(), self.peer,
+                                   self.group))
+        works.append(self.send(out["commit"].contiguous(), self.peer, self.group))
+        works.append(self.send(out["out_exact"].reshape(B, -1).contiguous(), self.peer,
+                               self.group))
         return out, works
 
 
 class ProjectionRank:
     """The rank that runs the post-attention projection speculatively."""
 
-    def __init__(self, w_o, batch: int, kdim: int, peer: int, group=None, project_fn=None):
+    def __init__(self, w_o, batch: int, kdim: int, peer: int, group=None, project_fn=None,
+                 recv_fn=None):
         self.w = w_o
         self.batch = batch
         self.kdim = kdim
         self.peer = peer
         self.group = group
         self.project_fn = project_fn or _default_project
+        self.recv = recv_fn or _recv
 
     def step(self):
         """One layer: returns (y, o_spec, commit, o_exact) as received and
@@ -112,11 +126,11 @@ class ProjectionRank:
         commit = torch.empty(B, dtype=torch.uint8, device=dev)
         o_exact = torch.empty(B, K, dtype=torch.float32, device=dev)
         y = torch.empty(B, N, dtype=torch.float32, device=dev)
-        dist.recv(o_spec, self.peer, group=self.group)
+        self.recv(o_spec, self.peer, self.group)
         # Speculative: project O_spec for every token at once.
         self.project_fn(o_spec, self.w, y, None)
-        dist.recv(commit, self.peer, group=self.group)
-        dist.recv(o_exact, self.peer, group=self.group)
+        self.recv(commit, self.peer, self.group)
+        self.recv(o_exact, self.peer, self.group)
         # Verified: redo the discarded tokens' rows on O_exact.
         self.project_fn(o_exact, self.w, y, commit)
         return y, o_spec, commit, o_exact

@@ -10,12 +10,17 @@ import pytest
 import speculative_flash_decoding_b200 as sfd
 from speculative_flash_decoding_b200 import alspec as ab
 
-HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include",
-                      "alspec.h")
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+INCLUDE = os.path.join(ROOT, "include")
+PKG = os.path.join(ROOT, "speculative_flash_decoding_b200")
+HEADER = os.path.join(INCLUDE, "alspec.h")
+# Every header under include/ and the library that implements it.
+LIBRARY_OF = {"alspec.h": os.path.join(PKG, "libalspec.so"),
+              "alspec_read_probe.h": os.path.join(PKG, "libalspec_read_probe.so")}
 
 
-def declared_functions():
-    text = open(HEADER).read()
+def declared_functions(header=HEADER):
+    text = open(header).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     return sorted(set(re.findall(r"\b(alspec_[a-z_0-9]+)\s*\(", text)))
 
@@ -26,10 +31,22 @@ def test_header_declares_the_binding_surface():
     assert set(names) == set(ab.SIGNATURES), "binding and header disagree"
 
 
-def test_library_exports_every_declared_symbol():
-    lib = ctypes.CDLL(sfd.LIB_PATH)
-    for name in declared_functions():
-        assert hasattr(lib, name), f"libalspec.so does not export {name}"
+def test_every_header_has_its_library():
+    assert sorted(f for f in os.listdir(INCLUDE) if f.endswith(".h")) == sorted(LIBRARY_OF)
+
+
+@pytest.mark.parametrize("header", sorted(LIBRARY_OF))
+def test_library_exports_every_declared_symbol(header):
+    names = declared_functions(os.path.join(INCLUDE, header))
+    assert names
+    lib = ctypes.CDLL(LIBRARY_OF[header])
+    for name in names:
+        assert hasattr(lib, name), f"{os.path.basename(LIBRARY_OF[header])} does not export {name}"
+
+
+def test_decode_library_has_no_benchmark_probe():
+    """The read-bandwidth probe is a measurement aid in its own library."""
+    assert not hasattr(ctypes.CDLL(sfd.LIB_PATH), "alspec_read_probe")
 
 
 def test_version_and_status_strings():
@@ -169,7 +186,22 @@ def test_traced_decode_rejects_bad_trace_buffer(trace, code):
 @pytest.mark.parametrize("buf,nbytes", [(0, 1024), ((1 << 20) + 8, 1024), (1 << 20, 1000),
                                         (1 << 20, 0)])
 def test_read_probe_rejects_bad_buffers(buf, nbytes):
-    assert sfd.alspec_read_probe(buf, nbytes, 0) == ab.ALSPEC_ERR_INVALID_ARG
+    import bench
+    assert bench.read_probe_fn()(buf, nbytes, 0) == ab.ALSPEC_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("kw", [dict(max_seq_len=0), dict(head_dim=96), dict(n_kv_heads=3)])
+def test_noalloc_rejects_bad_descriptions_before_launching(kw):
+    d = desc(**kw)
+    fake = 1 << 20
+    st = sfd.alspec_decode_noalloc(d, fake, fake, fake, fake, 4, 64, 0.1, fake, fake, fake, fake,
+                                   0)
+    assert st in (ab.ALSPEC_ERR_INVALID_ARG, ab.ALSPEC_ERR_UNSUPPORTED)
+
+
+def test_noalloc_error_getter_needs_an_output():
+    from speculative_flash_decoding_b200 import alspec as abm
+    assert abm._lib.alspec_noalloc_device_error(None, None) == ab.ALSPEC_ERR_INVALID_ARG
 
 
 @pytest.mark.parametrize("ws,nbytes,ms", [(0, 4096, 1), (1 << 20, 4096, 0), (1 << 20, 4096, 20000),

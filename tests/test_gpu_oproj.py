@@ -125,11 +125,11 @@ def test_graph_with_all_committed_skips_the_recomputation(cuda_device, gate):
 
 
 def test_read_probe_streams_without_error(cuda_device):
-    import speculative_flash_decoding_b200 as sfd
+    import bench
     buf = torch.empty(256 << 20, dtype=torch.uint8, device=cuda_device)
     err = torch.zeros(1, dtype=torch.int32, device=cuda_device)
     s = torch.cuda.current_stream()
-    assert sfd.alspec_read_probe(buf.data_ptr(), buf.numel() - 48, s.cuda_stream,
+    assert bench.read_probe_fn()(buf.data_ptr(), buf.numel() - 48, s.cuda_stream,
                                  err.data_ptr()) == 0
     torch.cuda.synchronize()
     assert err.item() == 0

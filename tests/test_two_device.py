@@ -135,3 +135,113 @@ def test_default_projection_on_one_gpu(cuda_device):
     wf = w.double()
     want = torch.where(skip.bool()[:, None], x.double() @ wf.T, x2.double() @ wf.T)
     assert torch.allclose(y.double(), want, rtol=1e-4, atol=1e-4)
+
+
+class _LocalLink:
+    """Same-GPU stand-in for the NCCL transport: a send copies its tensor,
+    on the CUDA stream current at the send (the attention rank's side
+    stream for O_spec), into a buffer of its own and records a timing event
+    after the copy; a receive waits for that event and takes the oldest
+    message.  Point-to-point messages of a pair arrive in issue order, as
+    with NCCL."""
+
+    class _Done:
+        def wait(self):
+            return True
+
+    def __init__(self):
+        import collections
+        self.pending = collections.deque()
+        self.sent = []
+
+    def send(self, tensor, peer, group=None):
+        import torch
+        buf = torch.empty_like(tensor)
+        buf.copy_(tensor, non_blocking=True)
+        ev = torch.cuda.Event(enable_timing=True)
+        ev.record()
+        self.pending.append((buf, ev))
+        self.sent.append((buf, ev))
+        return self._Done()
+
+    def recv(self, tensor, peer, group=None):
+        import torch
+        buf, ev = self.pending.popleft()
+        torch.cuda.current_stream(tensor.device).wait_event(ev)
+        tensor.copy_(buf)
+
+
+class _EventDecoder:
+    """The library's Decoder, with timing events on every call (events [0]
+    at the call's start and [4] when all of its work is complete)."""
+
+    def __init__(self, dec):
+        self.dec = dec
+        self.events = None
+
+    def decode(self, q, k, v, seq_lens, lam, spec_event=None):
+        import torch
+        import speculative_flash_decoding_b200 as sfd
+        self.events = [torch.cuda.Event(enable_timing=True) for _ in range(sfd.ALSPEC_PROF_EVENTS)]
+        for e in self.events:
+            e.record()  # gives each event its CUDA handle
+        return self.dec.decode(q, k, v, seq_lens, lam, spec_event=spec_event,
+                               prof_events=self.events)
+
+
+@pytest.mark.gpu
+def test_spec_event_branch_on_one_gpu(cuda_device):
+    """The attention rank with the real CUDA decoder (no decode_fn): O_spec
+    leaves from the side stream at spec_event while the exact path runs.
+    The received O_spec is the decoder's bit for bit, it was sent before the
+    decode's work completed, and the projection rank's y follows the
+    oracle's chain (project O_spec, redo discarded rows on O_exact)."""
+    import torch
+    import oracle
+    import workloads
+    import speculative_flash_decoding_b200 as sfd
+    from speculative_flash_decoding_b200 import two_device
+    from parity import FLAG_BAND, oracle_decode
+
+    # Long caches (so the exact path runs well past O_spec), strong sinks and
+    # a few needles (so the flags mix commit and discard).
+    wl = workloads.COMMIT_VARIANT.replace(L=65536, ragged=(49152, 65536))
+    hidden = 1024
+    kdim = wl.Hq * wl.d
+    g = torch.Generator().manual_seed(11)
+    w = (torch.randn(hidden, kdim, generator=g) / 64).to(torch.bfloat16).to(cuda_device)
+    link = _LocalLink()
+    dec = _EventDecoder(sfd.Decoder(wl.B, wl.Hq, wl.Hkv, wl.d, wl.L, wl.dtype, wl.S, wl.W,
+                                    device=cuda_device))
+    att = two_device.AttentionRank(dec, peer=1, send_fn=link.send)
+    proj = two_device.ProjectionRank(w, wl.B, kdim, peer=0, recv_fn=link.recv)
+    for layer in range(2):
+        data = workloads.make_layer(wl, layer=layer, device=cuda_device)
+        out, works = att.step(data["q"], data["k"], data["v"], data["seq_lens"], wl.lam)
+        for wk in works:
+            wk.wait()
+        (spec_buf, spec_ev), (commit_buf, _), (exact_buf, _) = link.sent[-3:]
+        y, o_spec, commit, o_exact = proj.step()
+        torch.cuda.synchronize(cuda_device)
+        # What crossed is what the decoder wrote.
+        assert torch.equal(spec_buf, out["out_spec"].reshape(wl.B, -1))
+        assert torch.equal(o_spec, out["out_spec"].reshape(wl.B, -1))
+        assert torch.equal(commit, out["commit"])
+        assert torch.equal(o_exact, out["out_exact"].reshape(wl.B, -1))
+        # O_spec was on its way before the decode's work (exact path, merge,
+        # flags) was complete -- well before, with these cache lengths.
+        start, done = dec.events[0], dec.events[4]
+        t_spec = start.elapsed_time(spec_ev)
+        t_done = start.elapsed_time(done)
+        assert 0 < t_spec < 0.5 * t_done, (t_spec, t_done)
+        # The projection rank's result against the oracle's chain.
+        ref = oracle_decode(wl, data)
+        assert not (np.abs(ref["rel_l2"] - wl.lam) <= FLAG_BAND).any()
+        assert (commit.cpu().numpy() == ref["commit"]).all()
+        assert 0 < ref["commit"].sum() < wl.B, "the flags should mix commit and discard"
+        chain = oracle.oproj_gated(ref["out_spec"].reshape(wl.B, -1),
+                                   ref["out_exact"].reshape(wl.B, -1), ref["commit"],
+                                   workloads.to_numpy_bits(w))
+        got = y.double().cpu().numpy()
+        rel = np.linalg.norm(got - chain, axis=-1) / np.linalg.norm(chain, axis=-1)
+        assert rel.max() < 2e-3, rel
