@@ -3,9 +3,9 @@
 
 One step = one decode token through the 32 layers of a Llama-3.1-8B-shaped
 model at 131072 context (batch 1, 32 query / 8 KV heads, d 128, bf16 KV
-cache, sink 4, window 1024, lambda 0.10): per layer the sink-set kernel (on a
-high-priority stream), the split exact-attention kernel and the merge +
-relative-L2 + flag kernel, all captured in one CUDA graph.  Layers are
+cache, sink 4, window 1024, lambda 0.10): per layer the sink-set kernel (at
+high launch priority), the split exact-attention kernel beside it and the
+merge + relative-L2 + flag kernel, all captured in one CUDA graph.  Layers are
 independent caches generated from the seed; inputs are resident in HBM.
 
 The other four workloads (a tiny fp32 layer, a 32K layer, a ragged batch of
@@ -64,9 +64,10 @@ def parse_args():
     ap.add_argument("--engine", default="auto", choices=["auto", "cuda_cores", "tensor_cores"])
     ap.add_argument("--schedule", default="auto",
                     choices=["auto", "streams", "fused", "sink_first"],
-                    help="launch schedule: streams (sink set on a high-priority stream beside "
-                         "the exact path, three kernels), fused (one persistent launch) or "
-                         "sink_first (sink set alone first); auto = streams")
+                    help="launch schedule: streams (sink-set, exact-path and merge kernels "
+                         "chained on one stream, the exact path beside the sink set), fused "
+                         "(one persistent launch) or sink_first (the exact path after the sink "
+                         "set); auto = streams")
     ap.add_argument("--oproj", action="store_true",
                     help="speculative output projection against the serial one (32 x 128K)")
     ap.add_argument("--lambda-sweep", action="store_true",
@@ -184,9 +185,18 @@ class ClockSampler:
                                          text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
+            # nvidia-smi takes a while to start; a timed region shorter than
+            # that would get no sample, so wait for the first one (3 s at most).
+            t0 = time.time()
+            while not self.lines and self.proc.poll() is None and time.time() - t0 < 3.0:
+                time.sleep(0.01)
         except OSError:
             self.proc = None
         return self
+
+    def mark(self):
+        """Start of the region of interest: samples from here on count."""
+        self.start = len(self.lines)
 
     def _read(self):
         for line in self.proc.stdout:
@@ -204,7 +214,7 @@ class ClockSampler:
 
     def summary(self):
         mhz, mx, reasons = [], None, set()
-        for line in self.lines:
+        for line in self.lines[getattr(self, "start", 0):]:
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 7:
                 continue
@@ -313,6 +323,15 @@ def read_probe_fn():
     return lambda buf, nbytes, stream, err=0: int(fn(buf, nbytes, err or None, stream))
 
 
+def gpu_uuid(device):
+    import torch
+    try:
+        uuid = str(torch.cuda.get_device_properties(device).uuid)
+        return uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+    except Exception:
+        return None
+
+
 def workload_config(wl, n_layers, world):
     """The `config` object of both arms' lines: the workload, nothing about
     how either arm runs it."""
@@ -345,13 +364,16 @@ def measure(wl, n_layers, steps, warmup, device, ranks, args, want_e2e=True, lat
 
     A step is one decode token through the workload's n_layers layers (each
     its own seeded cache, all resident in HBM): per layer the sink-set
-    kernel on the library's high-priority stream, the exact-path (middle)
-    kernel and the merge, captured as one CUDA graph per step.  Passes:
+    kernel (high launch priority), the exact-path (middle) kernel beside it
+    and the merge, captured as one CUDA graph per step.  Passes:
       timed     `steps` graph replays, CUDA events on the launch stream;
                 a step whose caches fit a few times in L2 is preceded by an
                 untimed L2 flush and timed on its own;
       profiled  the same step with per-layer event nodes: the middle
-                kernel's duration (the roofline's denominator);
+                kernel's duration (the roofline's denominator).  Events
+                between the kernels take away their overlap, so there the
+                middle kernel runs once the sink-set kernel has completed:
+                its duration alone;
       latency   graphs through the traced entry point (kernel-written time
                 stamps of O_spec's and O_exact's publication), over the
                 step's layers, or over `lat_layers` distinct layers when the
@@ -426,12 +448,7 @@ def measure(wl, n_layers, steps, warmup, device, ranks, args, want_e2e=True, lat
         sfd.alspec_graph_launch(warm_graph, stream.cuda_stream)
     ranks.barrier()
 
-    uuid = None
-    try:
-        uuid = str(torch.cuda.get_device_properties(device).uuid)
-        uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
-    except Exception:
-        uuid = None
+    uuid = gpu_uuid(device)
     # Steps whose cache fits a few times in L2 are preceded by an untimed
     # write of twice the L2 size, then a read of another such buffer (so the
     # step does not pay for writing the flush's dirty lines back); each step
@@ -458,6 +475,7 @@ def measure(wl, n_layers, steps, warmup, device, ranks, args, want_e2e=True, lat
     nvtx = torch.cuda.nvtx
     with ClockSampler(uuid) as clocks:
         ranks.barrier()
+        clocks.mark()
         nvtx.range_push("timed steps " + wl.name)
         t_start.record(stream)
         for i in range(steps):
@@ -614,7 +632,6 @@ def config_summary(wl, m, world, peak):
         "e2e_us_per_step": m["e2e"]["us_per_step"] if m["e2e"] else None,
         "l2": "flushed before every timed step" if m["flush"] else "inputs larger than L2",
         "plan": m["plan"],
-        "clocks": m["clocks"],
     }
 
 
@@ -636,16 +653,20 @@ def run_alspec(args, wl):
     per_config = None
     if not args.no_per_config and args.layers == 0:
         per_config = {}
-        for idx in sorted(workloads.CONFIGS):
-            other = workloads.CONFIGS[idx]
-            if other.name == wl.name:
-                continue
-            mo = measure(other, other.n_layers, args.per_config_steps, max(3, args.warmup),
-                         device, ranks, args, want_e2e=not args.no_e2e)
-            per_config[other.name] = dict(workload_index=idx,
-                                          **config_summary(other, mo, world, peak))
-            del mo
-            torch.cuda.empty_cache()
+        # One clock record over all of them (each one's timed steps are far
+        # shorter than the sampling period).
+        with ClockSampler(gpu_uuid(device)) as clocks:
+            for idx in sorted(workloads.CONFIGS):
+                other = workloads.CONFIGS[idx]
+                if other.name == wl.name:
+                    continue
+                mo = measure(other, other.n_layers, args.per_config_steps, max(3, args.warmup),
+                             device, ranks, args, want_e2e=not args.no_e2e)
+                per_config[other.name] = dict(workload_index=idx,
+                                              **config_summary(other, mo, world, peak))
+                del mo
+                torch.cuda.empty_cache()
+        per_config["clocks"] = clocks.summary()
     ranks.close()
     if rank != 0:
         return
@@ -704,8 +725,10 @@ def run_alspec(args, wl):
                    % (2 * l2_bytes >> 20, 2 * l2_bytes >> 20, m["kv_bytes"] / 1e6))
             if m["flush"] else ("inputs larger than L2: %.1f MB of KV per step against %d MB "
                                 "of L2; no flush" % (m["kv_bytes"] / 1e6, l2_bytes >> 20)),
-            "timing": "CUDA graph per step, CUDA events on the launch stream; per-kernel times "
-                      "from a second pass of graphs with per-layer events",
+            "timing": "CUDA graph per step, CUDA events on the launch stream; the middle "
+                      "kernel's duration from a second pass of graphs with event nodes around "
+                      "it (where it starts once the sink-set kernel has completed, so it runs "
+                      "alone); O_spec latency from kernel-written time stamps in a third pass",
             "schedule": {1: "streams", 2: "fused", 3: "sink_first"}[plan["schedule"]],
             "plan": plan},
         "roofline": {"bound": "hbm",
@@ -723,7 +746,8 @@ def run_alspec(args, wl):
         "spec_latency": dict(spec_summary(m),
                              profiled_graph_us_median=statistics.median(m["spec_ms"]) * 1e3,
                              profiled_graph_layer_us_median=statistics.median(m["layer_ms"]) * 1e3),
-        "layer_breakdown_us_median": {
+        "profiled_pass_us_median": {
+            "what": "graphs with event nodes between the kernels (no overlap between them)",
             "start_to_middle_kernel": statistics.median(m["pre_ms"]) * 1e3,
             "middle_kernel": statistics.median(m["mid_ms"]) * 1e3,
             "middle_end_to_layer_end": statistics.median(m["post_ms"]) * 1e3,

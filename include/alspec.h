@@ -20,8 +20,8 @@
  *   - Pointers named "device" are CUDA device pointers; "host" pointers are
  *     ordinary host memory.  The caller owns every buffer.  The library never
  *     allocates device memory in alspec_decode; it owns only a
- *     high-priority stream, a lowest-priority stream and three events per
- *     device, created on first use and released by alspec_shutdown().
+ *     lowest-priority stream and two events per device, created on first
+ *     use and released by alspec_shutdown().
  *   - Streams and events are passed as `void*` holding a cudaStream_t /
  *     cudaEvent_t (NULL stream = the legacy default stream).
  *   - Calls are asynchronous on the given stream unless stated otherwise;
@@ -68,10 +68,20 @@ typedef enum {
 
 /*
  * Launch schedule of one decode call (alspec_desc.schedule).
- *   STREAMS: the sink-set kernel on a high-priority stream forked from the
- *            caller's (O_spec early, marked by spec_event), the exact-path
- *            kernel on the caller's stream, then a merge kernel that also
- *            writes rel_l2 and the flags: three launches and a fork/join.
+ *   STREAMS: three kernels in order on the caller's stream: the sink-set
+ *            kernel (at high launch priority; O_spec early), the exact-path
+ *            kernel and a merge kernel that also writes rel_l2 and the flags.
+ *            Each launch is released as soon as every CTA of the one before
+ *            it has started, so the exact-path kernel (persistent, one CTA
+ *            per SM) runs beside the sink-set kernel on the SMs it leaves and
+ *            takes over each SM it frees.  When the caller asks for
+ *            spec_event (or the speculative projection), the library's
+ *            lowest-priority stream waits for the sink-set kernel (an event
+ *            recorded right behind it), records spec_event there (and runs
+ *            the projection), and the caller's stream joins it at the end.
+ *            Inside a CUDA graph that event record is only a dependency, so
+ *            the kernels keep their overlap; outside one, the exact-path
+ *            kernel may then start only once the sink-set kernel completed.
  *   FUSED:   one persistent launch on the caller's stream.  The sink-set
  *            work items come first in the same work queue as the exact
  *            path's; the CTA that completes a (sequence, KV head) writes its
@@ -79,10 +89,10 @@ typedef enum {
  *            writes rel_l2 and the flag (ticket counters in the workspace).
  *            O_spec is complete only when the launch ends (spec_event marks
  *            that point); alspec_decode_oproj is not available with it.
- *   SINK_FIRST: as STREAMS, but the sink-set kernel runs alone first on the
- *            caller's stream with every SM, and the exact-path kernel after
- *            it: O_spec sooner when the sink set is large (many sequences or
- *            a long window), at some cost in throughput.
+ *   SINK_FIRST: as STREAMS, but the exact-path kernel starts only once the
+ *            sink-set kernel has completed, which then has every SM: O_spec
+ *            sooner when the sink set is large (many sequences or a long
+ *            window), at some cost in throughput.
  */
 typedef enum {
     ALSPEC_SCHEDULE_AUTO = 0,     /* STREAMS */
@@ -173,17 +183,19 @@ alspec_status alspec_workspace_init(void* workspace, size_t workspace_bytes, voi
  *               cudaEventRecordExternal so that they become event nodes when
  *               the call is captured in a graph:
  *                 [0] on `stream` when the call starts,
- *                 [1] on the high-priority stream when O_spec is complete,
+ *                 [1] on `stream` after the sink-set kernel (O_spec complete),
  *                 [2] on `stream` before the exact-path (middle) kernel,
  *                 [3] on `stream` after it,
  *                 [4] on `stream` when the call's work is complete.
- *               [1]-[0] is the latency of O_spec, [3]-[2] the duration of
- *               the middle kernel, [4]-[0] the latency of the whole step.
+ *               Events between the kernels take away their overlap: with
+ *               them, the middle kernel starts once the sink-set kernel has
+ *               completed, so [3]-[2] is the middle kernel's duration alone
+ *               and [4]-[0] is longer than the step without events.
  *
- * STREAMS schedule: the sink-set attention runs on a high-priority stream
- * forked from `stream` with events; the rest runs on `stream`.  FUSED
- * schedule: one launch on `stream`; spec_event and prof_events [1]-[3] are
- * recorded around it.  Safe to capture in a CUDA graph (no host
+ * Everything runs on `stream` (and, for spec_event, on the library's
+ * lowest-priority stream, joined before the call's work is complete).
+ * FUSED schedule: one launch on `stream`; spec_event and prof_events [1]-[3]
+ * are recorded around it.  Safe to capture in a CUDA graph (no host
  * synchronization, no allocation).  With L_b <= S + W the two outputs are
  * bit-identical and rel_l2 is exactly 0.
  */
@@ -302,9 +314,11 @@ alspec_status alspec_test_wait_timeout(void* workspace, size_t workspace_bytes, 
  *     0 when the merge runs as one CTA per 32 output columns (a CTA's share
  *     of the middle partials does not fit in shared memory; and the FUSED
  *     schedule, which merges inside its one kernel)
+ *  11 CTAs of the sink-set kernel (batch * n_kv_heads * entry 1; none with
+ *     the FUSED schedule's one kernel, which queues those items)
  * (entries 4-7 describe the exact-path kernel, or with the FUSED schedule
  * the one kernel, whose queue holds both kinds of items).  n_info is the
- * capacity of info (11 fills all).
+ * capacity of info (12 fills all).
  */
 alspec_status alspec_query_plan(const alspec_desc* desc, int n_sink, int window,
                                 int* info, int n_info);

@@ -196,10 +196,10 @@ def alspec_noalloc_device_error(stream: int):
 
 
 def alspec_query_plan(desc: alspec_desc, n_sink: int, window: int):
-    info = (ctypes.c_int * 11)()
-    st = int(_lib.alspec_query_plan(ctypes.byref(desc), n_sink, window, info, 11))
+    info = (ctypes.c_int * 12)()
+    st = int(_lib.alspec_query_plan(ctypes.byref(desc), n_sink, window, info, 12))
     keys = ("c1", "n1", "c2", "n2", "grid2", "threads", "smem", "stages", "engine", "schedule",
-            "merge_c")
+            "merge_c", "grid1")
     return st, dict(zip(keys, list(info)))
 
 

@@ -65,6 +65,14 @@ constexpr int kMaxSpecItems = kMaxSpecCtas;  // sink-set CTAs per (sequence, KV 
 constexpr int kFusedSpecMinTiles = 4;
 constexpr int kFusedSpecMaxItems = kMaxSpecItemsFused;
 constexpr size_t kAlign = 256;
+// SMs the middle kernel leaves free when the caller works on O_spec beside
+// the exact path (spec_event, the speculative projection): a kernel of
+// another stream (a transfer of O_spec, the projection) found no room on an
+// SM beside a middle-kernel CTA, and with every SM holding one it ran only
+// once the exact path ended (measured).
+#ifndef ALSPEC_SIDE_SMS
+#define ALSPEC_SIDE_SMS 2
+#endif
 
 thread_local cudaError_t t_last_error = cudaSuccess;
 
@@ -93,15 +101,14 @@ int round_up(int a, int b) { return ceil_div(a, b) * b; }
 // the SM count, and which kernels already got their shared-memory attribute.
 struct DeviceState {
     bool ready = false;
-    cudaStream_t hi = nullptr;
-    cudaStream_t lo = nullptr;    // lowest priority: speculative post-attention work
-    cudaEvent_t fork = nullptr;
-    cudaEvent_t join = nullptr;
-    cudaEvent_t join2 = nullptr;  // after the speculative output projection
+    cudaStream_t lo = nullptr;    // lowest priority: work on O_spec beside the exact path
+    cudaEvent_t fork = nullptr;   // behind the sink-set kernel, for the lowest-priority stream
+    cudaEvent_t join = nullptr;   // that stream's work of the call done
     int sm_count = 0;
-    int prio_hi = 0;
+    int prio_hi = 0;              // launch priority of the sink-set kernel
     std::set<const void*> attr_done;
 };
+
 
 std::mutex g_mutex;
 DeviceState g_dev[kMaxDevices];
@@ -119,11 +126,9 @@ alspec_status get_device_state(DeviceState** out) {
         int lo = 0, hi = 0;
         if (!ok(cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev)) ||
             !ok(cudaDeviceGetStreamPriorityRange(&lo, &hi)) ||
-            !ok(cudaStreamCreateWithPriority(&d.hi, cudaStreamNonBlocking, hi)) ||
             !ok(cudaStreamCreateWithPriority(&d.lo, cudaStreamNonBlocking, lo)) ||
             !ok(cudaEventCreateWithFlags(&d.fork, cudaEventDisableTiming)) ||
-            !ok(cudaEventCreateWithFlags(&d.join, cudaEventDisableTiming)) ||
-            !ok(cudaEventCreateWithFlags(&d.join2, cudaEventDisableTiming))) {
+            !ok(cudaEventCreateWithFlags(&d.join, cudaEventDisableTiming))) {
             return ALSPEC_ERR_CUDA;
         }
         d.prio_hi = hi;
@@ -308,6 +313,7 @@ void make_plan(const alspec_desc& d, int S, int W, int sms, Plan* pl) {
     }
     const long long items2 = (long long)heads * (pl->n2 + (fused ? pl->n1 : 0));
     pl->grid2 = (int)std::min<long long>(P, items2);
+
     const int G = d.n_q_heads / d.n_kv_heads;
     kernel_shape(d.dtype, d.head_dim, G, pl->engine, fused, &pl->threads, &pl->smem, &pl->stages);
 
@@ -506,9 +512,9 @@ alspec_status alspec_query_plan(const alspec_desc* desc, int n_sink, int window,
     if (!info || n_info < 0) return ALSPEC_ERR_INVALID_ARG;
     Plan pl{};
     make_plan(*desc, n_sink, window, sm_count_for_plan(), &pl);
-    const int vals[11] = {pl.c1,      pl.n1,   pl.c2,     pl.n2,     pl.grid2,   pl.threads,
-                          pl.smem,    pl.stages, pl.engine, pl.schedule, pl.merge_c};
-    for (int i = 0; i < n_info && i < 11; ++i) info[i] = vals[i];
+    const int vals[12] = {pl.c1,   pl.n1,     pl.c2,     pl.n2,       pl.grid2,   pl.threads,
+                          pl.smem, pl.stages, pl.engine, pl.schedule, pl.merge_c, pl.grid1};
+    for (int i = 0; i < n_info && i < 12; ++i) info[i] = vals[i];
     return ALSPEC_OK;
 }
 
@@ -637,6 +643,7 @@ alspec_status decode_impl(const alspec_desc* desc, const void* q, const void* k_
     p.c1 = pl.c1;
     p.n1 = pl.n1;
     p.n2 = pl.n2;
+    p.mid_ctas = pl.grid2;
     std::memcpy(p.fq, pl.fq, sizeof p.fq);
     p.ctr = reinterpret_cast<unsigned*>(ws + pl.off_ctr);
     p.spec_ml = reinterpret_cast<float*>(ws + pl.off_spec_ml);
@@ -678,44 +685,58 @@ alspec_status decode_impl(const alspec_desc* desc, const void* q, const void* k_
             return ALSPEC_ERR_CUDA;
         return prof(4, s) ? ALSPEC_OK : ALSPEC_ERR_CUDA;
     }
-    // Fork: the sink-set kernel runs on the high-priority stream, beside the
-    // middle kernel -- or (SINK_FIRST) alone first on the caller's stream,
-    // the middle kernel following it there.
-    cudaStream_t ss = pl.sink_first ? s : ds->hi;
-    if (!pl.sink_first &&
-        (!ok(cudaEventRecord(ds->fork, s)) || !ok(cudaStreamWaitEvent(ds->hi, ds->fork, 0))))
-        return ALSPEC_ERR_CUDA;
-    const dim3 grid1(pl.grid1);
-    if ((st = launch(ks.spec, grid1, dim3(ks.threads_spec), ks.smem_spec, ss, p,
-                     pl.sink_first ? 0 : kLaunchHighPriority, ds->prio_hi, pl.n1)) != ALSPEC_OK)
-        return st;
-    if (spec_event && !ok(record_event(static_cast<cudaEvent_t>(spec_event), ss)))
-        return ALSPEC_ERR_CUDA;
-    if (!prof(1, ss)) return ALSPEC_ERR_CUDA;
-    if (!ok(cudaEventRecord(ds->join, ss))) return ALSPEC_ERR_CUDA;
+    // The three kernels run in order on the caller's stream.  The sink-set
+    // kernel goes first, at high launch priority; each of its CTAs lets the
+    // middle kernel launch as soon as it starts, so the middle kernel is
+    // released once every sink-set CTA (and thread-block cluster) is
+    // resident: its persistent CTAs take the SMs left over at once and each
+    // SM a sink-set CTA frees -- the sink set always finds its SMs, and
+    // nothing waits for it to complete.  (SINK_FIRST: the middle kernel
+    // starts after it completes.)  The merge kernel follows the middle one
+    // the same way.
+    //
+    // Work on O_spec elsewhere (spec_event, the speculative projection) runs
+    // on the library's lowest-priority stream, after an event recorded
+    // right behind the sink-set kernel: under stream capture that record is
+    // not a node, only the sink-set kernel's dependency handed to the other
+    // stream, so the programmatic edge to the middle kernel stays.  The
+    // caller's stream joins that stream at the end of the call.
+    const bool side = spec_event != nullptr || op != nullptr;
     const int kdim = desc->n_q_heads * desc->head_dim;
-    if (op) {
-        // Speculative output projection of O_spec, beside the exact path, on
-        // the lowest-priority stream: it has until the merge to finish, and
-        // the middle kernel's CTAs come first.
-        const OprojParams o = oproj_params(out_spec, op->w, op->y, nullptr, desc->batch, kdim,
-                                           op->hidden, trace_ns ? trace_ns + 2 : nullptr,
-                                           p.ctr + kCtrError, p.timeout_ns);
-        if (!ok(cudaStreamWaitEvent(ds->lo, ds->join, 0))) return ALSPEC_ERR_CUDA;
-        oproj_kernel_for(o.B)<<<oproj_grid(op->hidden), kOprojWarps * 32, 0, ds->lo>>>(o);
-        if (!ok(cudaGetLastError()) || !ok(cudaEventRecord(ds->join2, ds->lo)))
+    const dim3 grid1(pl.grid1);
+    if ((st = launch(ks.spec, grid1, dim3(ks.threads_spec), ks.smem_spec, s, p,
+                     kLaunchHighPriority, ds->prio_hi, pl.n1)) != ALSPEC_OK)
+        return st;
+    if (side) {
+        cudaStream_t lo = ds->lo;
+        if (!ok(cudaEventRecord(ds->fork, s)) || !ok(cudaStreamWaitEvent(lo, ds->fork, 0)))
             return ALSPEC_ERR_CUDA;
+        if (spec_event && !ok(record_event(static_cast<cudaEvent_t>(spec_event), lo)))
+            return ALSPEC_ERR_CUDA;
+        if (op) {
+            // Speculative output projection of O_spec, beside the exact
+            // path: a kernel without shared memory, so it fits beside the
+            // middle kernel's CTAs, whose work comes first.
+            const OprojParams o = oproj_params(out_spec, op->w, op->y, nullptr, desc->batch, kdim,
+                                               op->hidden, trace_ns ? trace_ns + 2 : nullptr,
+                                               p.ctr + kCtrError, p.timeout_ns);
+            oproj_kernel_for(o.B)<<<oproj_grid(op->hidden), kOprojWarps * 32, 0, lo>>>(o);
+            if (!ok(cudaGetLastError())) return ALSPEC_ERR_CUDA;
+        }
+        if (!ok(cudaEventRecord(ds->join, lo))) return ALSPEC_ERR_CUDA;
     }
-    // The middle of every sequence on the caller's stream.
-    if (!prof(2, s)) return ALSPEC_ERR_CUDA;
+    // Profiling events between the kernels take away their overlap: the
+    // middle kernel then starts once the sink set has completed.
+    if (!prof(1, s) || !prof(2, s)) return ALSPEC_ERR_CUDA;
     if (pl.n2 > 0) {
-        if ((st = launch(ks.mid, dim3(pl.grid2), dim3(ks.threads_mid), ks.smem_mid, s, p, 0, 0)) !=
-            ALSPEC_OK)
+        const int flags = pl.sink_first || prof_events ? 0 : kLaunchProgrammatic;
+        Params pm = p;
+        if (side && pl.grid2 > ALSPEC_SIDE_SMS) pm.mid_ctas = pl.grid2 - ALSPEC_SIDE_SMS;
+        if ((st = launch(ks.mid, dim3(pm.mid_ctas), dim3(ks.threads_mid), ks.smem_mid, s, pm,
+                         flags, 0)) != ALSPEC_OK)
             return st;
     }
     if (!prof(3, s)) return ALSPEC_ERR_CUDA;
-    // Join, then merge + relative L2 + flag.
-    if (!ok(cudaStreamWaitEvent(s, ds->join, 0))) return ALSPEC_ERR_CUDA;
     KernelFn mk = nullptr;
     if (pl.merge_c > 0) {
         if (desc->head_dim == 128)
@@ -745,9 +766,9 @@ alspec_status decode_impl(const alspec_desc* desc, const void* q, const void* k_
             !ok(cudaGraphConditionalHandleCreate(&cond, cg, 0, cudaGraphCondAssignDefault)))
             return ALSPEC_ERR_CUDA;
     }
-    // Programmatic launch right behind the middle kernel (when there is one
-    // and no profiling event sits between them).
-    const bool pdl = pl.n2 > 0 && !prof_events;
+    // Programmatic launch right behind the middle kernel (or the sink-set
+    // kernel, with no middle), unless a profiling event sits between them.
+    const bool pdl = !prof_events;
     if (pl.merge_c > 0) {
         if ((st = launch(mk, dim3(pl.merge_c, desc->batch), dim3(kCmThreads), pl.merge_smem, s, p,
                          pdl ? kLaunchProgrammatic : 0, 0, pl.merge_c)) != ALSPEC_OK)
@@ -757,10 +778,11 @@ alspec_status decode_impl(const alspec_desc* desc, const void* q, const void* k_
                ALSPEC_OK) {
         return st;
     }
+    // The side stream's work on O_spec belongs to this call.
+    if (side && !ok(cudaStreamWaitEvent(s, ds->join, 0))) return ALSPEC_ERR_CUDA;
     if (op) {
         // Redo the projection on O_exact for the discarded tokens, after the
         // speculative one (both write y).
-        if (!ok(cudaStreamWaitEvent(s, ds->join2, 0))) return ALSPEC_ERR_CUDA;
         OprojParams r = oproj_params(out_exact, op->w, op->y, commit, desc->batch, kdim,
                                      op->hidden, trace_ns ? trace_ns + 2 : nullptr,
                                      p.ctr + kCtrError, p.timeout_ns);
@@ -940,12 +962,9 @@ alspec_status alspec_shutdown(void) {
             st = ALSPEC_ERR_CUDA;
             continue;
         }
-        if (cudaStreamSynchronize(s.hi) != cudaSuccess) st = ALSPEC_ERR_CUDA;
         if (s.lo && cudaStreamSynchronize(s.lo) != cudaSuccess) st = ALSPEC_ERR_CUDA;
         cudaEventDestroy(s.fork);
         cudaEventDestroy(s.join);
-        if (s.join2) cudaEventDestroy(s.join2);
-        cudaStreamDestroy(s.hi);
         if (s.lo) cudaStreamDestroy(s.lo);
         s = DeviceState{};
     }
@@ -966,7 +985,7 @@ const char* alspec_status_string(alspec_status status) {
     }
 }
 
-int alspec_version(void) { return 300; }
+int alspec_version(void) { return 301; }
 
 int alspec_last_cuda_error(void) { return (int)t_last_error; }
 

@@ -28,10 +28,11 @@
 //
 // Inside a CTA one producer lane fills a ring of shared-memory stages with
 // K and V tiles through the TMA engine (mbarrier completion); consumer warps
-// compute.  Each stage belongs to one consumer warp ("token slot"), so a
-// warp visits its stages in order and every item is padded to a multiple
-// of the slot count.  At the end of an item the warps' states are merged
-// through shared memory and one partial per query head is written.
+// compute.  Tile t of a CTA goes to consumer warp t mod (warps) ("token
+// slot") and every item is padded to a multiple of the slot count; each
+// stage carries a fill ticket naming the tile it holds.  At the end of an
+// item the warps' states are merged through shared memory and one partial
+// per query head is written.
 //
 // Two compute engines share that pipeline:
 //   * tensor cores (bf16 caches): 32-token tiles loaded as 2-D TMA boxes
@@ -71,10 +72,14 @@ constexpr int kMaxSpecCtas = 8;
 #define ALSPEC_SPEC_WARPS 5
 #endif
 
-// Stages per token slot of the tensor-core middle kernel: 3 stages of 16 KB
-// per consumer warp keep up to 192 KB in flight per SM (a warp holds one of
-// its stages for the ~0.8 us its tile's math takes), so the producer keeps
-// streaming through the few microseconds an item's end takes.
+// Stages of the tensor-core middle kernel's ring: 12 stages of 16 KB keep
+// up to 192 KB in flight per SM, so the producer keeps streaming through the
+// few microseconds an item's end takes.  A 13th stage fits beside the
+// item-end deposit (the stages' fill tickets keep any count sound, see
+// Cfg::STAGES) but measured no faster on the 128K step.
+#ifndef ALSPEC_MID_STAGES
+#define ALSPEC_MID_STAGES 12
+#endif
 #ifndef ALSPEC_MID_SPW
 #define ALSPEC_MID_SPW 3
 #endif
@@ -131,6 +136,7 @@ struct Params {
     int c1, n1;     // sink-set items: tokens per item, items per (b, kv head) (the
                     // sink-set kernel: CTAs of one cluster)
     int n2;         // middle chunks per (b, kv head)
+    int mid_ctas;   // CTAs of the middle (or one-launch) kernel's launches together
     unsigned fq[kMaxChunks + 1];  // chunk c covers middle tiles
                                   // [mt * fq[c] >> 24, mt * fq[c+1] >> 24)
     unsigned* ctr;
@@ -177,14 +183,19 @@ __host__ __device__ __forceinline__ SeqGeom geom_of(int L, int S, int W) {
     return g;
 }
 
-// Reads seq_lens[b]; out-of-range lengths are clamped (and flagged).
-__device__ __forceinline__ SeqGeom seq_geom(const Params& p, int b, bool flag) {
-    int L = __ldg(p.seq_lens + b);
+// Geometry of a sequence of stored length L; out-of-range lengths are
+// clamped (and flagged).
+__device__ __forceinline__ SeqGeom seq_geom_of_len(const Params& p, int L, bool flag) {
     if (L < 1 || L > p.Lmax) {
         if (flag) atomicOr(p.ctr + kCtrError, kErrSeqLen);
         L = L < 1 ? 1 : p.Lmax;
     }
     return geom_of(L, p.S, p.W);
+}
+
+// Reads seq_lens[b].
+__device__ __forceinline__ SeqGeom seq_geom(const Params& p, int b, bool flag) {
+    return seq_geom_of_len(p, __ldg(p.seq_lens + b), flag);
 }
 
 // Tiles of the sink-set list: the sink run and the window run are tiled
@@ -223,14 +234,23 @@ __device__ __forceinline__ void item_index(const Params& p, int item, bool& spec
     chunk = spec ? item % p.n1 : item / heads;
 }
 
+// `lane_len`: with a full warp calling, lane i may hold seq_lens[i] already
+// (loaded beforehand, for i < min(B, 32)); -1 to read the length here.
 template <bool SPEC, int TT, bool FUSED = false>
-__device__ __forceinline__ Item decode_item(const Params& p, int item, bool flag) {
+__device__ __forceinline__ Item decode_item(const Params& p, int item, bool flag,
+                                            int lane_len = -1) {
     Item it;
     int bh;
     item_index<SPEC, FUSED>(p, item, it.spec, bh, it.chunk);
     it.b = bh / p.Hkv;
     it.kvh = bh % p.Hkv;
-    const SeqGeom g = seq_geom(p, it.b, flag);
+    int L;
+    if (lane_len >= 0 && it.b < 32) {
+        L = __shfl_sync(0xffffffffu, lane_len, it.b);  // the warp agrees on it.b
+    } else {
+        L = __ldg(p.seq_lens + it.b);
+    }
+    const SeqGeom g = seq_geom_of_len(p, L, flag);
     it.ns = g.ns;
     it.ws = g.ws;
     it.L = g.L;
@@ -341,24 +361,34 @@ struct Cfg {
     static constexpr int kScratchFloats = kMaxChunks * (G + 1) + 2 * G + 4 + kMaxChunks + 4;
     static constexpr int kScratchBytes = FUSED ? kScratchFloats * 4 : 0;
 
-    static constexpr int kSpwBudget =
+    // Tile t goes to stage t mod STAGES and to consumer warp t mod NTW.  A
+    // phase-parity wait alone is only sound if no waiter can be a ring lap
+    // ahead of the stage's previous fill; when STAGES is not a multiple of
+    // NTW, consecutive fills of a stage belong to different warps and a fast
+    // warp could pass the parity test on the previous fill's phase.  So
+    // every stage carries a fill ticket: the producer stores the tile's
+    // global index (release) before filling it, and a consumer first waits
+    // for its own index (acquire), which proves the previous fill's phase
+    // completed, then tests the parity.  The tensor-core middle kernel takes
+    // as many stages as fit (ALSPEC_MID_STAGES at most); the other kernels
+    // keep whole rounds of NTW stages.
+    static constexpr bool kFreeRing = MMA && !SPEC && !FUSED;
+    static constexpr int kStagesBudget =
         (kSmemLimit - 1024 - kDepositBytes - 4096 - 768 - kGatherBytes - kScratchBytes) /
-        (NTW * kStageBytes);
-    static constexpr int SPW = kSpwBudget < 1 ? 1 : (kSpwBudget > kSpwMax ? kSpwMax : kSpwBudget);
-    // Tile t goes to stage t mod STAGES and to consumer warp t mod NTW, so
-    // with STAGES a multiple of NTW every stage has one consumer warp, which
-    // waits for its stage's fills in order.  That is what makes the
-    // phase-parity waits sound: a waiter is never a ring lap ahead of the
-    // stage's previous fill (with a stage shared by several warps, a fast
-    // warp could pass the parity test on the previous fill's phase).
-    static constexpr int STAGES = NTW * SPW;
+        kStageBytes;
+    static constexpr int kStagesCap = kFreeRing ? ALSPEC_MID_STAGES : NTW * kSpwMax;
+    static constexpr int kStagesFit = kStagesBudget < kStagesCap ? kStagesBudget : kStagesCap;
+    static constexpr int kRounds = kStagesFit / NTW < 1 ? 1 : kStagesFit / NTW;
+    static constexpr int STAGES =
+        kFreeRing ? (kStagesFit < NTW ? NTW : kStagesFit) : NTW * kRounds;
     // Dynamic shared memory layout (offsets from a 1024-byte aligned base;
     // every region starts on a 128-byte boundary: the stage metadata are
     // int4, the barriers 8-byte words).
     static constexpr int align128(int x) { return (x + 127) / 128 * 128; }
     static constexpr int kOffDeposit = STAGES * kStageBytes;
     static constexpr int kOffMeta = align128(kOffDeposit + kDepositBytes);
-    static constexpr int kOffBar = align128(kOffMeta + STAGES * 16);
+    static constexpr int kOffFill = align128(kOffMeta + STAGES * 16);
+    static constexpr int kOffBar = align128(kOffFill + STAGES * 4);
     static constexpr int kNumBars = 2 * STAGES + 4;
     static constexpr int kOffMisc = align128(kOffBar + kNumBars * 8);
     static constexpr int kOffGather = align128(kOffMisc + 16);
@@ -375,7 +405,8 @@ struct Cfg {
     static_assert(!MMA || (sizeof(T) == 2 && G <= 8), "tensor-core engine: bf16, g <= 8");
     static_assert(kSmemBytes <= kSmemLimit, "shared memory budget");
     static_assert(NTW >= 1 && NCW <= 8, "warp split");
-    static_assert(STAGES % NTW == 0, "each stage must belong to one consumer warp");
+    static_assert(STAGES >= NTW, "every consumer warp needs a stage");
+    static_assert(kFreeRing || STAGES % NTW == 0, "whole rounds of stages");
     static_assert(!(SPEC && FUSED), "the one-launch kernel is a middle-kernel variant");
 };
 
@@ -412,6 +443,34 @@ __device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, volati
     uint64_t t0 = 0;
     for (uint32_t it = 0;; ++it) {
         const bool ok = mbar_try_wait(bar, parity);
+        if (__all_sync(0xffffffffu, ok)) return true;
+        if ((it & 31) == 31) {
+            int stop = 0;
+            if (lane == 0) {
+                const uint64_t now = global_ns();
+                if (t0 == 0) {
+                    t0 = now;
+                } else if (now - t0 > p.timeout_ns) {
+                    *abort = 1;
+                    atomicOr(p.ctr + kCtrError, kErrTimeout);
+                }
+                stop = *abort;
+            }
+            if (__shfl_sync(0xffffffffu, stop, 0)) return false;
+        }
+    }
+}
+
+// Consumer-side bounded wait for the fill with global tile index `gt` of a
+// stage: first the stage's fill ticket must name that tile (which proves
+// the stage's previous fill completed its phase), then the phase with
+// `parity` must complete.  Every lane probes; the warp leaves together.
+__device__ __forceinline__ bool wait_fill(uint64_t* bar, const uint32_t* ticket, uint32_t gt,
+                                          uint32_t parity, volatile int* abort, const Params& p,
+                                          int lane) {
+    uint64_t t0 = 0;
+    for (uint32_t it = 0;; ++it) {
+        const bool ok = ld_acquire_shared(ticket) == gt && mbar_try_wait(bar, parity);
         if (__all_sync(0xffffffffu, ok)) return true;
         if ((it & 31) == 31) {
             int stop = 0;
@@ -981,13 +1040,14 @@ __device__ __forceinline__ void write_flag(const Params& p, int b, int lane) {
 // the expected bytes, the K and V copies).  Any lane may fill any stage.
 template <typename T, int D, int G, bool SPEC, bool MMA, bool FUSED>
 __device__ __forceinline__ void fill_stage(const Params& p, unsigned char* smem, int4* meta,
-                                           uint64_t* full_bar, int s, int item, const Item& it,
-                                           int t, int ntiles) {
+                                           uint32_t* fill, uint64_t* full_bar, int s, uint32_t gt,
+                                           int item, const Item& it, int t, int ntiles) {
     using C = Cfg<T, D, G, SPEC, MMA, FUSED>;
     constexpr int TT = C::TT;
     const int head_row = (it.b * p.Hkv + it.kvh) * p.Lmax;
     int start = 0, nvalid = 0;
     if (t < it.ntiles) tile_rows<SPEC, TT, FUSED>(it, t, start, nvalid);
+    st_release_shared(fill + s, gt);  // this fill is the one for tile gt
     meta[s] = make_int4(item, t, nvalid,
                         (FUSED ? it.ntiles << 1 : 0) | (t >= ntiles - C::NTW ? kLastTileFlag : 0));
     if (nvalid == 0) {
@@ -1022,7 +1082,7 @@ __device__ __forceinline__ void fill_stage(const Params& p, unsigned char* smem,
 // with the rest, waiting for each stage to be released.
 template <typename T, int D, int G, bool SPEC, bool MMA, bool FUSED>
 __device__ __forceinline__ void produce(const Params& p, unsigned char* smem, int4* meta,
-                                        uint64_t* full_bar, uint64_t* empty_bar,
+                                        uint32_t* fill, uint64_t* full_bar, uint64_t* empty_bar,
                                         volatile int* abort, int lane, int item0,
                                         const Item& it0) {
     using C = Cfg<T, D, G, SPEC, MMA, FUSED>;
@@ -1031,8 +1091,8 @@ __device__ __forceinline__ void produce(const Params& p, unsigned char* smem, in
     const bool have0 = item0 < n_items && it0.ntiles > 0;
     const int fresh = have0 ? min(rounded(it0), C::STAGES) : 0;
     for (int t = lane; t < fresh; t += 32)
-        fill_stage<T, D, G, SPEC, MMA, FUSED>(p, smem, meta, full_bar, t, item0, it0, t,
-                                              rounded(it0));
+        fill_stage<T, D, G, SPEC, MMA, FUSED>(p, smem, meta, fill, full_bar, t, (uint32_t)t, item0,
+                                              it0, t, rounded(it0));
     if (lane != 0) return;
 
     uint32_t gt = (uint32_t)fresh;
@@ -1046,7 +1106,8 @@ __device__ __forceinline__ void produce(const Params& p, unsigned char* smem, in
                 ok = false;
                 return;
             }
-            fill_stage<T, D, G, SPEC, MMA, FUSED>(p, smem, meta, full_bar, s, item, it, t, ntiles);
+            fill_stage<T, D, G, SPEC, MMA, FUSED>(p, smem, meta, fill, full_bar, s, gt, item, it, t,
+                                                  ntiles);
         }
     };
     if (have0) run(item0, it0, fresh);
@@ -1066,6 +1127,7 @@ __device__ __forceinline__ void produce(const Params& p, unsigned char* smem, in
                 ok = false;
                 break;
             }
+            st_release_shared(fill + s, gt);
             meta[s] = make_int4(-1, 0, 0, 0);
             mbar_arrive(full_bar + s);
         }
@@ -1083,9 +1145,10 @@ __device__ __forceinline__ void produce(const Params& p, unsigned char* smem, in
         }
     }
     if (!SPEC) {
-        // The CTA that stops last resets the queue for the next call.
+        // The CTA that stops last (of every launch sharing the queue)
+        // resets the queue for the next call.
         const unsigned t = atomicAdd(p.ctr + kCtrDone, 1u);
-        if (t == gridDim.x - 1) {
+        if (t == (unsigned)p.mid_ctas - 1) {
             atomicExch(p.ctr + kCtrQueue, 0u);
             atomicExch(p.ctr + kCtrDone, 0u);
         }
@@ -1427,7 +1490,7 @@ __device__ __forceinline__ bool fused_head_merge(const Params& p, int bh, float*
 // share of it).
 template <typename T, int D, int G, bool SPEC, bool MMA, bool FUSED>
 __device__ __forceinline__ void consume(const Params& p, unsigned char* smem, float* deposit,
-                                        int4* meta, uint64_t* full_bar,
+                                        int4* meta, const uint32_t* fill, uint64_t* full_bar,
                                         uint64_t* empty_bar, uint64_t* dep_bar, uint64_t* free_bar,
                                         uint64_t* merge_bar, volatile int* abort, Shared* sh,
                                         float* scratch) {
@@ -1501,7 +1564,7 @@ __device__ __forceinline__ void consume(const Params& p, unsigned char* smem, fl
     }
     for (;; gt += C::NTW) {
         const int s = gt % C::STAGES;
-        if (!wait_warp(full_bar + s, (gt / C::STAGES) & 1, abort, p, lane)) break;
+        if (!wait_fill(full_bar + s, fill + s, gt, (gt / C::STAGES) & 1, abort, p, lane)) break;
         const int4 mt = meta[s];
         if (mt.x < 0) break;
         if (!SPEC && mt.y < C::NTW) {
@@ -1613,6 +1676,7 @@ __global__ void __launch_bounds__(Cfg<T, D, G, SPEC, MMA, FUSED>::kThreads, 1)
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float* deposit = reinterpret_cast<float*>(smem + C::kOffDeposit);
     int4* meta = reinterpret_cast<int4*>(smem + C::kOffMeta);
+    uint32_t* fill = reinterpret_cast<uint32_t*>(smem + C::kOffFill);
     uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
     uint64_t* empty_bar = full_bar + C::STAGES;
     uint64_t* dep_bar = empty_bar + C::STAGES;  // consumer warps: phase sync
@@ -1633,6 +1697,7 @@ __global__ void __launch_bounds__(Cfg<T, D, G, SPEC, MMA, FUSED>::kThreads, 1)
         for (int s = 0; s < C::STAGES; ++s) {
             mbar_init(full_bar + s, 1);
             mbar_init(empty_bar + s, C::NHW);
+            fill[s] = 0xffffffffu;  // no tile yet
         }
         mbar_init(dep_bar, C::NCW);
         mbar_init(free_bar, C::NCW);
@@ -1655,6 +1720,9 @@ __global__ void __launch_bounds__(Cfg<T, D, G, SPEC, MMA, FUSED>::kThreads, 1)
             prefetch_tmap(&p.tmap_k);
             prefetch_tmap(&p.tmap_v);
         }
+        // The sequence lengths travel while the queue ticket does (the
+        // item's sequence is known only once the ticket is back).
+        const int lane_len = lane < p.B ? __ldg(p.seq_lens + lane) : 0;
         if (SPEC) {
             item0 = (int)blockIdx.x;
         } else {
@@ -1662,24 +1730,29 @@ __global__ void __launch_bounds__(Cfg<T, D, G, SPEC, MMA, FUSED>::kThreads, 1)
             if (lane == 0) v = atomicAdd(p.ctr + kCtrQueue, 1u);
             item0 = (int)__shfl_sync(0xffffffffu, v, 0);
         }
-        if (item0 < n_items) it0 = decode_item<SPEC, C::TT, FUSED>(p, item0, lane == 0);
+        if (item0 < n_items)
+            it0 = decode_item<SPEC, C::TT, FUSED>(p, item0, lane == 0, max(lane_len, 0));
     }
-    // The merge kernel that follows this (middle) kernel may be resident
-    // already: it only prepares until this grid has completed.
-    if (!SPEC && !FUSED) pdl_launch_dependents();
+    // The kernel that follows this one on its stream may be launched now
+    // (when it was launched for that): after the middle kernel the merge
+    // kernel, which only prepares until this grid has completed; after the
+    // sink-set kernel the middle kernel's second launch, whose CTAs then
+    // take each SM a sink-set CTA leaves (every sink-set CTA is resident by
+    // the time all of them have passed this point).
+    if (!FUSED) pdl_launch_dependents();
     __syncthreads();
     if (clustered) cluster_arrive_relaxed();  // this CTA's barriers are set up
 
     if (warp == C::NCW) {
         // ---------------------------------------------------- producer
-        produce<T, D, G, SPEC, MMA, FUSED>(p, smem, meta, full_bar, empty_bar, abort, lane, item0,
-                                           it0);
+        produce<T, D, G, SPEC, MMA, FUSED>(p, smem, meta, fill, full_bar, empty_bar, abort, lane,
+                                           item0, it0);
         if (!clustered) return;
         cluster_wait_any();  // the cluster's barriers are set up
         __syncwarp();  // the warp waits for its producer lane, then joins the cluster merge
     } else {
-        consume<T, D, G, SPEC, MMA, FUSED>(p, smem, deposit, meta, full_bar, empty_bar, dep_bar,
-                                           free_bar, merge_bar, abort, sh, scratch);
+        consume<T, D, G, SPEC, MMA, FUSED>(p, smem, deposit, meta, fill, full_bar, empty_bar,
+                                           dep_bar, free_bar, merge_bar, abort, sh, scratch);
     }
     if (SPEC && !clustered && warp < C::NCW && p.trace) {
         // One CTA per head: its consumer warps wrote O_spec.
@@ -1691,6 +1764,10 @@ __global__ void __launch_bounds__(Cfg<T, D, G, SPEC, MMA, FUSED>::kThreads, 1)
         __syncthreads();
         cluster_gather<D, G, C>(p, deposit, gather, gather_bar);
     }
+    // The middle kernel, launched behind the sink-set kernel before it has
+    // completed, does not complete before it: what follows on the stream
+    // (the merge) may read the sink set's results.  (No-op otherwise.)
+    if (!SPEC && !FUSED && threadIdx.x == 0) pdl_wait_prerequisite();
 }
 
 // ------------------------------------------------------- merge + verify

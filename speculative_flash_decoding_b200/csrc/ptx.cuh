@@ -227,6 +227,19 @@ __device__ __forceinline__ unsigned atom_add_acq_rel_gpu(unsigned* addr, unsigne
     return old;
 }
 
+// Shared-memory word with release / acquire semantics at CTA scope: a
+// thread that reads (acquire) the value another thread stored (release)
+// also sees everything that thread had observed before the store.
+__device__ __forceinline__ void st_release_shared(uint32_t* p, uint32_t v) {
+    asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" ::"r"(smem_addr(p)), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_shared(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_addr(p)) : "memory");
+    return v;
+}
+
 __device__ __forceinline__ uint64_t global_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

@@ -23,11 +23,11 @@ int main(void) {
     printf("version %d\n", alspec_version());
     for (int sch = ALSPEC_SCHEDULE_AUTO; sch <= ALSPEC_SCHEDULE_SINK_FIRST; ++sch) {
         d.schedule = sch;
-        int info[11];
-        const alspec_status st = alspec_query_plan(&d, 4, 1024, info, 11);
+        int info[12];
+        const alspec_status st = alspec_query_plan(&d, 4, 1024, info, 12);
         printf("schedule %d status %d workspace %zu plan", sch, (int)st,
                alspec_workspace_size(&d, 4, 1024));
-        for (int i = 0; i < 11; ++i) printf(" %d", info[i]);
+        for (int i = 0; i < 12; ++i) printf(" %d", info[i]);
         printf("\n");
     }
     int scratch[11];

@@ -50,7 +50,7 @@ def test_decode_library_has_no_benchmark_probe():
 
 
 def test_version_and_status_strings():
-    assert sfd.alspec_version() == 300
+    assert sfd.alspec_version() == 301
     for st in range(7):
         assert sfd.alspec_status_string(st) and "unknown" not in sfd.alspec_status_string(st)
     assert "unknown" in sfd.alspec_status_string(99)

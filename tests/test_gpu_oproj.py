@@ -24,7 +24,10 @@ def _bf16_weights(n, k, seed, device):
     return w.to(device)
 
 
-@pytest.mark.parametrize("B,K,N", [(1, 4096, 4096), (3, 520, 77), (8, 1024, 300), (2, 8, 5)])
+# K = 8192 (Llama-70B-shaped, 64 heads x 128) and 12296 give rows of several
+# bulk-copy pieces, so consecutive fills of a stage go to different warps.
+@pytest.mark.parametrize("B,K,N", [(1, 4096, 4096), (3, 520, 77), (8, 1024, 300), (2, 8, 5),
+                                   (4, 8192, 8192), (2, 12296, 1000)])
 def test_oproj_matches_oracle(cuda_device, B, K, N):
     import speculative_flash_decoding_b200 as sfd
     g = torch.Generator(device="cpu").manual_seed(B * 1000 + K + N)

@@ -204,3 +204,26 @@ def test_query_chunks_rejects_small_buffer():
     st = ab._lib.alspec_query_chunks(ctypes.byref(desc), 4, 1024, fq, 2, ctypes.byref(n2),
                                      ctypes.byref(tile))
     assert st == ab.ALSPEC_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("shape", [(1, 32, 8, 128, 131072, 4, 1024), (1, 32, 8, 128, 32768, 4, 1024),
+                                   (8, 32, 8, 128, 65536, 4, 2048), (4, 64, 8, 128, 131072, 4, 4096),
+                                   (1, 4, 1, 64, 1024, 4, 128), (64, 32, 8, 128, 4096, 4, 64)])
+def test_sink_set_ctas_and_middle_grid(shape):
+    """The sink-set kernel has n1 CTAs (one cluster) per (sequence, KV head),
+    together within 3/4 of the SMs unless one per head already exceeds it
+    (all SMs with SINK_FIRST); the persistent middle kernel takes every SM
+    (148 without a GPU), or one CTA per item when there are fewer."""
+    import speculative_flash_decoding_b200 as sfd
+    B, Hq, Hkv, d, L, S, W = shape
+    sms = 148
+    for sched in ("streams", "sink_first"):
+        desc = sfd.make_desc(B, Hq, Hkv, d, L, "bf16", schedule=sched)
+        st, plan = sfd.alspec_query_plan(desc, S, W)
+        assert st == 0
+        heads = B * Hkv
+        assert plan["grid1"] == heads * plan["n1"]
+        share = sms if sched == "sink_first" else sms * 3 // 4
+        assert plan["n1"] == 1 or plan["grid1"] <= share
+        if plan["n2"]:
+            assert plan["grid2"] == min(sms, heads * plan["n2"])
