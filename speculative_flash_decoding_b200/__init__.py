@@ -2,9 +2,10 @@
 
 For every decode query the library computes, in CUDA kernels for sm_100a,
 the attention-sink approximation O_spec (softmax attention over the first S
-and last W cached tokens, published early on a high-priority stream), the
-exact attention O_exact over the whole cache (split-K flash decoding), the
-per-token relative L2 error of O_spec and the commit/discard flag.
+and last W cached tokens, published early by a kernel launched first at high
+priority, with the exact path running beside it), the exact attention
+O_exact over the whole cache (split-K flash decoding), the per-token
+relative L2 error of O_spec and the commit/discard flag.
 
 The C ABI is include/alspec.h (libalspec.so); ``alspec`` is its ctypes
 binding.  Importing the package raises if libalspec.so is missing.

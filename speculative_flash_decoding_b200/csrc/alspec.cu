@@ -1,7 +1,8 @@
 // Host side of libalspec.so: argument checks, work planning, workspace
-// layout, the launch schedules (the sink-set kernel forked onto a
-// high-priority stream, or first on the caller's stream, or one fused
-// launch), kernel launches and the C ABI declared in include/alspec.h.
+// layout, the launch schedules (the sink-set, middle and merge kernels
+// chained on the caller's stream with programmatic launches, the middle
+// kernel beside the sink set or after it, or one fused launch), kernel
+// launches and the C ABI declared in include/alspec.h.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
@@ -97,7 +98,7 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 int ceil_div(int a, int b) { return (a + b - 1) / b; }
 int round_up(int a, int b) { return ceil_div(a, b) * b; }
 
-// Per-device library state: the high-priority stream, the fork/join events,
+// Per-device library state: the lowest-priority stream, the fork/join events,
 // the SM count, and which kernels already got their shared-memory attribute.
 struct DeviceState {
     bool ready = false;

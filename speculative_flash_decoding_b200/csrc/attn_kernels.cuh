@@ -1603,6 +1603,9 @@ __device__ __forceinline__ void consume(const Params& p, unsigned char* smem, fl
             float* part_ml = sp ? p.spec_pml : p.mid_ml;
             float* part_o = sp ? p.spec_po : p.mid_o;
             const int per = SPEC || sp ? p.n1 : p.n2;
+            // Partials are read back by the merge after the whole stream of
+            // cache rows has gone through L2: keep them ahead of those.
+            const uint64_t keep = l2_evict_last_policy();
             for (int idx = ctid; idx < G * D; idx += C::NCW * 32) {
                 const int hh = idx / D;
                 const int e = idx % D;
@@ -1624,19 +1627,19 @@ __device__ __forceinline__ void consume(const Params& p, unsigned char* smem, fl
                     // A single sink-set CTA per head holds the whole sink
                     // set: publish O_spec directly.
                     if (e == 0) {
-                        p.spec_ml[bh * 2] = M;
-                        p.spec_ml[bh * 2 + 1] = L;
+                        st_global_hint(p.spec_ml + bh * 2, M, keep);
+                        st_global_hint(p.spec_ml + bh * 2 + 1, L, keep);
                     }
-                    p.spec_o[bh * D + e] = O;
+                    st_global_hint(p.spec_o + bh * D + e, O, keep);
                     p.out_spec[bh * D + e] = __fdiv_rn(O, L);
                     continue;
                 }
                 const size_t row = bh * per + chunk;
                 if (e == 0) {
-                    part_ml[row * 2] = M;
-                    part_ml[row * 2 + 1] = L;
+                    st_global_hint(part_ml + row * 2, M, keep);
+                    st_global_hint(part_ml + row * 2 + 1, L, keep);
                 }
-                part_o[row * D + e] = O;
+                st_global_hint(part_o + row * D + e, O, keep);
             }
         }
         // Every consumer thread's partial is written (and the deposit slots

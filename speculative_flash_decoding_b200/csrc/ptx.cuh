@@ -66,6 +66,20 @@ __device__ __forceinline__ uint64_t l2_evict_first_policy() {
     return pol;
 }
 
+// L2 cache policy for data written once and read back soon by another
+// kernel or CTA (partials): kept in L2 ahead of evict-first lines.
+__device__ __forceinline__ uint64_t l2_evict_last_policy() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+// Global store with an L2 cache policy.
+__device__ __forceinline__ void st_global_hint(float* p, float v, uint64_t pol) {
+    asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;" ::"l"(p), "f"(v), "l"(pol)
+                 : "memory");
+}
+
 // 1-D bulk copy of `bytes` (a multiple of 16, both addresses 16-byte
 // aligned) from global to this CTA's shared memory, with L2 policy `pol`;
 // completion arrives as transaction bytes on `bar`.
