@@ -95,7 +95,9 @@ typedef enum {
  *            window), at some cost in throughput.
  */
 typedef enum {
-    ALSPEC_SCHEDULE_AUTO = 0,     /* STREAMS */
+    ALSPEC_SCHEDULE_AUTO = 0,     /* STREAMS; the sink-set kernel may take every SM (rather
+                                     than 3/4 of them) when a CTA would otherwise get more
+                                     than 24 tiles of 32 rows, so O_spec stays early */
     ALSPEC_SCHEDULE_STREAMS = 1,
     ALSPEC_SCHEDULE_FUSED = 2,
     ALSPEC_SCHEDULE_SINK_FIRST = 3

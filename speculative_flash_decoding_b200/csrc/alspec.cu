@@ -39,6 +39,11 @@ constexpr int kMaxSpecItems = kMaxSpecCtas;  // sink-set CTAs per (sequence, KV 
 #ifndef ALSPEC_SPEC_SM_SHARE_DEN
 #define ALSPEC_SPEC_SM_SHARE_DEN 4
 #endif
+// Sink-set tiles per CTA beyond which the automatic schedule lets the
+// sink-set CTAs take every SM (see make_plan).
+#ifndef ALSPEC_SPEC_TILES_WIDE
+#define ALSPEC_SPEC_TILES_WIDE 24
+#endif
 // Smallest middle chunk of the guided self-scheduled split, in tiles, and
 // the divisor of its chunk size (chunk c takes H * r_c / (DIV * P) of each
 // head's middle): DIV_SINGLE for a batch of one sequence, DIV otherwise.
@@ -235,11 +240,24 @@ void make_plan(const alspec_desc& d, int S, int W, int sms, Plan* pl) {
     // and all heads together within ALSPEC_SPEC_SM_SHARE of the SMs.
     // SINK_FIRST: the sink-set kernel runs alone, so it may take every SM.
     pl->sink_first = pl->schedule == ALSPEC_SCHEDULE_SINK_FIRST;
+    auto sink_ctas = [&](int share) {
+        const int room = std::max(1, share / std::max(1, heads));
+        return std::max(1, std::min({kMaxSpecItems, room, ceil_div(tiles_max, ALSPEC_SPEC_TILES)}));
+    };
     const int share_sms = pl->sink_first
                               ? sms
                               : sms * ALSPEC_SPEC_SM_SHARE_NUM / ALSPEC_SPEC_SM_SHARE_DEN;
-    const int room1 = std::max(1, share_sms / std::max(1, heads));
-    pl->n1 = std::max(1, std::min({kMaxSpecItems, room1, ceil_div(tiles_max, ALSPEC_SPEC_TILES)}));
+    pl->n1 = sink_ctas(share_sms);
+    // The automatic schedule aims at O_spec within a tenth of the layer:
+    // when that share leaves each sink-set CTA more than
+    // ALSPEC_SPEC_TILES_WIDE tiles (many sequences or a long window), the
+    // sink-set CTAs may take every SM.  Measured: the ragged batch of 8
+    // (64 heads, 65 tiles each) O_spec 27.7 -> 18.7 us, 0.149 -> 0.093 of
+    // the layer, for 2.9% of its step; the 70B batch of 4 (32 heads, 129
+    // tiles) 0.074 -> 0.063 for 0.7%.  An explicit STREAMS keeps the share.
+    if (d.schedule == ALSPEC_SCHEDULE_AUTO &&
+        ceil_div(tiles_max, pl->n1) > ALSPEC_SPEC_TILES_WIDE)
+        pl->n1 = sink_ctas(sms);
     if (fused)
         pl->n1 = std::max(1, std::min({kFusedSpecMaxItems, ceil_div(tiles_max, kFusedSpecMinTiles),
                                        std::max(1, sms / std::max(1, heads))}));

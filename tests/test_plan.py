@@ -217,13 +217,24 @@ def test_sink_set_ctas_and_middle_grid(shape):
     import speculative_flash_decoding_b200 as sfd
     B, Hq, Hkv, d, L, S, W = shape
     sms = 148
-    for sched in ("streams", "sink_first"):
+    tiles = -(-min(S, L) // 32) + -(-min(W, L) // 32)
+    heads = B * Hkv
+    n1_of = {}
+    for sched in ("streams", "sink_first", "auto"):
         desc = sfd.make_desc(B, Hq, Hkv, d, L, "bf16", schedule=sched)
         st, plan = sfd.alspec_query_plan(desc, S, W)
         assert st == 0
-        heads = B * Hkv
         assert plan["grid1"] == heads * plan["n1"]
-        share = sms if sched == "sink_first" else sms * 3 // 4
+        share = sms if sched in ("sink_first", "auto") else sms * 3 // 4
         assert plan["n1"] == 1 or plan["grid1"] <= share
         if plan["n2"]:
             assert plan["grid2"] == min(sms, heads * plan["n2"])
+        n1_of[sched] = plan["n1"]
+    # The automatic schedule widens the sink set only when 3/4 of the SMs
+    # would leave a sink-set CTA more than 24 tiles.
+    per_cta = -(-tiles // n1_of["streams"])
+    if per_cta > 24:
+        assert n1_of["auto"] >= n1_of["streams"]
+        assert n1_of["auto"] == max(1, min(8, sms // heads, -(-tiles // 5)))
+    else:
+        assert n1_of["auto"] == n1_of["streams"]
