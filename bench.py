@@ -830,28 +830,65 @@ def run_oproj_bench(args):
     weights = [(torch.randn(hidden, base.Hq * base.d, generator=g) / 64.0).to(torch.bfloat16)
                .to(device) for _ in range(n_layers)]
     results = {}
-    # The projection alone: 32 back-to-back calls (one per layer's weights),
-    # 32 MB of weights each, larger than L2 together.
+    # The projection alone: a CUDA graph of back-to-back calls (one per
+    # layer's weights, 32 MB each, larger than L2 together); each call's
+    # weights start streaming while the call before it finishes.  Beside
+    # it, one call on its own after an L2 scrub: launch, ramp and tail
+    # included.
     x = torch.randn(base.B, base.Hq * base.d, device=device)
     y = torch.empty(base.B, hidden, device=device)
     st = torch.cuda.Stream(device)
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+
+    def call(w):
+        assert sfd.alspec_oproj(x.data_ptr(), w.data_ptr(), y.data_ptr(), 0, base.B,
+                                base.Hq * base.d, hidden, st.cuda_stream) == 0
+
     with torch.cuda.stream(st):
-        for rep in range(4):
-            if rep == 3:
-                ev[0].record(st)
-            for w in weights:
-                assert sfd.alspec_oproj(x.data_ptr(), w.data_ptr(), y.data_ptr(), 0, base.B,
-                                        base.Hq * base.d, hidden, st.cuda_stream) == 0
+        for w in weights:
+            call(w)
+        assert sfd.alspec_graph_begin(st.cuda_stream) == 0
+        for w in weights:
+            call(w)
+        s_, gr = sfd.alspec_graph_end(st.cuda_stream)
+        assert s_ == 0
+        for _ in range(3):
+            assert sfd.alspec_graph_launch(gr, st.cuda_stream) == 0
+        ev[0].record(st)
+        for _ in range(4):
+            assert sfd.alspec_graph_launch(gr, st.cuda_stream) == 0
         ev[1].record(st)
     st.synchronize()
-    us = ev[0].elapsed_time(ev[1]) * 1e3 / n_layers
+    us = ev[0].elapsed_time(ev[1]) * 1e3 / (4 * n_layers)
+    assert sfd.alspec_graph_destroy(gr) == 0
+    # The L2 scrub: a write of twice its size, then a read of another such
+    # buffer, so the call does not pay for writing dirty lines back.
+    scrub = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    clean = torch.ones(32 << 20, dtype=torch.int32, device=device)
+    sink = torch.empty((), dtype=torch.int64, device=device)
+    # Everything is queued before the first scrub ends, so no call waits
+    # for the host.
+    iso_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(13)]
+    with torch.cuda.stream(st):
+        for i, (e0, e1) in enumerate(iso_ev):
+            scrub.zero_()
+            torch.sum(clean, dim=0, out=sink)
+            e0.record(st)
+            call(weights[i % n_layers])
+            e1.record(st)
+    st.synchronize()
+    iso = [e0.elapsed_time(e1) * 1e3 for e0, e1 in iso_ev[3:]]
+    del scrub, clean, sink
+    us_iso = statistics.median(iso)
     w_bytes = hidden * base.Hq * base.d * 2
     peak, peak_kind = measured_peak()
     results["oproj_alone"] = {"us_per_call": us, "weight_bytes": w_bytes,
                               "gbs": w_bytes / (us * 1e-6) / 1e9,
                               "frac_of_hbm_peak": w_bytes / (us * 1e-6) / 1e9 / peak,
-                              "peak_kind": peak_kind}
+                              "peak_kind": peak_kind,
+                              "timing": f"graph of {n_layers} back-to-back calls, 4 launches",
+                              "one_call_us": us_iso,
+                              "one_call_frac_of_hbm_peak": w_bytes / (us_iso * 1e-6) / 1e9 / peak}
     for tag, wl in (("as_specified", base),
                     ("strong_sinks_no_needles", base.replace(sink_bump=24.0, needles=("none",)))):
         layers = [workloads.make_layer(wl, layer=i, device=device) for i in range(n_layers)]

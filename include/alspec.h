@@ -239,7 +239,10 @@ alspec_status alspec_decode_traced(const alspec_desc* desc,
  * speculatively, "Approach"):
  *     y[b, j] = sum_i x[b, i] * w[j, i]
  * on CUDA cores (decode batches are small: the op streams w once, with bulk
- * copies, one CTA per SM).
+ * copies, two CTAs per SM).  The launch is programmatic: without `skip`, w
+ * starts streaming before the kernel ahead of it on `stream` has completed
+ * (x is read, and y written, only after it has), so w must not be written
+ * by that kernel; with `skip`, nothing is read before it has completed.
  *   x     device fp32 [batch][k], 16-byte aligned
  *   w     device bf16 [n][k] (row j = output feature j), 16-byte aligned
  *   y     device fp32 [batch][n]

@@ -80,6 +80,11 @@ constexpr size_t kAlign = 256;
 #define ALSPEC_SIDE_SMS 2
 #endif
 
+// CTAs of the projection's bulk-copy kernel per SM (its grid).
+#ifndef ALSPEC_OB_GRID_PER_SM
+#define ALSPEC_OB_GRID_PER_SM 2
+#endif
+
 thread_local cudaError_t t_last_error = cudaSuccess;
 
 // Remember the most recent failing CUDA call of this thread.
@@ -589,14 +594,25 @@ OprojParams oproj_params(const float* x, const void* w, float* y, const uint8_t*
 
 dim3 oproj_grid(int n) { return dim3((unsigned)ceil_div(n, kOprojWarps)); }
 
-// Foreground projection: the bulk-copy kernel, one CTA per SM (at most one
-// per output row).
+// Foreground projection: the bulk-copy kernel, ALSPEC_OB_GRID_PER_SM CTAs
+// per SM (at most one per output row).
 alspec_status launch_oproj_bulk(DeviceState* ds, const OprojParams& o, cudaStream_t s) {
     const OprojFn fn = oproj_bulk_kernel_for(o.B);
     alspec_status st = ensure_smem_attr(ds, reinterpret_cast<const void*>(fn), kObSmem);
     if (st != ALSPEC_OK) return st;
-    fn<<<std::min(ds->sm_count, o.N), kObThreads, kObSmem, s>>>(o);
-    return ok(cudaGetLastError()) ? ALSPEC_OK : ALSPEC_ERR_CUDA;
+    // Programmatic: the weights start streaming while the kernel ahead on
+    // the stream finishes (its SMs free up one by one).
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)std::min(ALSPEC_OB_GRID_PER_SM * ds->sm_count, o.N));
+    cfg.blockDim = dim3(kObThreads);
+    cfg.dynamicSmemBytes = kObSmem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr{};
+    attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr.val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    return ok(cudaLaunchKernelEx(&cfg, fn, o)) ? ALSPEC_OK : ALSPEC_ERR_CUDA;
 }
 
 alspec_status decode_impl(const alspec_desc* desc, const void* q, const void* k_cache,
@@ -827,7 +843,8 @@ alspec_status decode_impl(const alspec_desc* desc, const void* q, const void* k_
             cudaGraphNodeParams kp{};
             kp.type = cudaGraphNodeTypeKernel;
             kp.kernel.func = reinterpret_cast<void*>(rfn);
-            kp.kernel.gridDim = dim3((unsigned)std::min(ds->sm_count, op->hidden));
+            kp.kernel.gridDim =
+                dim3((unsigned)std::min(ALSPEC_OB_GRID_PER_SM * ds->sm_count, op->hidden));
             kp.kernel.blockDim = dim3(kObThreads);
             kp.kernel.sharedMemBytes = kObSmem;
             void* args[] = {&r};

@@ -1810,6 +1810,10 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const __grid_const
     __shared__ float accs[kMergeParts][kMergeCols];
     __shared__ int nlist;
     __shared__ int last;
+    // A kernel launched programmatically after this one (the output
+    // projection) may start now; it waits for this grid before it reads
+    // the outputs.
+    pdl_launch_dependents();
 
     const int mid_tiles = cdiv(seq_geom(p, b, false).mid_len, TT);
     const float2* mml = reinterpret_cast<const float2*>(p.mid_ml) + bh * p.n2;
@@ -1959,6 +1963,7 @@ __global__ void __launch_bounds__(kCmThreads, 1) merge_cluster_kernel(const __gr
     static_assert(sizeof(int) * kMaxChunks + sizeof(float) * kCmMaxHeads * (kMaxChunks + 2) +
                           sizeof(double) * (2 * kCmWarps + 2) + 8 + 4 <= kCmStatic,
                   "static shared memory");
+    pdl_launch_dependents();  // as in merge_kernel
 
     // Inputs only: the non-empty chunks of this sequence, in order.
     if (tid == 0) {

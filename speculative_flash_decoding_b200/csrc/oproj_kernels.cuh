@@ -119,17 +119,26 @@ __global__ void __launch_bounds__(kOprojWarps * 32) oproj_kernel(const __grid_co
 }
 
 // ----------------------------------------------------------------------
-// Foreground form: a persistent kernel, one CTA per SM, that streams the
-// weight rows with 1-D bulk copies (TMA, evict-first) into a ring of
-// 8 KB shared-memory stages -- so the bytes in flight are not bounded by the
-// L1's outstanding-miss tracking, which held plain loads near 2 TB/s; with
-// 24 stages (192 KB) nearly an SM's whole share of a 4096 x 4096 matrix is
-// in flight at once.  CTA c owns rows [c * R, (c + 1) * R); a row is
+// Foreground form: two CTAs per SM (a grid of twice the SM count), each
+// streaming its rows with 1-D bulk copies (TMA, evict-first) into a ring of
+// 12 8 KB shared-memory stages -- so the bytes in flight are not bounded by
+// the L1's outstanding-miss tracking, which held plain loads near 2 TB/s;
+// the two rings (192 KB per SM) hold nearly an SM's whole share of a
+// 4096 x 4096 matrix at once.  A CTA of 97 KB also fits beside the merge
+// kernel's CTAs, so a projection launched programmatically behind the merge
+// streams its weights while the merge runs (measured: 24 stages and one CTA
+// per SM streamed as fast alone, but the projection after the merge took
+// 2.5 us longer per layer).  CTA c owns rows [c * R, (c + 1) * R); a row is
 // P = 2K / 8192 stages; consumer warp w owns the CTA's rows w, w + 8, ...;
 // one producer lane fills the stages in order; for B <= 2 each lane loads
-// four chunks (and their x) before it computes on any of them.  Every wait is bounded: on expiry the kernel ORs the
-// timeout bit into p.err, stops, lets its copies land (bounded) and returns.
-constexpr int kObStages = 24;
+// four chunks (and their x) before it computes on any of them.  Every wait
+// is bounded: on expiry the kernel ORs the timeout bit into p.err, stops,
+// lets its copies land (bounded) and returns.
+#ifndef ALSPEC_OB_STAGES
+#define ALSPEC_OB_STAGES 12
+#endif
+constexpr int kObStages = ALSPEC_OB_STAGES;
+constexpr int kObMinBlocks = kObStages <= 13 ? 2 : 1;  // CTAs an SM can hold
 constexpr int kObPiece = 8192;   // bytes per stage
 constexpr int kObConsumers = 8;
 constexpr int kObThreads = (kObConsumers + 1) * 32;
@@ -153,7 +162,7 @@ __device__ __forceinline__ bool ob_wait(uint64_t* bar, uint32_t parity, volatile
 }
 
 template <int NB>
-__global__ void __launch_bounds__(kObThreads, 1) oproj_bulk_kernel(const __grid_constant__ OprojParams p) {
+__global__ void __launch_bounds__(kObThreads, kObMinBlocks) oproj_bulk_kernel(const __grid_constant__ OprojParams p) {
     extern __shared__ unsigned char ob_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(ob_raw) + 1023) & ~uintptr_t(1023));
@@ -167,11 +176,22 @@ __global__ void __launch_bounds__(kObThreads, 1) oproj_bulk_kernel(const __grid_
     volatile int* abort = reinterpret_cast<volatile int*>(ticket + kObStages);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-
-    unsigned live = 0;
-    for (int b = 0; b < p.B; ++b)
-        if (!p.skip || p.skip[b] == 0) live |= 1u << b;
-    if (live == 0) return;
+    // The kernel after this one on the stream may launch now (launched for
+    // that, it waits for this grid before it uses what this one writes).
+    pdl_launch_dependents();
+    // x, the gate and y belong to the kernels ahead of this one, which may
+    // still run (programmatic launch): the gate is read once they are done,
+    // and nothing streams before it says there is work.  Without a gate
+    // the weights (not written by those kernels: static in decode) stream
+    // at once, and the consumers wait before they read x.
+    unsigned live = (1u << p.B) - 1u;
+    if (p.skip) {
+        pdl_wait_prerequisite();
+        live = 0;
+        for (int b = 0; b < p.B; ++b)
+            if (p.skip[b] == 0) live |= 1u << b;
+        if (live == 0) return;
+    }
 
     const int row_bytes = p.K * 2;
     const int P = (row_bytes + kObPiece - 1) / kObPiece;  // stages per row
@@ -230,6 +250,7 @@ __global__ void __launch_bounds__(kObThreads, 1) oproj_bulk_kernel(const __grid_
     }
 
     // Consumers.
+    if (!p.skip) pdl_wait_prerequisite();
     for (int rl = warp; rl < nrows; rl += kObConsumers) {
         float2 acc[NB];
 #pragma unroll
@@ -266,17 +287,21 @@ __global__ void __launch_bounds__(kObThreads, 1) oproj_bulk_kernel(const __grid_
             const int nch = min(kObPiece, row_bytes - off) >> 4;  // 16-byte chunks
             const uint4* ws = reinterpret_cast<const uint4*>(smem + slot * kObPiece);
             const int c_base = off >> 4;
-            constexpr int U = NB <= 2 ? 4 : 1;  // chunks per lane loaded before use
+            // Chunks per lane loaded (with their x) before use; a batch of 8
+            // reads x as it goes.  Both keep the kernel within the registers
+            // of two CTAs per SM.
+            constexpr int U = NB == 1 ? 4 : NB == 2 ? 2 : 1;
+            constexpr bool kPre = NB <= 4;
             for (int c0 = lane; c0 < nch; c0 += 32 * U) {
                 uint4 wq[U];
-                float4 xv[U][NB][2];
+                float4 xv[U][kPre ? NB : 1][2];
 #pragma unroll
                 for (int u = 0; u < U; ++u) {
                     const int c = c0 + 32 * u;
                     if (c < nch) {
                         wq[u] = ws[c];
 #pragma unroll
-                        for (int b = 0; b < NB; ++b) {
+                        for (int b = 0; b < (kPre ? NB : 0); ++b) {
                             if (!((live >> b) & 1u)) continue;
                             const float4* xp = reinterpret_cast<const float4*>(
                                                    p.x + (size_t)b * p.K) + 2 * (c_base + c);
@@ -297,8 +322,16 @@ __global__ void __launch_bounds__(kObThreads, 1) oproj_bulk_kernel(const __grid_
 #pragma unroll
                     for (int b = 0; b < NB; ++b) {
                         if (!((live >> b) & 1u)) continue;
-                        const float4 x0 = xv[u][b][0];
-                        const float4 x1 = xv[u][b][1];
+                        float4 x0, x1;
+                        if constexpr (kPre) {
+                            x0 = xv[u][b][0];
+                            x1 = xv[u][b][1];
+                        } else {
+                            const float4* xp = reinterpret_cast<const float4*>(
+                                                   p.x + (size_t)b * p.K) + 2 * (c_base + c0);
+                            x0 = __ldg(xp);
+                            x1 = __ldg(xp + 1);
+                        }
                         acc[b] = __ffma2_rn(wp[0], make_float2(x0.x, x0.y), acc[b]);
                         acc[b] = __ffma2_rn(wp[1], make_float2(x0.z, x0.w), acc[b]);
                         acc[b] = __ffma2_rn(wp[2], make_float2(x1.x, x1.y), acc[b]);
@@ -339,7 +372,7 @@ using OprojFn = void (*)(OprojParams);
 
 // The kernels for a batch of B rows (1 <= B <= kOprojMaxB): the background
 // form (no shared memory, so it shares SMs with a running middle kernel) and
-// the foreground form (bulk copies, one CTA per SM).
+// the foreground form (bulk copies, two CTAs per SM).
 inline OprojFn oproj_kernel_for(int B) {
     return B <= 1 ? oproj_kernel<1> : B <= 2 ? oproj_kernel<2> : B <= 4 ? oproj_kernel<4>
                                                                        : oproj_kernel<8>;

@@ -173,3 +173,45 @@ def test_speculative_projection_over_layers_in_one_graph(cuda_device):
                                   workloads.to_numpy_bits(w))
         assert _row_rel(o["y"].cpu().numpy(), mine).max() < ROW_TOL
     assert dec.device_error() == (0, 0)
+
+
+def test_projection_behind_the_merge_reads_fresh_outputs(cuda_device):
+    """The projection is launched programmatically and the merge lets its
+    dependents launch early: captured right behind two decodes that write
+    the same O_exact buffer, each projection must see its own layer's
+    O_exact (x is read only once the merge has completed), never the
+    previous layer's."""
+    import speculative_flash_decoding_b200 as sfd
+    wl = workloads.CONFIGS[1].replace(L=16384)
+    layers = [workloads.make_layer(wl, layer=i, device=cuda_device) for i in range(2)]
+    kdim = wl.Hq * wl.d
+    hidden = 4096
+    w = _bf16_weights(hidden, kdim, 77, cuda_device)
+    dec = sfd.Decoder(wl.B, wl.Hq, wl.Hkv, wl.d, wl.L, wl.dtype, wl.S, wl.W, device=cuda_device)
+    exact = []
+    for d in layers:
+        o = dec.decode(d["q"], d["k"], d["v"], d["seq_lens"], wl.lam)
+        torch.cuda.synchronize()
+        exact.append(o["out_exact"].cpu().numpy().reshape(wl.B, -1))
+    assert _row_rel(exact[0], exact[1]).min() > 0.5
+    out = dec.alloc_outputs()
+    ys = [torch.full((wl.B, hidden), 7.0, device=cuda_device) for _ in layers]
+    stream = torch.cuda.Stream(cuda_device)
+    with torch.cuda.stream(stream):
+        assert sfd.alspec_graph_begin(stream.cuda_stream) == 0
+        for d, y in zip(layers, ys):
+            dec.decode(d["q"], d["k"], d["v"], d["seq_lens"], wl.lam, out=out, stream=stream)
+            assert sfd.alspec_oproj(out["out_exact"].data_ptr(), w.data_ptr(), y.data_ptr(), 0,
+                                    wl.B, kdim, hidden, stream.cuda_stream) == 0
+        st, g = sfd.alspec_graph_end(stream.cuda_stream)
+        assert st == 0 and g
+        w_bits = workloads.to_numpy_bits(w)
+        for _ in range(3):
+            for y in ys:
+                y.fill_(7.0)
+            assert sfd.alspec_graph_launch(g, stream.cuda_stream) == 0
+            stream.synchronize()
+            for y, x in zip(ys, exact):
+                assert _row_rel(y.cpu().numpy(), oracle.oproj(x, w_bits)).max() < ROW_TOL
+        assert sfd.alspec_graph_destroy(g) == 0
+    assert dec.device_error() == (0, 0)
