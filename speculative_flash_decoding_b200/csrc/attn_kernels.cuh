@@ -1080,6 +1080,51 @@ __device__ __forceinline__ void fill_stage(const Params& p, unsigned char* smem,
 // CTA's init barrier) fills the untouched stages one tile per lane, so the
 // first copies leave within a few hundred cycles; lane 0 alone continues
 // with the rest, waiting for each stage to be released.
+// The ring's first fills on the tensor-core engine, by the producer warp:
+// lane l issues copy l % OPS (K or V, 64 columns) of stage l / OPS, so one
+// copy instruction of the warp issues stage 0's copies first, then stage
+// 1's, ... (one lane per stage, each issuing all of its stage's copies,
+// put the first stage's last copy behind every other stage's first ones:
+// measured, the burst of 48 copies took ~1.5 us to issue).  Same stage
+// state as fill_stage for tiles 0 .. fresh-1 of `it`.
+template <typename T, int D, int G, bool SPEC, bool MMA, bool FUSED>
+__device__ __forceinline__ void fill_fresh(const Params& p, unsigned char* smem, int4* meta,
+                                           uint32_t* fill, uint64_t* full_bar, int item,
+                                           const Item& it, int fresh, int ntiles, int lane) {
+    using C = Cfg<T, D, G, SPEC, MMA, FUSED>;
+    constexpr int TT = C::TT;
+    constexpr int OPS = 2 * (D / 64);  // copies per stage
+    constexpr int PER = 32 / OPS;      // stages per round of the warp
+    static_assert(32 % OPS == 0, "copies per stage");
+    const int head_row = (it.b * p.Hkv + it.kvh) * p.Lmax;
+    const uint64_t pol = l2_evict_first_policy();
+    for (int s0 = 0; s0 < fresh; s0 += PER) {
+        const int s = s0 + lane / OPS;
+        const int op = lane % OPS;
+        const bool mine = s < fresh;
+        int start = 0, nvalid = 0;
+        if (mine && s < it.ntiles) tile_rows<SPEC, TT, FUSED>(it, s, start, nvalid);
+        if (mine && op == 0) {
+            st_release_shared(fill + s, (uint32_t)s);
+            meta[s] = make_int4(item, s, nvalid,
+                                (FUSED ? it.ntiles << 1 : 0) |
+                                    (s >= ntiles - C::NTW ? kLastTileFlag : 0));
+            if (nvalid == 0)
+                mbar_arrive(full_bar + s);
+            else
+                mbar_arrive_expect_tx(full_bar + s, (uint32_t)C::kStageBytes);
+        }
+        __syncwarp();  // each stage's expected bytes are set before its copies
+        if (mine && nvalid > 0) {
+            const int h = op >> 1;
+            char* dst = reinterpret_cast<char*>(smem) + s * C::kStageBytes +
+                        ((op & 1) ? C::kTileBytes : 0) + h * TT * 128;
+            tma_load_2d(dst, (op & 1) ? static_cast<const void*>(&p.tmap_v) : &p.tmap_k, 64 * h,
+                        head_row + start, full_bar + s, pol);
+        }
+    }
+}
+
 template <typename T, int D, int G, bool SPEC, bool MMA, bool FUSED>
 __device__ __forceinline__ void produce(const Params& p, unsigned char* smem, int4* meta,
                                         uint32_t* fill, uint64_t* full_bar, uint64_t* empty_bar,
@@ -1090,9 +1135,14 @@ __device__ __forceinline__ void produce(const Params& p, unsigned char* smem, in
     auto rounded = [](const Item& it) { return (it.ntiles + C::NTW - 1) / C::NTW * C::NTW; };
     const bool have0 = item0 < n_items && it0.ntiles > 0;
     const int fresh = have0 ? min(rounded(it0), C::STAGES) : 0;
-    for (int t = lane; t < fresh; t += 32)
-        fill_stage<T, D, G, SPEC, MMA, FUSED>(p, smem, meta, fill, full_bar, t, (uint32_t)t, item0,
-                                              it0, t, rounded(it0));
+    if constexpr (MMA) {
+        fill_fresh<T, D, G, SPEC, MMA, FUSED>(p, smem, meta, fill, full_bar, item0, it0, fresh,
+                                              rounded(it0), lane);
+    } else {
+        for (int t = lane; t < fresh; t += 32)
+            fill_stage<T, D, G, SPEC, MMA, FUSED>(p, smem, meta, fill, full_bar, t, (uint32_t)t,
+                                                  item0, it0, t, rounded(it0));
+    }
     if (lane != 0) return;
 
     uint32_t gt = (uint32_t)fresh;
