@@ -257,9 +257,9 @@ void make_plan(const alspec_desc& d, int S, int W, int sms, Plan* pl) {
     // when that share leaves each sink-set CTA more than
     // ALSPEC_SPEC_TILES_WIDE tiles (many sequences or a long window), the
     // sink-set CTAs may take every SM.  Measured: the ragged batch of 8
-    // (64 heads, 65 tiles each) O_spec 27.7 -> 18.7 us, 0.149 -> 0.093 of
-    // the layer, for 2.9% of its step; the 70B batch of 4 (32 heads, 129
-    // tiles) 0.074 -> 0.063 for 0.7%.  An explicit STREAMS keeps the share.
+    // (64 heads, 65 tiles each) O_spec 27.9 -> 17.2 us, 0.150 -> 0.087 of
+    // the layer, for 1.6% of its step; the 70B batch of 4 (32 heads, 129
+    // tiles) 0.071 -> 0.061 for 0.3%.  An explicit STREAMS keeps the share.
     if (d.schedule == ALSPEC_SCHEDULE_AUTO &&
         ceil_div(tiles_max, pl->n1) > ALSPEC_SPEC_TILES_WIDE)
         pl->n1 = sink_ctas(sms);
