@@ -1868,17 +1868,25 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const __grid_const
     const int mid_tiles = cdiv(seq_geom(p, b, false).mid_len, TT);
     const float2* mml = reinterpret_cast<const float2*>(p.mid_ml) + bh * p.n2;
 
-    // Non-empty chunks, in chunk order (thread 0 walks the table with
-    // uniform indices; the table lives in parameter space).
-    if (tid == 0) {
-        int count = 0, prev = 0;
-#pragma unroll 8
-        for (int c = 0; c < p.n2; ++c) {
-            const int t = (int)(((unsigned long long)mid_tiles * p.fq[c + 1]) >> kFracBits);
-            if (t > prev) list[count++] = c;
-            prev = t;
+    // Non-empty chunks, in chunk order: warp 0 tests 32 chunks at a time
+    // (chunk c covers tiles [mt * fq[c] >> 24, mt * fq[c + 1] >> 24)) and
+    // compacts them with a ballot (merge CTAs placed as the last middle
+    // CTAs exit do this on the layer's critical path).
+    if (warp == 0) {
+        int count = 0;
+        for (int c0 = 0; c0 < p.n2; c0 += 32) {
+            const int c = c0 + lane;
+            bool nonempty = false;
+            if (c < p.n2) {
+                const int lo = (int)(((unsigned long long)mid_tiles * p.fq[c]) >> kFracBits);
+                const int hi = (int)(((unsigned long long)mid_tiles * p.fq[c + 1]) >> kFracBits);
+                nonempty = hi > lo;
+            }
+            const unsigned m = __ballot_sync(0xffffffffu, nonempty);
+            if (nonempty) list[count + __popc(m & ((1u << lane) - 1u))] = c;
+            count += __popc(m);
         }
-        nlist = count;
+        if (lane == 0) nlist = count;
     }
     __syncthreads();
     const int n = nlist;
