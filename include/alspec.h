@@ -115,6 +115,11 @@ typedef enum {
 /* Bits of the device error word (alspec_get_device_error). */
 #define ALSPEC_DEVERR_SEQ_LEN 0x1u   /* a seq_lens entry outside [1, max_seq_len]; it was clamped */
 #define ALSPEC_DEVERR_TIMEOUT 0x2u   /* a bounded wait inside a kernel gave up; outputs invalid   */
+/* Only in the bounds-checked debug build of this library (libalspec_debug.so,
+ * the same sources compiled with ALSPEC_DEBUG_BOUNDS): a kernel found an
+ * index outside its buffer (shared-memory slot, chunk list, partial slot,
+ * copy source or output) and skipped that access; outputs invalid. */
+#define ALSPEC_DEVERR_BOUNDS 0x4u
 
 /*
  * Problem description.  Shapes (row-major, last index fastest):

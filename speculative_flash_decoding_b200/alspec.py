@@ -15,7 +15,11 @@ import ctypes
 import os
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libalspec.so")
+# ALSPEC_LIBRARY=debug loads the bounds-checked build of the same sources
+# (libalspec_debug.so); the default is libalspec.so.
+_LIB_NAME = {"": "libalspec.so", "default": "libalspec.so",
+             "debug": "libalspec_debug.so"}[os.environ.get("ALSPEC_LIBRARY", "")]
+LIB_PATH = os.path.join(_PKG, _LIB_NAME)
 
 ALSPEC_OK = 0
 ALSPEC_ERR_INVALID_ARG = 1
@@ -32,6 +36,7 @@ ALSPEC_PROF_EVENTS = 5
 
 ALSPEC_DEVERR_SEQ_LEN = 0x1
 ALSPEC_DEVERR_TIMEOUT = 0x2
+ALSPEC_DEVERR_BOUNDS = 0x4   # bounds-checked debug build only
 
 # Every symbol the header declares, with (restype, argtypes).
 _vp, _i, _f, _sz, _u32p = (ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t,
@@ -90,7 +95,7 @@ ALSPEC_NOALLOC_SCRATCH_BYTES = 8 << 20
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(
-            f"libalspec.so not found at {LIB_PATH}; build it with "
+            f"{_LIB_NAME} not found at {LIB_PATH}; build it with "
             "`python speculative_flash_decoding_b200/build.py` (there is no CPU fallback)")
     lib = ctypes.CDLL(LIB_PATH)
     for name, (res, args) in SIGNATURES.items():

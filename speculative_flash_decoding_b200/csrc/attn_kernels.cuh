@@ -86,6 +86,7 @@ constexpr int kMaxSpecCtas = 8;
 
 constexpr unsigned kErrSeqLen = 1u;   // ALSPEC_DEVERR_SEQ_LEN
 constexpr unsigned kErrTimeout = 2u;  // ALSPEC_DEVERR_TIMEOUT
+constexpr unsigned kErrBounds = 4u;   // ALSPEC_DEVERR_BOUNDS (debug build)
 
 // Counter words at the head of the workspace, then the per-sequence
 // tickets [B] (merge kernel: one per CTA of the sequence; one-launch
@@ -166,6 +167,20 @@ __device__ __forceinline__ void trace_publish(const Params& p, int which) {
 }
 
 __host__ __device__ __forceinline__ int cdiv(int a, int b) { return (a + b - 1) / b; }
+
+// Bounds checks of the debug build (compiled with ALSPEC_DEBUG_BOUNDS): an
+// index outside its buffer ORs kErrBounds into the workspace's error word
+// and the caller skips the access (never a trap).  In the normal build
+// every check is the constant true and its condition is not evaluated.
+#ifdef ALSPEC_DEBUG_BOUNDS
+__device__ __noinline__ bool bounds_fail(unsigned* ctr) {
+    atomicOr(ctr + kCtrError, kErrBounds);
+    return false;
+}
+#define ALSPEC_IN_BOUNDS(p, cond) ((cond) ? true : ::alspec::bounds_fail((p).ctr))
+#else
+#define ALSPEC_IN_BOUNDS(p, cond) true
+#endif
 
 // Token geometry of one sequence: sink tokens [0, ns), window [ws, L),
 // middle [ns, ws).
@@ -938,9 +953,10 @@ __device__ __forceinline__ void cluster_gather(const Params& p, const float* dep
             }
             x[k] = val;  // (m, l, o[0..D)) of head hh
         }
-        for (int j = 0; j < n; ++j)
-            st_async_v4(dsmem_addr(dst, (uint32_t)j) + 16u * (uint32_t)v, x,
-                        dsmem_addr(bar, (uint32_t)j));
+        if (ALSPEC_IN_BOUNDS(p, rank < (uint32_t)n && n <= kMaxSpecCtas))
+            for (int j = 0; j < n; ++j)
+                st_async_v4(dsmem_addr(dst, (uint32_t)j) + 16u * (uint32_t)v, x,
+                            dsmem_addr(bar, (uint32_t)j));
     }
 
     // Wait (bounded) for the n1 slots sent to this CTA.
@@ -981,6 +997,7 @@ __device__ __forceinline__ void cluster_gather(const Params& p, const float* dep
             }
         }
         const size_t bh = (size_t)b * p.Hq + kvh * G + hh;
+        if (!ALSPEC_IN_BOUNDS(p, b < p.B && kvh * G + hh < p.Hq)) continue;
         if (e == 0) {
             p.spec_ml[bh * 2] = M;
             p.spec_ml[bh * 2 + 1] = L;
@@ -1012,6 +1029,7 @@ template <int D>
 __device__ __forceinline__ void write_flag(const Params& p, int b, int lane) {
     constexpr int NS = merge_splits(D);
     __syncwarp();  // orders lane 0's acquire of the ticket before every lane's loads
+    if (!ALSPEC_IN_BOUNDS(p, b >= 0 && b < p.B)) return;
     double D2 = 0.0, N2 = 0.0;
     const float2* dn = reinterpret_cast<const float2*>(p.dn) + (size_t)b * p.Hq * NS;
     for (int i = lane; i < p.Hq * NS; i += 32) {
@@ -1047,6 +1065,10 @@ __device__ __forceinline__ void fill_stage(const Params& p, unsigned char* smem,
     const int head_row = (it.b * p.Hkv + it.kvh) * p.Lmax;
     int start = 0, nvalid = 0;
     if (t < it.ntiles) tile_rows<SPEC, TT, FUSED>(it, t, start, nvalid);
+    if (!ALSPEC_IN_BOUNDS(p, nvalid <= 0 || (start >= 0 && nvalid <= TT &&
+                                             start + nvalid <= p.Lmax && it.b < p.B &&
+                                             it.kvh < p.Hkv)))
+        nvalid = 0;  // (the stage then arrives empty)
     st_release_shared(fill + s, gt);  // this fill is the one for tile gt
     meta[s] = make_int4(item, t, nvalid,
                         (FUSED ? it.ntiles << 1 : 0) | (t >= ntiles - C::NTW ? kLastTileFlag : 0));
@@ -1104,6 +1126,10 @@ __device__ __forceinline__ void fill_fresh(const Params& p, unsigned char* smem,
         const bool mine = s < fresh;
         int start = 0, nvalid = 0;
         if (mine && s < it.ntiles) tile_rows<SPEC, TT, FUSED>(it, s, start, nvalid);
+        if (mine && !ALSPEC_IN_BOUNDS(p, nvalid <= 0 || (start >= 0 && nvalid <= TT &&
+                                                         start + nvalid <= p.Lmax &&
+                                                         it.b < p.B && it.kvh < p.Hkv)))
+            nvalid = 0;  // (the stage then arrives empty)
         if (mine && op == 0) {
             st_release_shared(fill + s, (uint32_t)s);
             meta[s] = make_int4(item, s, nvalid,
@@ -1369,7 +1395,8 @@ __device__ __forceinline__ bool fused_head_merge(const Params& p, int bh, float*
         const uint64_t pol = l2_evict_first_policy();
         for (size_t off = (size_t)lane * kPiece; off < blk_bytes; off += 32 * (size_t)kPiece) {
             const uint32_t nb = (uint32_t)(blk_bytes - off < kPiece ? blk_bytes - off : kPiece);
-            bulk_load(ring + off, src + off, nb, mbar, pol);
+            if (ALSPEC_IN_BOUNDS(p, off + nb <= ring_bytes && bq0 + G <= (size_t)p.B * p.Hq))
+                bulk_load(ring + off, src + off, nb, mbar, pol);
         }
     }
     // O_spec and the merged sink-set partial, while the copies land.
@@ -1389,7 +1416,8 @@ __device__ __forceinline__ bool fused_head_merge(const Params& p, int bh, float*
                 ne = hi > lo;
             }
             const unsigned bal = __ballot_sync(0xffffffffu, ne);
-            if (ne) list[count + __popc(bal & ((1u << lane) - 1u))] = c;
+            const int at = count + __popc(bal & ((1u << lane) - 1u));
+            if (ne && ALSPEC_IN_BOUNDS(p, at < kMaxChunks)) list[at] = c;
             count += __popc(bal);
         }
         if (lane == 0) *nlist = count;
@@ -1516,7 +1544,7 @@ __device__ __forceinline__ bool fused_head_merge(const Params& p, int bh, float*
             dd += __shfl_xor_sync(0xffffffffu, dd, o);
             nn += __shfl_xor_sync(0xffffffffu, nn, o);
         }
-        if (act && (lane & 7) == 0)
+        if (act && (lane & 7) == 0 && ALSPEC_IN_BOUNDS(p, bq < (size_t)p.B * p.Hq))
             *reinterpret_cast<float2*>(p.dn + (bq * NS + e4 / 8) * 2) = make_float2(dd, nn);
     }
     // Every slot of this head is written once this passes.
@@ -1636,7 +1664,9 @@ __device__ __forceinline__ void consume(const Params& p, unsigned char* smem, fl
         if (!(mt.w & kLastTileFlag)) continue;
 
         // ---- end of this item: combine the warps' states into one partial.
-        st.deposit(deposit + (hw * C::NTW + tw) * C::kSlotFloats, lane);
+        if (ALSPEC_IN_BOUNDS(p, (hw * C::NTW + tw + 1) * C::kSlotFloats * (int)sizeof(float) <=
+                                    C::kDepositBytes))
+            st.deposit(deposit + (hw * C::NTW + tw) * C::kSlotFloats, lane);
         if (SPEC && p.n1 > 1) {
             // Sink set split over a cluster: the warps' states stay in the
             // deposit slots and the cluster merge reads them directly.
@@ -1673,6 +1703,8 @@ __device__ __forceinline__ void consume(const Params& p, unsigned char* smem, fl
                     O = fmaf(f, ws[2 + e], O);
                 }
                 const size_t bh = (size_t)b * p.Hq + kvh * G + hh;
+                if (!ALSPEC_IN_BOUNDS(p, b < p.B && kvh < p.Hkv && chunk >= 0 && chunk < per))
+                    continue;
                 if (SPEC) {
                     // A single sink-set CTA per head holds the whole sink
                     // set: publish O_spec directly.
@@ -1883,13 +1915,22 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const __grid_const
                 nonempty = hi > lo;
             }
             const unsigned m = __ballot_sync(0xffffffffu, nonempty);
-            if (nonempty) list[count + __popc(m & ((1u << lane) - 1u))] = c;
+            const int at = count + __popc(m & ((1u << lane) - 1u));
+            if (nonempty && ALSPEC_IN_BOUNDS(p, at < kMaxChunks)) list[at] = c;
             count += __popc(m);
         }
         if (lane == 0) nlist = count;
     }
     __syncthreads();
     const int n = nlist;
+#ifdef ALSPEC_DEBUG_BOUNDS
+    // Every chunk of the list names a chunk of this head (a CTA-wide answer).
+    if (__syncthreads_or(!(h < p.Hq && b < p.B && n >= 0 && n <= p.n2 &&
+                           (tid >= n || (list[tid] >= 0 && list[tid] < p.n2))))) {
+        if (tid == 0) bounds_fail(p.ctr);
+        return;
+    }
+#endif
     // Everything above only read inputs; the partials are written by the
     // kernels this one follows, which may still be running.
     pdl_wait_prerequisite();
@@ -2038,11 +2079,22 @@ __global__ void __launch_bounds__(kCmThreads, 1) merge_cluster_kernel(const __gr
         fence_barrier_init();
     }
     __syncthreads();
-    const int n = nlist;
+    int n = nlist;
+#ifdef ALSPEC_DEBUG_BOUNDS
+    // Every chunk of the list names a chunk of the sequence; else no middle
+    // partial is read (a CTA-wide answer; the cluster's barriers still run).
+    if (__syncthreads_or(!(n >= 0 && n <= p.n2 &&
+                           (tid >= n || (list[tid] >= 0 && list[tid] < p.n2))))) {
+        if (tid == 0) bounds_fail(p.ctr);
+        n = 0;
+    }
+#endif
     // The partials are written by the kernels this one follows.
     pdl_wait_prerequisite();
     const size_t bytes = (size_t)hpc * p.n2 * D * sizeof(float);
-    if (warp == 0 && bytes > 0) {
+    if (warp == 0 && bytes > 0 &&
+        ALSPEC_IN_BOUNDS(p, bytes + 128 <= dynamic_smem_size() &&
+                                bq0 + hpc <= (size_t)p.B * p.Hq)) {
         constexpr uint32_t kPiece = 16384;
         const char* src = reinterpret_cast<const char*>(p.mid_o + bq0 * p.n2 * D);
         fence_proxy_async_global();
@@ -2129,7 +2181,7 @@ __global__ void __launch_bounds__(kCmThreads, 1) merge_cluster_kernel(const __gr
         const float a = (acc[0] + acc[1]) + (acc[2] + acc[3]);
         const float o_exact = __fdiv_rn(a, fl[hh][1]);
         const float o_spec = __fdiv_rn(os, sl);
-        p.out_exact[bq * D + e] = o_exact;
+        if (ALSPEC_IN_BOUNDS(p, bq < (size_t)p.B * p.Hq)) p.out_exact[bq * D + e] = o_exact;
         const float diff = o_exact - o_spec;
         dd += (double)(diff * diff);
         nn += (double)(o_exact * o_exact);

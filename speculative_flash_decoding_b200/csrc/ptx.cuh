@@ -105,6 +105,13 @@ __device__ __forceinline__ void tma_load_2d(void* dst_smem, const void* tmap, in
         : "memory");
 }
 
+// Bytes of dynamic shared memory the launch gave this CTA.
+__device__ __forceinline__ uint32_t dynamic_smem_size() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%dynamic_smem_size;" : "=r"(r));
+    return r;
+}
+
 __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
 }

@@ -44,6 +44,20 @@ def test_library_exports_every_declared_symbol(header):
         assert hasattr(lib, name), f"{os.path.basename(LIBRARY_OF[header])} does not export {name}"
 
 
+def test_debug_library_exports_the_decode_surface():
+    """The bounds-checked build exports exactly the decode library's symbols."""
+    debug = ctypes.CDLL(os.path.join(PKG, "libalspec_debug.so"))
+    for name in declared_functions():
+        assert hasattr(debug, name), f"libalspec_debug.so does not export {name}"
+    assert not hasattr(debug, "alspec_read_probe")
+
+
+def test_debug_bounds_bit_is_declared():
+    text = open(HEADER).read()
+    assert "#define ALSPEC_DEVERR_BOUNDS 0x4u" in text
+    assert sfd.ALSPEC_DEVERR_BOUNDS == 0x4
+
+
 def test_decode_library_has_no_benchmark_probe():
     """The read-bandwidth probe is a measurement aid in its own library."""
     assert not hasattr(ctypes.CDLL(sfd.LIB_PATH), "alspec_read_probe")
