@@ -137,10 +137,16 @@ __global__ void __launch_bounds__(kOprojWarps * 32) oproj_kernel(const __grid_co
 #ifndef ALSPEC_OB_STAGES
 #define ALSPEC_OB_STAGES 12
 #endif
+#ifndef ALSPEC_OB_CONSUMERS
+#define ALSPEC_OB_CONSUMERS 8
+#endif
+#ifndef ALSPEC_OB_MIN_BLOCKS
+#define ALSPEC_OB_MIN_BLOCKS (ALSPEC_OB_STAGES <= 13 ? 2 : 1)
+#endif
 constexpr int kObStages = ALSPEC_OB_STAGES;
-constexpr int kObMinBlocks = kObStages <= 13 ? 2 : 1;  // CTAs an SM can hold
+constexpr int kObMinBlocks = ALSPEC_OB_MIN_BLOCKS;  // CTAs an SM can hold
 constexpr int kObPiece = 8192;   // bytes per stage
-constexpr int kObConsumers = 8;
+constexpr int kObConsumers = ALSPEC_OB_CONSUMERS;
 constexpr int kObThreads = (kObConsumers + 1) * 32;
 constexpr int kObSmem = kObStages * kObPiece + 2 * kObStages * 8 + kObStages * 4 + 16 + 1024;
 
