@@ -386,11 +386,22 @@ def measure(wl, n_layers, steps, warmup, device, ranks, args, want_e2e=True, lat
 
     n_lat = n_layers if n_layers >= 2 else lat_layers
     layers = [workloads.make_layer(wl, layer=i, device=device) for i in range(max(n_layers, n_lat))]
-    q_all = torch.stack([d["q"] for d in layers]).contiguous()            # [layers, B, Hq, d]
-    lens_all = torch.stack([d["seq_lens"] for d in layers]).contiguous()  # [layers, B]
+    # Each layer's query vectors and lengths side by side in one buffer
+    # (q_i, then lens_i padded to 16 bytes), so that a step's inputs are one
+    # contiguous host-to-device copy; likewise every layer's rel_l2, then
+    # every layer's flag, for the copy back.
+    q_bytes = wl.B * wl.Hq * wl.d * wl.elem_bytes
+    l_bytes = wl.B * 4
+    in_stride = q_bytes + (l_bytes + 15) // 16 * 16
+    inputs = torch.empty(len(layers) * in_stride, dtype=torch.uint8, device=device)
     for i, d in enumerate(layers):
-        d["q"] = q_all[i]
-        d["seq_lens"] = lens_all[i]
+        base = i * in_stride
+        q_view = inputs[base:base + q_bytes].view(d["q"].dtype).view(d["q"].shape)
+        l_view = inputs[base + q_bytes:base + q_bytes + l_bytes].view(torch.int32)
+        q_view.copy_(d["q"])
+        l_view.copy_(d["seq_lens"])
+        d["q"] = q_view
+        d["seq_lens"] = l_view
     kv_bytes = sum(workloads.kv_bytes(wl, d["lens"]) for d in layers[:n_layers])
     lat_kv_bytes = sum(workloads.kv_bytes(wl, d["lens"]) for d in layers[:n_lat])
     dec = sfd.Decoder(wl.B, wl.Hq, wl.Hkv, wl.d, wl.L, wl.dtype, wl.S, wl.W, device=device,
@@ -400,8 +411,9 @@ def measure(wl, n_layers, steps, warmup, device, ranks, args, want_e2e=True, lat
     n_all = len(layers)
     out_spec = torch.empty(n_all, wl.B, wl.Hq, wl.d, dtype=torch.float32, device=device)
     out_exact = torch.empty_like(out_spec)
-    rel_all = torch.empty(n_all, wl.B, dtype=torch.float32, device=device)
-    commit_all = torch.empty(n_all, wl.B, dtype=torch.uint8, device=device)
+    results = torch.empty(n_all * wl.B * 5, dtype=torch.uint8, device=device)
+    rel_all = results[:n_all * wl.B * 4].view(torch.float32).view(n_all, wl.B)
+    commit_all = results[n_all * wl.B * 4:].view(n_all, wl.B)
     outs = [dict(out_spec=out_spec[i], out_exact=out_exact[i], rel_l2=rel_all[i],
                  commit=commit_all[i]) for i in range(n_all)]
     stream = torch.cuda.Stream(device)
@@ -546,10 +558,9 @@ def measure(wl, n_layers, steps, warmup, device, ranks, args, want_e2e=True, lat
     # replay the step, read every layer's rel_l2 and flag back.
     e2e = None
     if want_e2e:
-        q_host = q_all[:n_layers].cpu().pin_memory()
-        lens_host = lens_all[:n_layers].cpu().pin_memory()
-        rel_host = torch.empty((n_layers, wl.B), dtype=rel_all.dtype).pin_memory()
-        com_host = torch.empty((n_layers, wl.B), dtype=commit_all.dtype).pin_memory()
+        in_dev = inputs[:n_layers * in_stride]
+        in_host = in_dev.cpu().pin_memory()
+        out_host = torch.empty(results.numel(), dtype=torch.uint8).pin_memory()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         ranks.barrier()
@@ -557,25 +568,23 @@ def measure(wl, n_layers, steps, warmup, device, ranks, args, want_e2e=True, lat
         with torch.cuda.stream(stream):
             e0.record(stream)
             for i in range(steps):
-                q_all[:n_layers].copy_(q_host, non_blocking=True)
-                lens_all[:n_layers].copy_(lens_host, non_blocking=True)
+                in_dev.copy_(in_host, non_blocking=True)
                 sfd.alspec_graph_launch(graphs[i], stream.cuda_stream)
-                rel_host.copy_(rel_all[:n_layers], non_blocking=True)
-                com_host.copy_(commit_all[:n_layers], non_blocking=True)
+                out_host.copy_(results, non_blocking=True)
                 stream.synchronize()
             e1.record(stream)
         ranks.barrier()
         nvtx.range_pop()
         e2e_ms = ranks.max(e0.elapsed_time(e1) / steps)
-        h2d = q_host.numel() * q_host.element_size() + lens_host.numel() * lens_host.element_size()
-        d2h = rel_host.numel() * rel_host.element_size() + com_host.numel() * com_host.element_size()
+        h2d = in_host.numel()
+        d2h = out_host.numel()
         e2e = {"value": job_throughput(kv_bytes, ranks.world, e2e_ms), "unit": "GB/s",
                "us_per_step": e2e_ms * 1e3, "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h),
-               "what": "per step: pinned host-to-device copy of every layer's q and seq_lens, "
-                       "the step's graph, device-to-host read of every layer's rel_l2 and "
-                       "commit flag, then a host synchronize; O_spec and O_exact stay on the "
-                       "device, where the post-attention ops that consume them run"}
+               "what": "per step: one pinned host-to-device copy of every layer's q and "
+                       "seq_lens, the step's graph, one device-to-host read of every layer's "
+                       "rel_l2 and commit flag, then a host synchronize; O_spec and O_exact "
+                       "stay on the device, where the post-attention ops that consume them run"}
 
     for g in [warm_graph] + graphs + prof_graphs + lat:
         sfd.alspec_graph_destroy(g)

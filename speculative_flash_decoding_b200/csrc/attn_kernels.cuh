@@ -1097,11 +1097,6 @@ __device__ __forceinline__ void fill_stage(const Params& p, unsigned char* smem,
     }
 }
 
-// The producer warp: fill the stage ring with the tiles of the items this CTA
-// pulls, then send end markers.  The first item (`item0`, taken before the
-// CTA's init barrier) fills the untouched stages one tile per lane, so the
-// first copies leave within a few hundred cycles; lane 0 alone continues
-// with the rest, waiting for each stage to be released.
 // The ring's first fills on the tensor-core engine, by the producer warp:
 // lane l issues copy l % OPS (K or V, 64 columns) of stage l / OPS, so one
 // copy instruction of the warp issues stage 0's copies first, then stage
@@ -1151,6 +1146,13 @@ __device__ __forceinline__ void fill_fresh(const Params& p, unsigned char* smem,
     }
 }
 
+// The producer warp: fill the stage ring with the tiles of the items this CTA
+// pulls, then send end markers.  The first item (`item0`, taken before the
+// CTA's init barrier) fills the untouched stages from every lane (one copy
+// per lane on the tensor-core engine, fill_fresh; one tile per lane on the
+// CUDA-core engine), so the first copies leave within a few hundred cycles;
+// lane 0 alone continues with the rest, waiting for each stage to be
+// released.
 template <typename T, int D, int G, bool SPEC, bool MMA, bool FUSED>
 __device__ __forceinline__ void produce(const Params& p, unsigned char* smem, int4* meta,
                                         uint32_t* fill, uint64_t* full_bar, uint64_t* empty_bar,
