@@ -17,8 +17,11 @@ import os
 _PKG = os.path.dirname(os.path.abspath(__file__))
 # ALSPEC_LIBRARY=debug loads the bounds-checked build of the same sources
 # (libalspec_debug.so); the default is libalspec.so.
-_LIB_NAME = {"": "libalspec.so", "default": "libalspec.so",
-             "debug": "libalspec_debug.so"}[os.environ.get("ALSPEC_LIBRARY", "")]
+_LIBRARIES = {"": "libalspec.so", "default": "libalspec.so", "debug": "libalspec_debug.so"}
+if os.environ.get("ALSPEC_LIBRARY", "") not in _LIBRARIES:
+    raise ImportError("ALSPEC_LIBRARY must be unset, 'default' or 'debug', not "
+                      f"{os.environ['ALSPEC_LIBRARY']!r}")
+_LIB_NAME = _LIBRARIES[os.environ.get("ALSPEC_LIBRARY", "")]
 LIB_PATH = os.path.join(_PKG, _LIB_NAME)
 
 ALSPEC_OK = 0

@@ -52,6 +52,29 @@ def test_debug_library_exports_the_decode_surface():
     assert not hasattr(debug, "alspec_read_probe")
 
 
+@pytest.mark.parametrize("value,library", [("debug", "libalspec_debug.so"),
+                                           ("default", "libalspec.so"), ("", "libalspec.so")])
+def test_library_switch(value, library):
+    """ALSPEC_LIBRARY picks the library the binding loads; there is no
+    fallback to another one."""
+    import subprocess
+    import sys
+    env = dict(os.environ, ALSPEC_LIBRARY=value, PYTHONPATH=ROOT)
+    out = subprocess.run([sys.executable, "-c", "import speculative_flash_decoding_b200 as s; "
+                          "print(s.LIB_PATH)"], env=env, capture_output=True, text=True,
+                         check=True, timeout=120)
+    assert out.stdout.strip() == os.path.join(PKG, library)
+
+
+def test_library_switch_rejects_unknown_values():
+    import subprocess
+    import sys
+    env = dict(os.environ, ALSPEC_LIBRARY="cpu", PYTHONPATH=ROOT)
+    out = subprocess.run([sys.executable, "-c", "import speculative_flash_decoding_b200"],
+                         env=env, capture_output=True, text=True, timeout=120)
+    assert out.returncode != 0 and "ALSPEC_LIBRARY" in out.stderr
+
+
 def test_debug_bounds_bit_is_declared():
     text = open(HEADER).read()
     assert "#define ALSPEC_DEVERR_BOUNDS 0x4u" in text
